@@ -1,0 +1,263 @@
+/*
+ * sd_attn.h -- C interface of libsdattn.so: the attention and acceptance hot path of
+ * speculative decoding in video LLMs, as hand-written CUDA kernels for NVIDIA B200 (sm_100a).
+ *
+ * Sources, by page title and section (the pages give the method, not formulas or code):
+ *  [StD] "Sparse-to-Dense: A Free Lunch for Lossless Acceleration of Video Understanding in
+ *        LLMs" (gist.science, pt), technical summary:
+ *        - "Procedimento de Decodificacao": the sparse model drafts gamma tokens; the dense
+ *          model verifies them in parallel with one read of the full KV cache; the longest
+ *          matching prefix (n tokens) is accepted plus one extra bonus token.
+ *        - "Metodologia": the sparse draft attends only to the top-K KV entries.
+ *        - "Selecao de Cache KV": the top-K selection is per layer and per head.
+ *        - "Principais Contribuicoes": lossless, the output distribution is unchanged.
+ *  [SPW] "Sparrow: Text-Anchored Window Attention with Visual-Semantic Glimpsing for
+ *        Speculative Decoding in Video LLMs" (gist.science zh section 3.1 HSR-VATA; pt
+ *        section 3.A): hidden-state reuse (an FC over [text embedding ; reused target hidden
+ *        state]) and text-anchored window attention that drops the visual KV cache.
+ *
+ * Conventions shared by every call
+ *  - Every pointer argument is DEVICE memory owned by the caller unless stated otherwise;
+ *    descriptor structs themselves are read on the host during the call and may be freed
+ *    after it returns.  The library allocates no device memory and keeps no global state;
+ *    scratch memory ("workspace") is passed in by the caller, sized by the *_workspace_size
+ *    queries.  Calls on different streams with different workspaces may run concurrently.
+ *  - Calls are asynchronous and stream-ordered on `stream` (a cudaStream_t; NULL means the
+ *    legacy default stream).  No call synchronises the device.
+ *  - Host-side validation runs before anything is launched.  An invalid argument returns a
+ *    status != SD_OK and launches nothing.  A launch failure returns SD_ERR_CUDA.
+ *  - Problems only visible on the device (an out-of-range page index, a bad sparse index,
+ *    an out-of-range drafted token, a length exceeding a host hint) are OR-ed as
+ *    SD_DEVERR_* bits into the optional int32 flag `dev_err` (device memory, may be NULL);
+ *    the offending element is skipped, nothing is read or written out of bounds.
+ *  - Tensors are row-major.  bf16 tensors hold IEEE bfloat16 bit patterns.
+ */
+#ifndef SD_ATTN_H
+#define SD_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+/* Exported symbols keep default visibility even when the library is built hidden-by-default. */
+#if defined(__GNUC__)
+#define SD_API __attribute__((visibility("default")))
+#else
+#define SD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SD_OK = 0,
+    SD_ERR_INVALID_ARG = 1, /* a host-checkable argument is wrong; nothing launched */
+    SD_ERR_UNSUPPORTED = 2, /* valid, but not a supported configuration (dtype, head_dim) */
+    SD_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the size query returned */
+    SD_ERR_CUDA = 4         /* a CUDA launch or runtime call failed */
+} sd_status;
+
+typedef enum { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
+
+/* Attention kinds, for sd_attention_workspace_size. */
+typedef enum {
+    SD_ATTN_VERIFY = 0,
+    SD_ATTN_TEXT_ANCHORED = 1,
+    SD_ATTN_SPARSE = 2
+} sd_attn_kind;
+
+/* Device error bits (OR-ed into *dev_err). */
+#define SD_DEVERR_PAGE 1u     /* block_table entry outside [0, num_pages) */
+#define SD_DEVERR_INDEX 2u    /* sparse index not strictly ascending, or candidate range bad */
+#define SD_DEVERR_TOKEN 4u    /* drafted token outside [0, vocab) */
+#define SD_DEVERR_NUMERIC 8u  /* non-finite softmax statistics during sampling */
+#define SD_DEVERR_SHAPE 16u   /* a device length exceeds its host hint (rows, kv_len) */
+
+/*
+ * KV cache of a batch of independent sequences.  A multi-layer problem is a batch whose
+ * entries are layers (each entry has its own cache, found through stride_b or block_table).
+ * Each sequence holds kv_len[b] positions: the context (visual span, then text), then the
+ * positions appended for the current draft / verify step.
+ *
+ *  dtype      SD_F32 or SD_BF16; Q and O of the attention calls use the same type.
+ *  h_kv       KV heads; query head h uses KV head h / (h_q / h_kv).
+ *  head_dim   64 or 128.
+ *  k, v       base pointers (device).
+ *  Contiguous layout (page_size == 0): element (b, h, j, e) of K is at
+ *             k[b*stride_b + h*stride_h + j*stride_pos + e]; strides in elements, e contiguous.
+ *             stride_pos must equal head_dim (rows are dense); for the tensor-core verify path
+ *             the base must be 16-byte aligned and stride_h, stride_b multiples of 8 elements.
+ *  Paged layout (page_size == 16): page p holds [h_kv][16][head_dim] elements at
+ *             k + p*h_kv*16*head_dim; position j of sequence b lives in page
+ *             block_table[b*max_pages_per_seq + j/16] at slot j%16.  num_pages bounds entries.
+ *  kv_len     device int32 [batch].
+ */
+typedef struct {
+    int32_t dtype;
+    int32_t h_kv;
+    int32_t head_dim;
+    int32_t page_size;
+    const void *k;
+    const void *v;
+    int64_t stride_b;
+    int64_t stride_h;
+    int64_t stride_pos;
+    const int32_t *block_table;
+    int32_t max_pages_per_seq;
+    int32_t num_pages;
+    const int32_t *kv_len;
+} sd_kv_desc;
+
+/*
+ * Query rows.  Q (and the output O) are [total_rows][h_q][head_dim]; sequence b owns rows
+ * [q_start[b], q_start[b+1]) (device int32 [batch+1], q_start[0] == 0).  Its n_q rows are the
+ * LAST n_q positions of its cache (the caller appended their K/V before the call), so row i
+ * sees positions j <= kv_len - n_q + i (bottom-right aligned causal mask).
+ *
+ *  max_q_rows     host hint: an upper bound of q_start[b+1] - q_start[b] (sizes grid/workspace).
+ *  max_kv_len     host hint: an upper bound of kv_len[b] (sizes the split-KV decomposition).
+ *  softmax_scale  scale of q.k; 0 selects 1/sqrt(head_dim).
+ */
+typedef struct {
+    int32_t h_q;
+    int32_t max_q_rows;
+    int32_t max_kv_len;
+    float softmax_scale;
+    const int32_t *q_start;
+} sd_q_desc;
+
+/* Human-readable name of a status. */
+SD_API const char *sd_status_string(sd_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+SD_API int32_t sd_version(void);
+
+/*
+ * Workspace bytes an attention call of `kind` needs for these descriptors (host hints only;
+ * device arrays are not read).  A call may be given more.  *bytes may be 0.
+ */
+SD_API sd_status sd_attention_workspace_size(sd_attn_kind kind, const sd_q_desc *q,
+                                      const sd_kv_desc *kv, int32_t batch, size_t *bytes);
+
+/*
+ * Dense verification attention [StD "Procedimento de Decodificacao"]: the target scores the
+ * gamma+1 new positions of every sequence in one pass over its full cache.  For every row i
+ * of sequence b and query head h:
+ *     O = softmax(scale * q . k_j  over j <= kv_len[b] - n_q + i) . V
+ * computed as split-KV flash-decoding (each split keeps an online softmax; the splits are
+ * merged by their log-sum-exp).  q: [rows][h_q][d], out: [rows][h_q][d] (kv dtype).
+ * Tensor cores (tcgen05) serve bf16 when G*n_q >= 16 rows; CUDA cores otherwise.
+ */
+SD_API sd_status sd_verify_attention(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
+                              int32_t batch, void *out, void *workspace, size_t workspace_bytes,
+                              int32_t *dev_err, void *stream);
+
+/*
+ * Text-anchored window attention [SPW 3.1 / 3.A]: Sparrow's draft drops the visual KV cache
+ * and attends only inside a text-anchored window.  For row i of sequence b the allowed
+ * positions are the last window[b] positions j <= kv_len[b] - n_q + i that lie outside the
+ * visual span [vis_begin[b], vis_end[b]) (the window counts non-visual positions and ends at
+ * the row's own position; it may reach below the visual span).  vis_begin, vis_end, window:
+ * device int32 [batch]; window >= 1; vis_begin <= vis_end (else the span is taken as empty
+ * and SD_DEVERR_INDEX is set).  max_window: host hint >= every window[b].
+ * A row with no allowed position outputs zeros.
+ */
+SD_API sd_status sd_text_anchored_attention(const sd_q_desc *q, const void *q_data,
+                                     const sd_kv_desc *kv, int32_t batch,
+                                     const int32_t *vis_begin, const int32_t *vis_end,
+                                     const int32_t *window, int32_t max_window, void *out,
+                                     void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                                     void *stream);
+
+/*
+ * Sparse draft attention [StD "Metodologia"]: the sparse model attends only to the selected
+ * top-K KV entries plus the dense tail.  For row i of sequence b and KV head g the allowed
+ * set is ({idx[b][g][0..k)} U [tail_begin[b], limit]) restricted to j <= limit,
+ * limit = kv_len[b] - n_q + i.  idx: device int32 [batch][h_kv][k], ascending; negative
+ * entries are padding and ignored; entries >= tail_begin are covered by the tail; a
+ * non-ascending list sets SD_DEVERR_INDEX and repeated entries are skipped.
+ * tail_begin: device int32 [batch].  max_tail: host hint >= kv_len[b] - tail_begin[b].
+ */
+SD_API sd_status sd_sparse_attention(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
+                              int32_t batch, const int32_t *idx, int32_t k,
+                              const int32_t *tail_begin, int32_t max_tail, void *out,
+                              void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                              void *stream);
+
+/*
+ * Workspace for sd_topk_select.  max_cand: host hint >= cand_end[b] - cand_begin[b].
+ */
+SD_API sd_status sd_topk_workspace_size(const sd_kv_desc *kv, int32_t batch, int32_t max_cand,
+                                 int32_t k, size_t *bytes);
+
+/*
+ * Top-K KV selection [StD "Selecao de Cache KV": top-K KV entries per layer and per head].
+ * For sequence b and KV head g, candidate j in [cand_begin[b], cand_end[b]) scores
+ *     s_j = sum over the group's query heads h of  q_last[h] . k_j
+ * where q_last is the LAST query row of the sequence (row q_start[b+1]-1 of q_data).  The
+ * scale 1/sqrt(d) changes no rank and is not applied.  Scores are accumulated in fp64.  The k
+ * highest scores are selected, equal scores going to the lower position, and written in
+ * ascending position order to idx_out [batch][h_kv][k] (device int32); when fewer than k
+ * candidates exist all of them are written and the rest is -1.
+ */
+SD_API sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
+                         int32_t batch, const int32_t *cand_begin, const int32_t *cand_end,
+                         int32_t max_cand, int32_t k, int32_t *idx_out, void *workspace,
+                         size_t workspace_bytes, int32_t *dev_err, void *stream);
+
+/*
+ * Hidden-state reuse projection [SPW 3.1]: the draft input is an FC over the concatenation
+ * of the current text embedding and the reused target hidden state:
+ *     y[r][o] = sum_i W[o][i] emb[r][i] + sum_i W[o][d_model+i] hid[r][i] (+ bias[o])
+ * emb, hid: [n_rows][d_model]; W: [d_model][2*d_model] (out x in); bias: [d_model] or NULL;
+ * y: [n_rows][d_model].  All bf16; fp32 accumulation.  The concatenation is never
+ * materialised.  1 <= n_rows <= 16; d_model a multiple of 8; pointers 16-byte aligned.
+ */
+SD_API sd_status sd_hsr_project(const void *emb, const void *hid, int32_t n_rows, int32_t d_model,
+                         const void *weight, const void *bias, void *y, void *stream);
+
+/*
+ * Workspace for sd_accept_greedy / sd_accept_sample.  max_gamma: host hint >= gamma[b].
+ */
+SD_API sd_status sd_accept_workspace_size(int32_t batch, int32_t max_gamma, int32_t vocab,
+                                   size_t *bytes);
+
+/*
+ * Greedy acceptance [StD "Procedimento de Decodificacao"].  Sequence b has gamma[b] drafted
+ * tokens and gamma[b]+1 target rows; rows and tokens are packed over the batch:
+ * tgt_logits [sum(gamma+1)][vocab] fp32, draft_tok [sum(gamma)] int32, gamma [batch] int32
+ * (all device).  t_i = argmax of target row i (equal values: lowest id; NaN ranks lowest);
+ * n = the longest prefix with draft_tok_{i} == t_i; the output row b of out_tok
+ * [batch][out_stride] receives d_1..d_n followed by the bonus t_n (n+1 tokens) and
+ * n_acc[b] = n.  out_stride >= max_gamma + 1.
+ */
+SD_API sd_status sd_accept_greedy(const float *tgt_logits, const int32_t *draft_tok,
+                           const int32_t *gamma, int32_t batch, int32_t max_gamma, int32_t vocab,
+                           int32_t *n_acc, int32_t *out_tok, int32_t out_stride, void *workspace,
+                           size_t workspace_bytes, int32_t *dev_err, void *stream);
+
+/*
+ * Speculative-sampling acceptance with residual resampling [StD "Principais Contribuicoes":
+ * lossless].  p_i = softmax(target row i), q_i = softmax(draft row i) (temperature 1).
+ * For i = 1..gamma the drafted d_i is accepted iff u_i <= p_{i-1}(d_i) / q_{i-1}(d_i); at the
+ * first rejection (n accepted) a token is drawn from norm(max(0, p_n - q_n)) with v_n (from p_n
+ * if that residual is all zero); after gamma acceptances the bonus is drawn from p_gamma with
+ * v_gamma.  A draw from weights w with uniform v is the smallest x with
+ * sum_{y<=x} w_y > v * sum_y w_y.
+ * draft_logits [sum(gamma)][vocab] fp32; u [sum(gamma)] fp32; v [sum(gamma+1)] fp32 (caller
+ * supplied uniforms in [0,1), so the kernels hold no RNG state).  Softmax statistics use fp32
+ * per element and fp64 for the per-row totals and the accept ratio.  near_boundary (device
+ * int32 [batch], may be NULL) receives the number of decisions of that sequence whose
+ * |u - ratio| < 1e-6 or whose draw fell within 1e-6*Z of a CDF edge.
+ */
+SD_API sd_status sd_accept_sample(const float *tgt_logits, const float *draft_logits,
+                           const int32_t *draft_tok, const float *u, const float *v,
+                           const int32_t *gamma, int32_t batch, int32_t max_gamma, int32_t vocab,
+                           int32_t *n_acc, int32_t *out_tok, int32_t out_stride,
+                           int32_t *near_boundary, void *workspace, size_t workspace_bytes,
+                           int32_t *dev_err, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SD_ATTN_H */

@@ -1,0 +1,382 @@
+// C-ABI entry points of libsdattn: host-side validation, decomposition and dispatch.
+// Every check here runs before any launch; on failure nothing is launched.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "sd_internal.h"
+
+namespace sd {
+
+int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();  // clear the sticky-free error of a failed query
+        return 148;
+    }
+    return n;
+}
+
+AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, int batch,
+                        int max_q_rows, long long max_stream) {
+    AttnPlan plan{};
+    const int G = h_q / h_kv;
+    const int rows = G * max_q_rows;
+    const int sms = device_sm_count();
+    const size_t rows_cap = (size_t)batch * max_q_rows;
+    if (max_stream < 1) max_stream = 1;
+    plan.tensor_core = tc_supported(kind, dtype, head_dim, rows);
+    if (plan.tensor_core) {
+        plan.rows_per_block = 128;
+        plan.n_rowblocks = 1;
+        const long long units = (long long)batch * h_kv;
+        const long long tiles = (max_stream + 127) / 128;
+        // one CTA per SM: aim for about two waves of position chunks of >= 4 tiles
+        long long splits = (2LL * sms + units - 1) / units;
+        long long by_len = (tiles + 3) / 4;
+        if (splits > by_len) splits = by_len;
+        if (splits < 1) splits = 1;
+        if (splits > 512) splits = 512;
+        plan.n_splits = (int)splits;
+    } else {
+        plan.rows_per_block = rows <= 8 ? 8 : 16;
+        plan.n_rowblocks = (rows + plan.rows_per_block - 1) / plan.rows_per_block;
+        const long long units = (long long)batch * h_kv * plan.n_rowblocks;
+        long long splits = (8LL * sms + units - 1) / units;
+        long long by_len = (max_stream + 255) / 256;
+        if (splits > by_len) splits = by_len;
+        if (splits < 1) splits = 1;
+        if (splits > 512) splits = 512;
+        plan.n_splits = (int)splits;
+    }
+    plan.ws_bytes = plan.n_splits > 1
+                        ? (size_t)plan.n_splits * rows_cap * h_q * (head_dim + 2) * sizeof(float)
+                        : 0;
+    return plan;
+}
+
+}  // namespace sd
+
+using namespace sd;
+
+namespace {
+
+bool kv_desc_ok(const sd_kv_desc *kv, int batch) {
+    if (!kv || batch < 1) return false;
+    if (kv->dtype != SD_F32 && kv->dtype != SD_BF16) return false;
+    if (kv->h_kv < 1 || !kv->k || !kv->v || !kv->kv_len) return false;
+    const int esz = kv->dtype == SD_BF16 ? 2 : 4;
+    if ((reinterpret_cast<uintptr_t>(kv->k) | reinterpret_cast<uintptr_t>(kv->v)) & 15) return false;
+    if (kv->page_size == 0) {
+        if (kv->stride_pos != kv->head_dim) return false;
+        if (kv->stride_h < 0 || kv->stride_b < 0) return false;
+        if (((kv->stride_h * esz) & 15) || ((kv->stride_b * esz) & 15)) return false;
+    } else {
+        if (kv->page_size != kPageSize) return false;
+        if (!kv->block_table || kv->max_pages_per_seq < 1 || kv->num_pages < 1) return false;
+    }
+    return true;
+}
+
+bool head_dim_supported(int d) { return d == 64 || d == 128; }
+
+KVView make_view(const sd_kv_desc *kv) {
+    KVView v;
+    v.dtype = kv->dtype;
+    v.h_kv = kv->h_kv;
+    v.head_dim = kv->head_dim;
+    v.page_size = kv->page_size;
+    v.k = kv->k;
+    v.v = kv->v;
+    v.stride_b = kv->stride_b;
+    v.stride_h = kv->stride_h;
+    v.stride_pos = kv->stride_pos;
+    v.block_table = kv->block_table;
+    v.max_pages = kv->max_pages_per_seq;
+    v.num_pages = kv->num_pages;
+    v.kv_len = kv->kv_len;
+    return v;
+}
+
+sd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SD_OK : SD_ERR_CUDA; }
+
+// Common validation of the attention calls; fills the plan for the kind.
+sd_status check_attention(sd_attn_kind kind, const sd_q_desc *q, const sd_kv_desc *kv, int batch,
+                          long long max_stream, AttnPlan *plan) {
+    if (!q || !kv || batch < 1 || batch > 65535) return SD_ERR_INVALID_ARG;
+    if (!kv_desc_ok(kv, batch)) return SD_ERR_INVALID_ARG;
+    if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
+    if (q->h_q < 1 || q->h_q % kv->h_kv != 0 || q->max_q_rows < 1 || q->max_kv_len < 1 ||
+        !q->q_start || !(q->softmax_scale >= 0.f) || isinf(q->softmax_scale))
+        return SD_ERR_INVALID_ARG;
+    if ((long long)batch * q->max_q_rows > (1LL << 30)) return SD_ERR_INVALID_ARG;
+    *plan = plan_attention(kind, kv->dtype, kv->head_dim, q->h_q, kv->h_kv, batch, q->max_q_rows,
+                           max_stream);
+    return SD_OK;
+}
+
+AttnParams base_params(sd_attn_kind kind, const sd_q_desc *q, const void *q_data,
+                       const sd_kv_desc *kv, int batch, void *out, const AttnPlan &plan,
+                       void *ws, int32_t *dev_err) {
+    AttnParams p{};
+    p.kind = kind;
+    p.kv = make_view(kv);
+    p.batch = batch;
+    p.h_q = q->h_q;
+    p.group = q->h_q / kv->h_kv;
+    p.max_q_rows = q->max_q_rows;
+    p.rows_cap = batch * q->max_q_rows;
+    const float scale = q->softmax_scale > 0.f ? q->softmax_scale
+                                               : (float)(1.0 / sqrt((double)kv->head_dim));
+    p.scale_log2 = scale * kLog2e;
+    p.q = q_data;
+    p.q_start = q->q_start;
+    p.out = out;
+    p.n_splits = plan.n_splits;
+    p.n_rowblocks = plan.n_rowblocks;
+    p.ws_o = reinterpret_cast<float *>(ws);
+    p.ws_ml = plan.n_splits > 1
+                  ? p.ws_o + (size_t)plan.n_splits * p.rows_cap * q->h_q * kv->head_dim
+                  : nullptr;
+    p.dev_err = dev_err;
+    return p;
+}
+
+sd_status run_attention(const AttnParams &p, const AttnPlan &plan, void *stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = plan.tensor_core ? launch_attention_tc(p, plan, s)
+                                     : launch_attention_simt(p, plan, s);
+    if (e != cudaSuccess) return SD_ERR_CUDA;
+    if (plan.n_splits > 1) e = launch_attention_merge(p, s);
+    return cuda_status(e);
+}
+
+long long stream_hint(sd_attn_kind kind, const sd_q_desc *q, long long extra) {
+    if (kind == SD_ATTN_TEXT_ANCHORED) {
+        const long long w = extra + q->max_q_rows - 1;
+        return w < q->max_kv_len ? w : q->max_kv_len;
+    }
+    if (kind == SD_ATTN_SPARSE) {
+        const long long w = extra;
+        return w < q->max_kv_len ? w : q->max_kv_len;
+    }
+    return q->max_kv_len;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sd_status_string(sd_status s) {
+    switch (s) {
+        case SD_OK: return "SD_OK";
+        case SD_ERR_INVALID_ARG: return "SD_ERR_INVALID_ARG: invalid argument";
+        case SD_ERR_UNSUPPORTED: return "SD_ERR_UNSUPPORTED: unsupported configuration";
+        case SD_ERR_WORKSPACE: return "SD_ERR_WORKSPACE: workspace missing or too small";
+        case SD_ERR_CUDA: return "SD_ERR_CUDA: CUDA launch or runtime error";
+    }
+    return "unknown sd_status";
+}
+
+int32_t sd_version(void) { return 100; }
+
+sd_status sd_attention_workspace_size(sd_attn_kind kind, const sd_q_desc *q,
+                                      const sd_kv_desc *kv, int32_t batch, size_t *bytes) {
+    if (!bytes || !q || !kv) return SD_ERR_INVALID_ARG;
+    if (kind != SD_ATTN_VERIFY && kind != SD_ATTN_TEXT_ANCHORED && kind != SD_ATTN_SPARSE)
+        return SD_ERR_INVALID_ARG;
+    if (kv->h_kv < 1 || q->h_q < 1 || q->h_q % kv->h_kv || batch < 1 || q->max_q_rows < 1)
+        return SD_ERR_INVALID_ARG;
+    if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
+    // Worst-case stream for the kind (hints of the specific call are not known here).
+    const AttnPlan plan = plan_attention(kind, kv->dtype, kv->head_dim, q->h_q, kv->h_kv, batch,
+                                         q->max_q_rows, q->max_kv_len);
+    *bytes = plan.ws_bytes;
+    return SD_OK;
+}
+
+sd_status sd_verify_attention(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
+                              int32_t batch, void *out, void *workspace, size_t workspace_bytes,
+                              int32_t *dev_err, void *stream) {
+    AttnPlan plan;
+    if (!q_data || !out) return SD_ERR_INVALID_ARG;
+    sd_status st = check_attention(SD_ATTN_VERIFY, q, kv, batch, q ? q->max_kv_len : 0, &plan);
+    if (st != SD_OK) return st;
+    if (plan.ws_bytes > workspace_bytes || (plan.ws_bytes && !workspace)) return SD_ERR_WORKSPACE;
+    AttnParams p = base_params(SD_ATTN_VERIFY, q, q_data, kv, batch, out, plan, workspace, dev_err);
+    return run_attention(p, plan, stream);
+}
+
+sd_status sd_text_anchored_attention(const sd_q_desc *q, const void *q_data,
+                                     const sd_kv_desc *kv, int32_t batch,
+                                     const int32_t *vis_begin, const int32_t *vis_end,
+                                     const int32_t *window, int32_t max_window, void *out,
+                                     void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                                     void *stream) {
+    if (!q_data || !out || !vis_begin || !vis_end || !window || max_window < 1)
+        return SD_ERR_INVALID_ARG;
+    AttnPlan plan;
+    if (!q) return SD_ERR_INVALID_ARG;
+    sd_status st = check_attention(SD_ATTN_TEXT_ANCHORED, q, kv, batch,
+                                   stream_hint(SD_ATTN_TEXT_ANCHORED, q, max_window), &plan);
+    if (st != SD_OK) return st;
+    if (plan.ws_bytes > workspace_bytes || (plan.ws_bytes && !workspace)) return SD_ERR_WORKSPACE;
+    AttnParams p = base_params(SD_ATTN_TEXT_ANCHORED, q, q_data, kv, batch, out, plan, workspace,
+                               dev_err);
+    p.vis_begin = vis_begin;
+    p.vis_end = vis_end;
+    p.window = window;
+    return run_attention(p, plan, stream);
+}
+
+sd_status sd_sparse_attention(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
+                              int32_t batch, const int32_t *idx, int32_t k,
+                              const int32_t *tail_begin, int32_t max_tail, void *out,
+                              void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                              void *stream) {
+    if (!q_data || !out || !tail_begin || k < 0 || (k > 0 && !idx) || max_tail < 0 ||
+        k > (1 << 16))
+        return SD_ERR_INVALID_ARG;
+    AttnPlan plan;
+    if (!q) return SD_ERR_INVALID_ARG;
+    sd_status st = check_attention(SD_ATTN_SPARSE, q, kv, batch,
+                                   stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail), &plan);
+    if (st != SD_OK) return st;
+    if (plan.tensor_core) {  // the sparse gather always runs on the CUDA-core engine
+        const int rows = (q->h_q / kv->h_kv) * q->max_q_rows;
+        plan.tensor_core = false;
+        plan.rows_per_block = rows <= 8 ? 8 : 16;
+        plan.n_rowblocks = (rows + plan.rows_per_block - 1) / plan.rows_per_block;
+    }
+    if (plan.ws_bytes > workspace_bytes || (plan.ws_bytes && !workspace)) return SD_ERR_WORKSPACE;
+    AttnParams p = base_params(SD_ATTN_SPARSE, q, q_data, kv, batch, out, plan, workspace, dev_err);
+    p.idx = idx;
+    p.k_sel = k;
+    p.tail_begin = tail_begin;
+    return run_attention(p, plan, stream);
+}
+
+sd_status sd_topk_workspace_size(const sd_kv_desc *kv, int32_t batch, int32_t max_cand,
+                                 int32_t k, size_t *bytes) {
+    if (!kv || !bytes || batch < 1 || max_cand < 0 || k < 1 || kv->h_kv < 1)
+        return SD_ERR_INVALID_ARG;
+    *bytes = topk_workspace_bytes(batch, kv->h_kv, max_cand);
+    return SD_OK;
+}
+
+sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
+                         int32_t batch, const int32_t *cand_begin, const int32_t *cand_end,
+                         int32_t max_cand, int32_t k, int32_t *idx_out, void *workspace,
+                         size_t workspace_bytes, int32_t *dev_err, void *stream) {
+    if (!q || !q_data || !cand_begin || !cand_end || !idx_out || k < 1 || max_cand < 0 ||
+        batch > 65535)
+        return SD_ERR_INVALID_ARG;
+    if (!kv_desc_ok(kv, batch)) return SD_ERR_INVALID_ARG;
+    if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
+    if (q->h_q < 1 || q->h_q % kv->h_kv != 0 || !q->q_start) return SD_ERR_INVALID_ARG;
+    const size_t need = topk_workspace_bytes(batch, kv->h_kv, max_cand);
+    if (need > workspace_bytes || (need && !workspace)) return SD_ERR_WORKSPACE;
+    TopkParams p{};
+    p.kv = make_view(kv);
+    p.batch = batch;
+    p.h_q = q->h_q;
+    p.group = q->h_q / kv->h_kv;
+    p.q = q_data;
+    p.q_start = q->q_start;
+    p.cand_begin = cand_begin;
+    p.cand_end = cand_end;
+    p.max_cand = max_cand;
+    p.k = k;
+    p.idx_out = idx_out;
+    p.keys = reinterpret_cast<unsigned long long *>(workspace);
+    p.dev_err = dev_err;
+    const int sms = device_sm_count();
+    const long long units = (long long)batch * kv->h_kv;
+    long long splits = (4LL * sms + units - 1) / units;
+    const long long by_len = ((long long)max_cand + 1023) / 1024;
+    if (splits > by_len) splits = by_len;
+    if (splits < 1) splits = 1;
+    if (splits > 1024) splits = 1024;
+    p.n_splits = (int)splits;
+    return cuda_status(launch_topk(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sd_status sd_hsr_project(const void *emb, const void *hid, int32_t n_rows, int32_t d_model,
+                         const void *weight, const void *bias, void *y, void *stream) {
+    if (!emb || !hid || !weight || !y || n_rows < 1 || n_rows > 16 || d_model < 8 ||
+        d_model % 8 != 0 || d_model > (1 << 20))
+        return SD_ERR_INVALID_ARG;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(emb) | reinterpret_cast<uintptr_t>(hid) |
+                        reinterpret_cast<uintptr_t>(weight);
+    if (a & 15) return SD_ERR_INVALID_ARG;
+    if ((size_t)4 * 2 * d_model * 2 > 200 * 1024) return SD_ERR_UNSUPPORTED;
+    return cuda_status(launch_hsr(emb, hid, n_rows, d_model, weight, bias, y,
+                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sd_status sd_accept_workspace_size(int32_t batch, int32_t max_gamma, int32_t vocab,
+                                   size_t *bytes) {
+    if (!bytes || batch < 1 || max_gamma < 0 || vocab < 1) return SD_ERR_INVALID_ARG;
+    *bytes = accept_workspace_bytes(batch, max_gamma, vocab, nullptr);
+    return SD_OK;
+}
+
+static sd_status accept_common(const float *tgt, const int32_t *draft_tok, const int32_t *gamma,
+                               int32_t batch, int32_t max_gamma, int32_t vocab, int32_t *n_acc,
+                               int32_t *out_tok, int32_t out_stride, void *workspace,
+                               size_t workspace_bytes, AcceptParams *p) {
+    if (!tgt || !gamma || !n_acc || !out_tok || batch < 1 || batch > 65535 || max_gamma < 0 ||
+        vocab < 1 || out_stride < max_gamma + 1 || (max_gamma > 0 && !draft_tok))
+        return SD_ERR_INVALID_ARG;
+    if ((long long)batch * (2 * max_gamma + 1) > 65535) return SD_ERR_UNSUPPORTED;
+    int n_chunks = 1;
+    const size_t need = accept_workspace_bytes(batch, max_gamma, vocab, &n_chunks);
+    if (need > workspace_bytes || !workspace) return SD_ERR_WORKSPACE;
+    *p = AcceptParams{};
+    p->tgt = tgt;
+    p->draft_tok = draft_tok;
+    p->gamma = gamma;
+    p->batch = batch;
+    p->max_gamma = max_gamma;
+    p->vocab = vocab;
+    p->n_acc = n_acc;
+    p->out_tok = out_tok;
+    p->out_stride = out_stride;
+    p->n_chunks = n_chunks;
+    p->ws = workspace;
+    return SD_OK;
+}
+
+sd_status sd_accept_greedy(const float *tgt_logits, const int32_t *draft_tok,
+                           const int32_t *gamma, int32_t batch, int32_t max_gamma, int32_t vocab,
+                           int32_t *n_acc, int32_t *out_tok, int32_t out_stride, void *workspace,
+                           size_t workspace_bytes, int32_t *dev_err, void *stream) {
+    AcceptParams p;
+    sd_status st = accept_common(tgt_logits, draft_tok, gamma, batch, max_gamma, vocab, n_acc,
+                                 out_tok, out_stride, workspace, workspace_bytes, &p);
+    if (st != SD_OK) return st;
+    p.dev_err = dev_err;
+    return cuda_status(launch_accept_greedy(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sd_status sd_accept_sample(const float *tgt_logits, const float *draft_logits,
+                           const int32_t *draft_tok, const float *u, const float *v,
+                           const int32_t *gamma, int32_t batch, int32_t max_gamma, int32_t vocab,
+                           int32_t *n_acc, int32_t *out_tok, int32_t out_stride,
+                           int32_t *near_boundary, void *workspace, size_t workspace_bytes,
+                           int32_t *dev_err, void *stream) {
+    if (!v || (max_gamma > 0 && (!draft_logits || !u))) return SD_ERR_INVALID_ARG;
+    AcceptParams p;
+    sd_status st = accept_common(tgt_logits, draft_tok, gamma, batch, max_gamma, vocab, n_acc,
+                                 out_tok, out_stride, workspace, workspace_bytes, &p);
+    if (st != SD_OK) return st;
+    p.drf = draft_logits;
+    p.u = u;
+    p.v = v;
+    p.near_boundary = near_boundary;
+    p.dev_err = dev_err;
+    return cuda_status(launch_accept_sample(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,107 @@
+// Internal interfaces between the C-ABI layer (sd_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sd_attn.h"
+#include "sd_common.cuh"
+
+namespace sd {
+
+// Parameters of one attention launch (all three kinds).
+struct AttnParams {
+    int kind;  // sd_attn_kind
+    KVView kv;
+    int batch;
+    int h_q;
+    int group;       // h_q / h_kv
+    int max_q_rows;  // host hint
+    int rows_cap;    // batch * max_q_rows: rows addressable in the split workspace
+    float scale_log2;  // softmax_scale * log2(e)
+    const void *q;
+    const int32_t *q_start;
+    void *out;
+    // text-anchored
+    const int32_t *vis_begin;
+    const int32_t *vis_end;
+    const int32_t *window;
+    // sparse
+    const int32_t *idx;
+    int k_sel;
+    const int32_t *tail_begin;
+    // split-KV decomposition
+    int n_splits;
+    int n_rowblocks;
+    float *ws_o;   // [n_splits][rows_cap][h_q][head_dim] unnormalised partial outputs
+    float *ws_ml;  // [n_splits][rows_cap][h_q][2] (running max in log2 units, sum)
+    int32_t *dev_err;
+};
+
+// Decomposition chosen for an attention call (host side; depends on host hints only).
+struct AttnPlan {
+    bool tensor_core;  // tcgen05 path
+    int n_splits;
+    int n_rowblocks;
+    int rows_per_block;
+    size_t ws_bytes;
+};
+
+int device_sm_count();
+AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, int batch,
+                        int max_q_rows, long long max_stream);
+
+cudaError_t launch_attention_simt(const AttnParams &p, const AttnPlan &plan, cudaStream_t s);
+cudaError_t launch_attention_tc(const AttnParams &p, const AttnPlan &plan, cudaStream_t s);
+cudaError_t launch_attention_merge(const AttnParams &p, cudaStream_t s);
+bool tc_supported(int kind, int dtype, int head_dim, int rows);
+
+// Top-K.
+struct TopkParams {
+    KVView kv;
+    int batch;
+    int h_q;
+    int group;
+    const void *q;
+    const int32_t *q_start;
+    const int32_t *cand_begin;
+    const int32_t *cand_end;
+    int max_cand;
+    int k;
+    int32_t *idx_out;
+    int n_splits;
+    unsigned long long *keys;  // [batch][h_kv][max_cand] order-preserving score keys
+    int32_t *dev_err;
+};
+size_t topk_workspace_bytes(int batch, int h_kv, int max_cand);
+cudaError_t launch_topk(const TopkParams &p, cudaStream_t s);
+
+// HSR projection.
+cudaError_t launch_hsr(const void *emb, const void *hid, int n_rows, int d_model, const void *w,
+                       const void *bias, void *y, cudaStream_t s);
+
+// Acceptance.
+struct AcceptParams {
+    const float *tgt;
+    const float *drf;
+    const int32_t *draft_tok;
+    const float *u;
+    const float *v;
+    const int32_t *gamma;
+    int batch;
+    int max_gamma;
+    int vocab;
+    int32_t *n_acc;
+    int32_t *out_tok;
+    int out_stride;
+    int32_t *near_boundary;
+    int n_chunks;  // vocabulary chunks per row
+    void *ws;
+    int32_t *dev_err;
+};
+size_t accept_workspace_bytes(int batch, int max_gamma, int vocab, int *n_chunks);
+cudaError_t launch_accept_greedy(const AcceptParams &p, cudaStream_t s);
+cudaError_t launch_accept_sample(const AcceptParams &p, cudaStream_t s);
+
+}  // namespace sd

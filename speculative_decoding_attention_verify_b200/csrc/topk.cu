@@ -1,0 +1,214 @@
+// Top-K KV selection per (sequence, KV head).
+//
+// 1. topk_score_kernel: grid (splits, KV heads, sequences).  The group's last query rows are
+//    summed once in fp64 (qbar); every candidate key row is streamed with 16-byte loads and
+//    dotted with qbar in fp64 (bf16 x bf16 products are exact in fp64, and the sum of the
+//    group's dot products equals qbar . k up to fp64 rounding).  The score is stored as an
+//    order-preserving 64-bit key (larger score -> larger key; -0 == +0; NaN lowest).
+// 2. topk_select_kernel: one CTA per (sequence, KV head).  An MSB-first radix select (eight
+//    8-bit digits, shared-memory histograms) finds the k-th largest key T exactly; then one
+//    pass in position order keeps every key > T and the first (k - #greater) keys == T, so
+//    equal scores go to the lower position, and block-wide prefix sums write the kept
+//    positions in ascending order.
+#include "sd_internal.h"
+
+namespace sd {
+namespace {
+
+constexpr int kScoreThreads = 256;
+constexpr int kSelectThreads = 1024;
+
+__device__ __forceinline__ unsigned long long score_key(double x) {
+    if (x != x) return 0ull;  // NaN ranks lowest
+    x += 0.0;                 // -0 -> +0
+    unsigned long long u = (unsigned long long)__double_as_longlong(x);
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// Clamp the candidate range of sequence b to [0, kv_len) and to max_cand entries.
+__device__ __forceinline__ void cand_range(const TopkParams &p, int b, int &cb, int &n) {
+    const int kv_len = __ldg(p.kv.kv_len + b);
+    int lo = __ldg(p.cand_begin + b), hi = __ldg(p.cand_end + b);
+    const bool bad = lo < 0 || hi > kv_len || hi - lo > p.max_cand ||
+                     (p.kv.page_size != 0 && kv_len > p.kv.max_pages * kPageSize);
+    lo = max(lo, 0);
+    hi = min(hi, kv_len);
+    if (p.kv.page_size != 0) hi = min(hi, p.kv.max_pages * kPageSize);
+    hi = min(hi, lo + p.max_cand);
+    cb = lo;
+    n = max(0, hi - lo);
+    if (bad && threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
+}
+
+template <bool BF16, int D>
+__global__ void __launch_bounds__(kScoreThreads) topk_score_kernel(const TopkParams p) {
+    using CH = Chunk<BF16>;
+    constexpr int ESZ = BF16 ? 2 : 4;
+    constexpr int NCHUNK = D * ESZ / 16;
+    __shared__ double s_qbar[D];
+    const int b = blockIdx.z, g = blockIdx.y, split = blockIdx.x;
+    const int last = __ldg(p.q_start + b + 1) - 1;
+    if (last < __ldg(p.q_start + b)) {
+        if (threadIdx.x == 0 && split == 0) set_dev_err(p.dev_err, SD_DEVERR_SHAPE);
+        return;
+    }
+    int cb, n;
+    cand_range(p, b, cb, n);
+    if (threadIdx.x < D) {
+        double acc = 0.0;
+        for (int h = g * p.group; h < (g + 1) * p.group; ++h) {
+            const int64_t off = ((int64_t)last * p.h_q + h) * D + threadIdx.x;
+            const float qf = BF16 ? __uint_as_float((uint32_t)__ldg(
+                                        reinterpret_cast<const unsigned short *>(p.q) + off) << 16)
+                                  : __ldg(reinterpret_cast<const float *>(p.q) + off);
+            acc += (double)qf;
+        }
+        s_qbar[threadIdx.x] = acc;
+    }
+    __syncthreads();
+    unsigned long long *keys = p.keys + ((int64_t)b * p.kv.h_kv + g) * p.max_cand;
+    const int t_begin = (int)((int64_t)n * split / p.n_splits);
+    const int t_end = (int)((int64_t)n * (split + 1) / p.n_splits);
+    for (int t = t_begin + threadIdx.x; t < t_end; t += kScoreThreads) {
+        const int64_t off = kv_row_offset(p.kv, b, g, cb + t, p.dev_err);
+        unsigned long long key = 0ull;
+        if (off >= 0) {
+            const char *row = reinterpret_cast<const char *>(p.kv.k) + off * ESZ;
+            double acc = 0.0;
+#pragma unroll
+            for (int c = 0; c < NCHUNK; c += 4) {
+                uint4 raw[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) raw[u] = ldg_stream16(row + (c + u) * 16);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float f[CH::kElems];
+                    CH::to_float(raw[u], f);
+#pragma unroll
+                    for (int e = 0; e < CH::kElems; ++e)
+                        acc = fma((double)f[e], s_qbar[(c + u) * CH::kElems + e], acc);
+                }
+            }
+            key = score_key(acc);
+        }
+        keys[t] = key;
+    }
+}
+
+// Inclusive block-wide prefix sum of one int per thread (kSelectThreads threads).
+__device__ __forceinline__ int block_inclusive_scan(int x, int *s_warp, int &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = s_warp[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        s_warp[lane] = w;
+    }
+    __syncthreads();
+    const int before = warp > 0 ? s_warp[warp - 1] : 0;
+    total = s_warp[31];
+    __syncthreads();
+    return x + before;
+}
+
+__global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(const TopkParams p) {
+    __shared__ int s_hist[256];
+    __shared__ int s_warp[32];
+    __shared__ unsigned long long s_prefix;
+    __shared__ int s_remaining;
+    const int b = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
+    int32_t *out = p.idx_out + ((int64_t)b * p.kv.h_kv + g) * p.k;
+    const int last = __ldg(p.q_start + b + 1) - 1;
+    if (last < __ldg(p.q_start + b)) {
+        for (int e = tid; e < p.k; e += kSelectThreads) out[e] = -1;
+        return;
+    }
+    int cb, n;
+    cand_range(p, b, cb, n);
+    const unsigned long long *keys = p.keys + ((int64_t)b * p.kv.h_kv + g) * p.max_cand;
+    if (n <= p.k) {  // everything is selected
+        for (int e = tid; e < p.k; e += kSelectThreads) out[e] = e < n ? cb + e : -1;
+        return;
+    }
+    // ---- radix select of the k-th largest key ----
+    unsigned long long prefix = 0ull, mask = 0ull;
+    int remaining = p.k;
+    for (int digit = 7; digit >= 0; --digit) {
+        const int shift = digit * 8;
+        if (tid < 256) s_hist[tid] = 0;
+        __syncthreads();
+        for (int t = tid; t < n; t += kSelectThreads) {
+            const unsigned long long key = keys[t];
+            if ((key & mask) == prefix) atomicAdd(&s_hist[(int)((key >> shift) & 255ull)], 1);
+        }
+        __syncthreads();
+        // Cumulative counts from the largest bucket down; 256 threads, descending order.
+        int c = tid < 256 ? s_hist[255 - tid] : 0;
+        int total;
+        const int incl = block_inclusive_scan(c, s_warp, total);
+        if (tid < 256 && incl >= remaining && incl - c < remaining) {
+            s_prefix = prefix | ((unsigned long long)(255 - tid) << shift);
+            s_remaining = remaining - (incl - c);
+        }
+        __syncthreads();
+        prefix = s_prefix;
+        remaining = s_remaining;
+        mask |= 255ull << shift;
+        __syncthreads();
+    }
+    // prefix == T exactly; `remaining` keys equal to T are taken, lowest positions first.
+    const unsigned long long T = prefix;
+    int eq_carry = 0, out_carry = 0;
+    for (int base = 0; base < n; base += kSelectThreads) {
+        const int t = base + tid;
+        const unsigned long long key = t < n ? keys[t] : 0ull;
+        const bool gt = t < n && key > T;
+        const bool eq = t < n && key == T;
+        int eq_total;
+        const int eq_incl = block_inclusive_scan(eq ? 1 : 0, s_warp, eq_total);
+        const bool keep = gt || (eq && eq_carry + eq_incl <= remaining);
+        int keep_total;
+        const int keep_incl = block_inclusive_scan(keep ? 1 : 0, s_warp, keep_total);
+        if (keep) out[out_carry + keep_incl - 1] = cb + t;
+        eq_carry += eq_total;
+        out_carry += keep_total;
+    }
+}
+
+template <bool BF16, int D>
+cudaError_t launch_score_t(const TopkParams &p, cudaStream_t s) {
+    dim3 grid(p.n_splits, p.kv.h_kv, p.batch);
+    topk_score_kernel<BF16, D><<<grid, kScoreThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t topk_workspace_bytes(int batch, int h_kv, int max_cand) {
+    return (size_t)batch * h_kv * (size_t)max_cand * sizeof(unsigned long long);
+}
+
+cudaError_t launch_topk(const TopkParams &p, cudaStream_t s) {
+    const bool bf = p.kv.dtype == SD_BF16;
+    cudaError_t e;
+    if (p.kv.head_dim == 128)
+        e = bf ? launch_score_t<true, 128>(p, s) : launch_score_t<false, 128>(p, s);
+    else
+        e = bf ? launch_score_t<true, 64>(p, s) : launch_score_t<false, 64>(p, s);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.kv.h_kv, p.batch);
+    topk_select_kernel<<<grid, kSelectThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace sd

@@ -1,0 +1,212 @@
+"""GPU parity of the three attention calls against the fp64 oracle (through the C-ABI).
+
+Tolerances (max-abs over every output element): 2e-2 for bf16 KV, 1e-4 for fp32 KV.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from speculative_decoding_attention_verify_b200 import device as dev
+from speculative_decoding_attention_verify_b200 import inputs as gen
+from speculative_decoding_attention_verify_b200 import sdattn as sd
+
+pytestmark = pytest.mark.gpu
+
+TOL = {gen.F32: 1e-4, gen.BF16: 2e-2}
+
+
+def _assert_close(out, ref, dtype, where=""):
+    got = dev.to_numpy_f64(out)
+    assert got.shape == ref.shape, where
+    assert np.isfinite(got).all(), f"{where}: non-finite output"
+    err = float(np.abs(got - ref).max())
+    assert err <= TOL[dtype], f"{where}: max-abs error {err} > {TOL[dtype]}"
+    return err
+
+
+# ---------------------------------------------------------------- verify -------------------
+
+VERIFY_CASES = [
+    (0, {}),                                                   # C0 tiny fp32
+    (0, dict(l_vis=1000, l_txt=333, gamma=6)),                 # fp32, several tiles, ragged tail
+    (1, {}),                                                   # C1 7B-like layer
+    (1, dict(l_vis=777, l_txt=45, gamma=1)),                   # bf16, ragged, R = 14 rows
+    (1, dict(l_vis=3000, l_txt=100, gamma=0)),                 # gamma = 0: one row per head
+    (1, dict(l_vis=5000, l_txt=300, gamma=4, l_cap_pad=37)),   # NaN-filled unused capacity
+    (2, dict(layers=3, l_vis=4000, l_txt=200)),                # multi-layer batch
+    (3, dict(layers=2, l_vis=2500, l_txt=300)),                # gamma 8: R = 63 rows
+    (4, dict(l_vis=1500, l_txt=100, batch=5)),                 # paged, ragged gammas, NaN page tails
+    (4, {}),                                                   # C4 full: 8 sequences up to 34.8k
+]
+
+
+@pytest.mark.parametrize("cfg,kw", VERIFY_CASES)
+def test_verify_matches_oracle(cfg, kw):
+    w = gen.make_attn_workload(cfg, **kw)
+    out = sd.sd_verify_attention(dev.verify_queries(w), dev.kv_cache(w))
+    ref = oracle.verify_attention(w.h_q, w.q_verify, w.q_verify_start, oracle.cache_from_workload(w))
+    _assert_close(out, ref, w.dtype, f"verify cfg{cfg} {kw}")
+
+
+def test_verify_c2_full_launch_sampled_layers():
+    """All 28 layers of the long-video case in one launch; three layers checked in full."""
+    w = gen.make_attn_workload(2)
+    out = sd.sd_verify_attention(dev.verify_queries(w), dev.kv_cache(w))
+    got = dev.to_numpy_f64(out)
+    n_q = int(w.n_q_verify[0])
+    for layer in (0, 13, 27):
+        sub = oracle.Cache(w.dtype, w.k[layer:layer + 1], w.v[layer:layer + 1],
+                           w.kv_len_verify[layer:layer + 1], w.h_kv, w.d)
+        rows = slice(layer * n_q, (layer + 1) * n_q)
+        ref = oracle.verify_attention(w.h_q, w.q_verify[rows], [0, n_q], sub)
+        err = np.abs(got[rows] - ref).max()
+        assert err <= TOL[w.dtype], (layer, err)
+
+
+def test_verify_gamma0_equals_single_token_decode():
+    w = gen.make_attn_workload(1, l_vis=2000, l_txt=64, gamma=0, layers=1)
+    out = sd.sd_verify_attention(dev.verify_queries(w), dev.kv_cache(w))
+    ref = oracle.decode_attention(w.h_q, w.q_verify, oracle.cache_from_workload(w))
+    _assert_close(out, ref, w.dtype, "gamma0")
+
+
+def test_verify_split_count_does_not_change_the_result():
+    w = gen.make_attn_workload(1, l_vis=6000, l_txt=200, gamma=2)
+    kv = dev.kv_cache(w)
+    a = sd.sd_verify_attention(dev.verify_queries(w), kv)
+    q_small_hint = dev.queries(w.q_verify, w.q_verify_start, w.dtype, 256)  # forces one split
+    b = sd.sd_verify_attention(q_small_hint, kv)
+    diff = (a.float() - b.float()).abs().max().item()
+    assert diff <= 2e-2
+
+
+def test_verify_is_deterministic():
+    w = gen.make_attn_workload(4, l_vis=3000, l_txt=150, batch=4)
+    kv, q = dev.kv_cache(w), dev.verify_queries(w)
+    a = sd.sd_verify_attention(q, kv)
+    b = sd.sd_verify_attention(q, kv)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_verify_bad_page_sets_flag_without_fault():
+    w = gen.make_attn_workload(4, l_vis=500, l_txt=40, batch=2)
+    bt = w.block_table.copy()
+    bt[1, 3] = w.num_pages + 5  # out of the pool
+    kv = dev.kv_cache(w)
+    kv = sd.KVCache(kv.k, kv.v, kv.kv_len, block_table=dev.int32(bt))
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sd.sd_verify_attention(dev.verify_queries(w), kv, dev_err=flag)
+    torch.cuda.synchronize()
+    assert flag.item() & sd.SD_DEVERR_PAGE
+
+
+# ---------------------------------------------------------------- text-anchored ------------
+
+
+def _text_anchored_case(w, step=0, vis=None, window=None):
+    lens = w.kv_len_draft(step)
+    kv = dev.kv_cache(w, kv_len=lens)
+    q = dev.draft_queries(w, step)
+    vb = np.zeros(w.n_seq, np.int32) if vis is None else np.full(w.n_seq, vis[0], np.int32)
+    ve = w.l_vis.astype(np.int32) if vis is None else np.full(w.n_seq, vis[1], np.int32)
+    win = w.window if window is None else np.full(w.n_seq, window, np.int32)
+    out = sd.sd_text_anchored_attention(q, kv, dev.int32(vb), dev.int32(ve), dev.int32(win),
+                                        int(win.max()))
+    ref = oracle.text_anchored_attention(w.h_q, w.q_draft[step], np.arange(w.n_seq + 1),
+                                         oracle.cache_from_workload(w, kv_len=lens), vb, ve, win)
+    return out, ref
+
+
+TA_CASES = [
+    (0, {}, {}),
+    (1, {}, {}),
+    (1, dict(l_vis=3000, l_txt=700), dict(step=3)),
+    (1, dict(l_vis=3000, l_txt=300), dict(vis=(1000, 2500), window=900)),   # window crosses span
+    (1, dict(l_vis=3000, l_txt=300), dict(vis=(0, 0), window=777)),        # no visual span
+    (1, dict(l_vis=3000, l_txt=300), dict(window=1)),
+    (2, dict(layers=4, l_vis=3000), {}),
+    (4, dict(l_vis=2000, l_txt=300, batch=6), {}),
+    (4, {}, {}),
+]
+
+
+@pytest.mark.parametrize("cfg,kw,case", TA_CASES)
+def test_text_anchored_matches_oracle(cfg, kw, case):
+    w = gen.make_attn_workload(cfg, **kw)
+    out, ref = _text_anchored_case(w, **case)
+    _assert_close(out, ref, w.dtype, f"text-anchored cfg{cfg} {kw} {case}")
+
+
+def test_text_anchored_multi_row_verify_shape():
+    """Text-anchored attention over gamma+1 rows at once (rows slide the window up)."""
+    w = gen.make_attn_workload(1, l_vis=2000, l_txt=400, gamma=5)
+    kv, q = dev.kv_cache(w), dev.verify_queries(w)
+    vb = np.zeros(1, np.int32)
+    ve = w.l_vis.astype(np.int32)
+    win = np.array([300], np.int32)
+    out = sd.sd_text_anchored_attention(q, kv, dev.int32(vb), dev.int32(ve), dev.int32(win), 300)
+    ref = oracle.text_anchored_attention(w.h_q, w.q_verify, w.q_verify_start,
+                                         oracle.cache_from_workload(w), vb, ve, win)
+    _assert_close(out, ref, w.dtype, "text-anchored multi-row")
+
+
+# ---------------------------------------------------------------- sparse -------------------
+
+
+def _oracle_topk(w, lens, k):
+    cache = oracle.cache_from_workload(w, kv_len=lens)
+    idx, _ = oracle.topk_select(w.h_q, w.q_verify, w.q_verify_start, cache,
+                                np.zeros(w.n_seq, np.int32), w.l_vis, k)
+    return idx
+
+
+SPARSE_CASES = [
+    (0, {}, 0),
+    (1, dict(l_vis=4000, l_txt=300), 0),
+    (3, dict(layers=3, l_vis=5000, l_txt=600), 2),
+    (4, dict(l_vis=3000, l_txt=200, batch=5), 0),
+    (4, {}, 1),
+]
+
+
+@pytest.mark.parametrize("cfg,kw,step", SPARSE_CASES)
+def test_sparse_matches_oracle(cfg, kw, step):
+    w = gen.make_attn_workload(cfg, **kw)
+    lens = w.kv_len_draft(step)
+    idx = _oracle_topk(w, w.kv_len_verify, w.topk)
+    kv = dev.kv_cache(w, kv_len=lens)
+    q = dev.draft_queries(w, step)
+    tail = w.l_vis.astype(np.int32)
+    max_tail = int((lens - tail).max())
+    out = sd.sd_sparse_attention(q, kv, dev.int32(idx), dev.int32(tail), max_tail)
+    ref = oracle.sparse_attention(w.h_q, w.q_draft[step], np.arange(w.n_seq + 1),
+                                  oracle.cache_from_workload(w, kv_len=lens), idx, tail)
+    _assert_close(out, ref, w.dtype, f"sparse cfg{cfg} {kw}")
+
+
+def test_sparse_with_every_candidate_equals_dense():
+    w = gen.make_attn_workload(1, l_vis=1500, l_txt=100)
+    lens = w.kv_len_draft(0)
+    ctx = int(lens[0]) - 1
+    idx = np.arange(ctx, dtype=np.int32).reshape(1, 1, -1).repeat(w.h_kv, axis=1)
+    kv = dev.kv_cache(w, kv_len=lens)
+    q = dev.draft_queries(w, 0)
+    sparse = sd.sd_sparse_attention(q, kv, dev.int32(idx), dev.int32([ctx]), 1)
+    dense = sd.sd_verify_attention(q, kv)
+    ref = oracle.verify_attention(w.h_q, w.q_draft[0], [0, 1],
+                                  oracle.cache_from_workload(w, kv_len=lens))
+    _assert_close(sparse, ref, w.dtype, "sparse-all")
+    _assert_close(dense, ref, w.dtype, "dense")
+
+
+def test_sparse_unsorted_indices_set_flag():
+    w = gen.make_attn_workload(0)
+    lens = w.kv_len_draft(0)
+    idx = np.array([[[5, 3, 9, 9, 100]]], np.int32)
+    kv = dev.kv_cache(w, kv_len=lens)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sd.sd_sparse_attention(dev.draft_queries(w, 0), kv, dev.int32(idx),
+                           dev.int32(w.l_vis), 100, dev_err=flag)
+    torch.cuda.synchronize()
+    assert flag.item() & sd.SD_DEVERR_INDEX

@@ -1,0 +1,105 @@
+"""GPU parity of top-K selection (bit-exact index sets) and the HSR projection."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from speculative_decoding_attention_verify_b200 import device as dev
+from speculative_decoding_attention_verify_b200 import inputs as gen
+from speculative_decoding_attention_verify_b200 import sdattn as sd
+
+pytestmark = pytest.mark.gpu
+
+NEAR_TIE = 1e-9
+
+
+def _run_topk(w, k, cand_begin=None, cand_end=None, lens=None):
+    lens = w.kv_len_verify if lens is None else lens
+    cb = np.zeros(w.n_seq, np.int32) if cand_begin is None else cand_begin
+    ce = w.l_vis.astype(np.int32) if cand_end is None else cand_end
+    kv = dev.kv_cache(w, kv_len=lens)
+    q = dev.verify_queries(w)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = sd.sd_topk_select(q, kv, dev.int32(cb), dev.int32(ce), int((ce - cb).max()), k,
+                            dev_err=flag).cpu().numpy()
+    ref, gap = oracle.topk_select(w.h_q, w.q_verify, w.q_verify_start,
+                                  oracle.cache_from_workload(w, kv_len=lens), cb, ce, k)
+    assert flag.item() == 0
+    return got, ref, gap
+
+
+def _assert_same_sets(got, ref, gap):
+    """Bit-exact, except where the oracle's boundary margin is a near-tie (counted)."""
+    near = 0
+    for b in range(got.shape[0]):
+        for g in range(got.shape[1]):
+            if not np.array_equal(got[b, g], ref[b, g]):
+                assert gap[b, g] < NEAR_TIE, f"(b={b}, g={g}) differs with boundary gap {gap[b, g]}"
+                near += 1
+    return near
+
+
+TOPK_CASES = [
+    (0, {}, 32),
+    (0, {}, 300),                                    # more than the 256 candidates
+    (1, {}, 1024),
+    (1, dict(l_vis=5000, l_txt=64), 7),
+    (3, dict(layers=3, l_vis=6000, l_txt=100), 1024),
+    (4, dict(l_vis=2500, l_txt=200, batch=6), 1024),
+    (4, {}, 1024),
+]
+
+
+@pytest.mark.parametrize("cfg,kw,k", TOPK_CASES)
+def test_topk_matches_oracle_exactly(cfg, kw, k):
+    w = gen.make_attn_workload(cfg, **kw)
+    got, ref, gap = _run_topk(w, k)
+    near = _assert_same_sets(got, ref, gap)
+    assert near == 0
+
+
+def test_topk_c3_full_launch_sampled_layers():
+    w = gen.make_attn_workload(3)
+    kv = dev.kv_cache(w)
+    cb = np.zeros(w.n_seq, np.int32)
+    ce = w.l_vis.astype(np.int32)
+    got = sd.sd_topk_select(dev.verify_queries(w), kv, dev.int32(cb), dev.int32(ce), 25000,
+                            1024).cpu().numpy()
+    n_q = int(w.n_q_verify[0])
+    for layer in (0, 11, 27):
+        sub = oracle.Cache(w.dtype, w.k[layer:layer + 1], w.v[layer:layer + 1],
+                           w.kv_len_verify[layer:layer + 1], w.h_kv, w.d)
+        ref, gap = oracle.topk_select(w.h_q, w.q_verify[layer * n_q:(layer + 1) * n_q], [0, n_q],
+                                      sub, [0], [25000], 1024)
+        assert _assert_same_sets(got[layer:layer + 1], ref, gap) == 0
+        # the salient keys (4x the query direction) are all selected
+        for g in range(w.h_kv):
+            assert set(w.salient[layer][g].tolist()) <= set(got[layer, g].tolist())
+
+
+def test_topk_offset_candidate_range_and_ties():
+    w = gen.make_attn_workload(1, l_vis=3000, l_txt=50)
+    k_dup = w.k.copy()
+    k_dup[0, :, 1000:1010] = k_dup[0, :, 999:1000]  # exact duplicate keys -> ties
+    w.k = k_dup
+    cb = np.array([500], np.int32)
+    ce = np.array([2500], np.int32)
+    got, ref, gap = _run_topk(w, 40, cand_begin=cb, cand_end=ce)
+    assert _assert_same_sets(got, ref, gap) == 0
+
+
+# ---------------------------------------------------------------- HSR ----------------------
+
+
+@pytest.mark.parametrize("n,bias,d_model", [(1, False, 3584), (3, True, 3584), (16, True, 3584),
+                                            (2, False, 512)])
+def test_hsr_matches_oracle(n, bias, d_model):
+    hw = gen.make_hsr_workload(n=n, d_model=d_model, with_bias=bias)
+    e = dev.tensor(hw.emb, gen.BF16)
+    h = dev.tensor(hw.hid, gen.BF16)
+    W = dev.tensor(hw.weight, gen.BF16)
+    b = dev.tensor(hw.bias, gen.BF16) if bias else None
+    y = sd.sd_hsr_project(e, h, W, b)
+    ref = oracle.hsr_project(hw.emb, hw.hid, hw.weight, hw.bias)
+    err = np.abs(dev.to_numpy_f64(y) - ref).max()
+    assert err <= 2e-2, err
