@@ -72,6 +72,7 @@ typedef enum {
 #define SD_DEVERR_TOKEN 4u    /* drafted token outside [0, vocab) */
 #define SD_DEVERR_NUMERIC 8u  /* non-finite softmax statistics during sampling */
 #define SD_DEVERR_SHAPE 16u   /* a device length exceeds its host hint (rows, kv_len) */
+#define SD_DEVERR_TIMEOUT 32u /* a bounded wait inside a kernel expired; its outputs are undefined */
 
 /*
  * KV cache of a batch of independent sequences.  A multi-layer problem is a batch whose

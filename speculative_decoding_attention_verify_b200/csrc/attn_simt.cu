@@ -444,7 +444,7 @@ cudaError_t launch_simt_t(const AttnParams &p, const AttnPlan &plan, cudaStream_
                                              (int)dyn);
         if (e != cudaSuccess) return e;
     }
-    dim3 grid(plan.n_splits * plan.n_rowblocks, p.kv.h_kv, p.batch);
+    dim3 grid(p.n_splits * plan.n_rowblocks, p.kv.h_kv, p.batch);
     kern<<<grid, kThreads, dyn, s>>>(p);
     return cudaGetLastError();
 }

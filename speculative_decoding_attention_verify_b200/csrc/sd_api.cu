@@ -26,33 +26,39 @@ AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, in
     const int sms = device_sm_count();
     const size_t rows_cap = (size_t)batch * max_q_rows;
     if (max_stream < 1) max_stream = 1;
+    plan.max_kv_len = (int)(max_stream < (1LL << 30) ? max_stream : (1LL << 30));
     plan.tensor_core = tc_supported(kind, dtype, head_dim, rows);
-    if (plan.tensor_core) {
-        plan.rows_per_block = 128;
-        plan.n_rowblocks = 1;
-        const long long units = (long long)batch * h_kv;
-        const long long tiles = (max_stream + 127) / 128;
-        // one CTA per SM: aim for about two waves of position chunks of >= 4 tiles
-        long long splits = (2LL * sms + units - 1) / units;
-        long long by_len = (tiles + 3) / 4;
-        if (splits > by_len) splits = by_len;
-        if (splits < 1) splits = 1;
-        if (splits > 512) splits = 512;
-        plan.n_splits = (int)splits;
-    } else {
-        plan.rows_per_block = rows <= 8 ? 8 : 16;
-        plan.n_rowblocks = (rows + plan.rows_per_block - 1) / plan.rows_per_block;
+    // CUDA-core decomposition: about eight resident-CTA slots' worth of work per SM.
+    plan.rows_per_block = rows <= 8 ? 8 : 16;
+    plan.n_rowblocks = (rows + plan.rows_per_block - 1) / plan.rows_per_block;
+    {
         const long long units = (long long)batch * h_kv * plan.n_rowblocks;
         long long splits = (8LL * sms + units - 1) / units;
-        long long by_len = (max_stream + 255) / 256;
+        const long long by_len = (max_stream + 255) / 256;
         if (splits > by_len) splits = by_len;
-        if (splits < 1) splits = 1;
-        if (splits > 512) splits = 512;
-        plan.n_splits = (int)splits;
+        plan.simt_splits = (int)(splits < 1 ? 1 : (splits > 512 ? 512 : splits));
     }
-    plan.ws_bytes = plan.n_splits > 1
-                        ? (size_t)plan.n_splits * rows_cap * h_q * (head_dim + 2) * sizeof(float)
-                        : 0;
+    // Tensor-core decomposition: one CTA per SM; pick the split count whose CTAs fill whole
+    // waves best, keeping at least two 128-position tiles per CTA.
+    plan.tc_splits = 1;
+    if (plan.tensor_core) {
+        const long long units = (long long)batch * h_kv;
+        const long long tiles = (max_stream + 127) / 128;
+        double best = -1.0;
+        for (long long s = 1; s <= 64; ++s) {
+            if (s > 1 && tiles / s < 2) break;
+            const long long ctas = units * s;
+            const long long waves = (ctas + sms - 1) / sms;
+            const double score = (double)ctas / (double)(waves * sms) - 0.003 * (double)s;
+            if (score > best) {
+                best = score;
+                plan.tc_splits = (int)s;
+            }
+        }
+    }
+    const int splits = plan.simt_splits > plan.tc_splits ? plan.simt_splits : plan.tc_splits;
+    plan.ws_bytes = splits > 1 ? (size_t)splits * rows_cap * h_q * (head_dim + 2) * sizeof(float)
+                               : 0;
     return plan;
 }
 
@@ -133,22 +139,34 @@ AttnParams base_params(sd_attn_kind kind, const sd_q_desc *q, const void *q_data
     p.q = q_data;
     p.q_start = q->q_start;
     p.out = out;
-    p.n_splits = plan.n_splits;
     p.n_rowblocks = plan.n_rowblocks;
     p.ws_o = reinterpret_cast<float *>(ws);
-    p.ws_ml = plan.n_splits > 1
-                  ? p.ws_o + (size_t)plan.n_splits * p.rows_cap * q->h_q * kv->head_dim
-                  : nullptr;
     p.dev_err = dev_err;
     return p;
 }
 
-sd_status run_attention(const AttnParams &p, const AttnPlan &plan, void *stream) {
+void set_splits(AttnParams &p, int n_splits) {
+    p.n_splits = n_splits;
+    p.ws_ml = n_splits > 1 ? p.ws_o + (size_t)n_splits * p.rows_cap * p.h_q * p.kv.head_dim
+                           : nullptr;
+}
+
+sd_status run_attention(AttnParams p, const AttnPlan &plan, void *stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = plan.tensor_core ? launch_attention_tc(p, plan, s)
-                                     : launch_attention_simt(p, plan, s);
+    cudaError_t e = cudaErrorNotSupported;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.out)) &
+                          15) == 0;
+    if (plan.tensor_core && aligned) {
+        set_splits(p, plan.tc_splits);
+        e = launch_attention_tc(p, plan, s);
+        if (e != cudaSuccess && e != cudaErrorNotSupported) return SD_ERR_CUDA;
+    }
+    if (e == cudaErrorNotSupported) {
+        set_splits(p, plan.simt_splits);
+        e = launch_attention_simt(p, plan, s);
+    }
     if (e != cudaSuccess) return SD_ERR_CUDA;
-    if (plan.n_splits > 1) e = launch_attention_merge(p, s);
+    if (p.n_splits > 1) e = launch_attention_merge(p, s);
     return cuda_status(e);
 }
 
@@ -243,12 +261,7 @@ sd_status sd_sparse_attention(const sd_q_desc *q, const void *q_data, const sd_k
     sd_status st = check_attention(SD_ATTN_SPARSE, q, kv, batch,
                                    stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail), &plan);
     if (st != SD_OK) return st;
-    if (plan.tensor_core) {  // the sparse gather always runs on the CUDA-core engine
-        const int rows = (q->h_q / kv->h_kv) * q->max_q_rows;
-        plan.tensor_core = false;
-        plan.rows_per_block = rows <= 8 ? 8 : 16;
-        plan.n_rowblocks = (rows + plan.rows_per_block - 1) / plan.rows_per_block;
-    }
+    plan.tensor_core = false;  // the sparse gather always runs on the CUDA-core engine
     if (plan.ws_bytes > workspace_bytes || (plan.ws_bytes && !workspace)) return SD_ERR_WORKSPACE;
     AttnParams p = base_params(SD_ATTN_SPARSE, q, q_data, kv, batch, out, plan, workspace, dev_err);
     p.idx = idx;

@@ -39,12 +39,16 @@ struct AttnParams {
     int32_t *dev_err;
 };
 
-// Decomposition chosen for an attention call (host side; depends on host hints only).
+// Decomposition of an attention call (host side; depends on host hints only).  Both the
+// tensor-core and the CUDA-core decompositions are planned; the workspace fits either, so a
+// call can fall back to the CUDA-core engine when the tensor-core path cannot be set up.
 struct AttnPlan {
-    bool tensor_core;  // tcgen05 path
-    int n_splits;
-    int n_rowblocks;
-    int rows_per_block;
+    bool tensor_core;  // tcgen05 path preferred
+    int tc_splits;
+    int simt_splits;
+    int n_rowblocks;     // CUDA-core path
+    int rows_per_block;  // CUDA-core path
+    int max_kv_len;
     size_t ws_bytes;
 };
 

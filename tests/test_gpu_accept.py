@@ -127,7 +127,7 @@ def test_sample_identical_distributions_accept_all():
 def test_sample_bad_token_sets_flag():
     aw = gen.make_accept_workload(0, batch=2, gammas=[3, 3])
     toks = aw.draft_tokens_sampled.copy()
-    toks[1] = aw.vocab + 7
+    toks[0] = aw.vocab + 7  # position 0 is always evaluated
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
     sd.sd_accept_sample(_t(aw.target_logits), _t(aw.draft_logits), _t(toks), _t(aw.u), _t(aw.v),
                         _t(aw.gamma), 3, dev_err=flag)
