@@ -254,6 +254,22 @@ class HostInputs:
             dst.copy_(src, non_blocking=True)
 
 
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity on one rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(bytes_per_step: int, steps: int, max_ms: float, world: int) -> float:
+    """GB/s of the whole job: every rank processed its own replica in at most max_ms."""
+    return world * bytes_per_step * steps / (max_ms / 1e3) / 1e9
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -323,12 +339,7 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    max_over_ranks = lambda x: reduce_max(x, world, device)
 
     # ---- device-resident timing (optionally replayed from a CUDA graph) ----
     graph = None
@@ -361,7 +372,7 @@ def run_ours(args):
     ms = max_over_ranks(ms)
     ms_per_step = ms / args.steps
     bytes_step = sum(cyc.bytes.values())
-    value = world * bytes_step * args.steps / (ms / 1e3) / 1e9
+    value = whole_job_value(bytes_step, args.steps, ms, world)
 
     # ---- dominant kernel: verify, timed live with events on the launching stream ----
     cyc.verify_events = []
@@ -391,7 +402,7 @@ def run_ours(args):
     e1.record()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * bytes_step * args.steps / (e2e_ms / 1e3) / 1e9
+    e2e_value = whole_job_value(bytes_step, args.steps, e2e_ms, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
