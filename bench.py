@@ -510,6 +510,64 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+CASES = ("verify", "sparse", "text_anchored", "topk", "hsr", "accept_greedy", "accept_sample")
+
+
+def run_case(args):
+    """One call kind of the cycle on a reduced workload (``--layers``), repeated ``--steps``
+    times after ``--warmup``; prints its device time.  Used for ncu captures of one kernel."""
+    import torch
+    from speculative_decoding_attention_verify_b200 import device as dev
+    from speculative_decoding_attention_verify_b200 import inputs as gen
+    from speculative_decoding_attention_verify_b200 import sdattn as sd
+    w = gen.make_attn_workload(CFG_INDEX, layers=args.layers)
+    L, g = w.n_seq, int(w.gamma[0])
+    k = dev.tensor(w.k, w.dtype)
+    v = dev.tensor(w.v, w.dtype)
+    kv_verify = dev.kv_cache(w, k=k, v=v)
+    lens = w.kv_len_draft(0)
+    kv_draft = dev.kv_cache(w, kv_len=lens, k=k, v=v)
+    qv, qd = dev.verify_queries(w), dev.draft_queries(w, 0)
+    i32 = dev.int32
+    if args.case == "verify":
+        call = lambda: sd.sd_verify_attention(qv, kv_verify)
+    elif args.case == "topk":
+        call = lambda: sd.sd_topk_select(qv, kv_verify, i32(np.zeros(L)), i32(w.l_vis),
+                                         int(w.l_vis.max()), w.topk)
+    elif args.case == "sparse":
+        idx = sd.sd_topk_select(qv, kv_verify, i32(np.zeros(L)), i32(w.l_vis),
+                                int(w.l_vis.max()), w.topk)
+        tail = i32(w.l_vis)
+        call = lambda: sd.sd_sparse_attention(qd, kv_draft, idx, tail, int((lens - w.l_vis).max()))
+    elif args.case == "text_anchored":
+        vb, ve, win = i32(np.zeros(L)), i32(w.l_vis), i32(w.window)
+        call = lambda: sd.sd_text_anchored_attention(qd, kv_draft, vb, ve, win, int(w.window.max()))
+    elif args.case == "hsr":
+        hw = gen.make_hsr_workload(n=1)
+        e, h, W = (dev.tensor(a, gen.BF16) for a in (hw.emb, hw.hid, hw.weight))
+        call = lambda: sd.sd_hsr_project(e, h, W)
+    else:
+        aw = gen.make_accept_workload(2, gammas=[g], batch=1)
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        tg, dr, ts, u, vv, gm = (t(a) for a in (aw.target_logits, aw.draft_logits,
+                                                aw.draft_tokens_sampled, aw.u, aw.v, aw.gamma))
+        if args.case == "accept_greedy":
+            call = lambda: sd.sd_accept_greedy(tg, ts, gm, g)
+        else:
+            call = lambda: sd.sd_accept_sample(tg, dr, ts, u, vv, gm, g)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"case": args.case, "layers": args.layers,
+                      "ms_per_call": round(e0.elapsed_time(e1) / args.steps, 4)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -519,10 +577,15 @@ def main():
     ap.add_argument("--no-graph", dest="graph", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="time one call kind on a reduced workload (for ncu captures)")
+    ap.add_argument("--layers", type=int, default=4)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.case is not None:
+        run_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -9,22 +9,26 @@
 // *position stream*:
 //   verify          [0, kv_len)
 //   text-anchored   the non-visual positions from the lowest windowed position to kv_len
-//   sparse          the compacted selected indices, then [tail_begin, kv_len)
-// Per 128-position tile: each thread scores one position against all RB rows (its K row is
-// streamed from HBM with 16-byte loads; the rows come from shared memory as broadcasts);
-// one warp per row updates the running max / sum (online softmax, base 2); then each warp
-// accumulates P.V for a quarter of the positions with lanes spread over head_dim (coalesced
-// V rows).  The four warps' partial outputs are summed in a fixed order (deterministic).
-// With one split the normalised output is written directly; otherwise the unnormalised
-// partial and its (max, sum) go to the workspace and attn_merge_kernel combines the splits
-// by their log-sum-exp.
+//   sparse          the selected indices (ascending), then [tail_begin, kv_len)
+// K and V rows of 64-position tiles are copied with 16-byte cp.async into a 3-stage
+// shared-memory ring (rows gathered through the position map, chunks XOR-swizzled so that
+// both the row-per-thread and the lanes-over-head_dim reads are conflict-free), so the copies
+// of the next two tiles overlap the arithmetic of the current one.  Per tile: two threads per
+// position score it against half of the RB rows each (packed fp32 FMA, query rows broadcast
+// from shared memory); one warp per row updates the running max / sum (online softmax, base
+// 2); then each warp accumulates P.V over a quarter of the positions with lanes spread over
+// head_dim.  The warps' partial outputs are summed in a fixed order (deterministic).  With
+// one split the normalised output is written directly; otherwise the unnormalised partial and
+// its (max, sum) go to the workspace and attn_merge_kernel combines the splits by their
+// log-sum-exp.
 #include "sd_internal.h"
 
 namespace sd {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kTile = 128;
+constexpr int kTile = 64;    // positions per tile
+constexpr int kStages = 3;  // cp.async ring depth
 
 // Positions of one row's text-anchored window: the last W positions j <= limit outside
 // [vb, ve), as up to two ranges [lo1, hi1] and [lo2, hi2] (a range with lo > hi is empty).
@@ -55,23 +59,52 @@ __device__ __forceinline__ void window_ranges(int limit, int vb, int ve, int W, 
     }
 }
 
+template <bool BF16, int D>
+struct SimtCfg {
+    static constexpr int ESZ = BF16 ? 2 : 4;
+    static constexpr int ROWB = D * ESZ;               // bytes per KV row
+    static constexpr int CH = ROWB / 16;               // 16-byte chunks per row
+    static constexpr int SWZ = CH < 16 ? CH - 1 : 15;  // chunk swizzle mask
+    static constexpr int TILEB = kTile * ROWB;         // one K (or V) tile
+    static constexpr int DYN = kStages * 2 * TILEB;    // dynamic shared memory
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *ptr) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <bool BF16, int D, int RB>
 __global__ void __launch_bounds__(kThreads)
 attn_simt_kernel(const AttnParams p) {
-    using CH = Chunk<BF16>;
-    constexpr int ESZ = BF16 ? 2 : 4;
-    constexpr int NCHUNK = D * ESZ / 16;  // 16-byte chunks per KV row
-    constexpr int EPL = D / 32;           // head_dim elements per lane in the P.V phase
-    static_assert(RB % 4 == 0 && RB * D <= RB * kTile, "tile shapes");
+    using C = SimtCfg<BF16, D>;
+    using CHK = Chunk<BF16>;
+    constexpr int EPL = D / 32;  // head_dim elements per lane in the P.V phase
+    constexpr int RH = RB / 2;   // rows per thread in the score phase
+    static_assert(RB % 8 == 0 && kThreads == 2 * kTile, "tile shapes");
 
-    extern __shared__ int s_sel[];  // sparse: compacted selected positions
-    __shared__ __align__(16) float s_q[RB][D];
+    extern __shared__ __align__(128) uint8_t s_kv[];  // [stage][K | V][kTile][ROWB]
+    __shared__ __align__(16) float s_q[RB][D];         // pre-scaled rows; output buffer at the end
     __shared__ __align__(16) float s_s[RB][kTile];
     __shared__ __align__(16) float s_p[kTile][RB];
-    __shared__ int64_t s_off[kTile];
+    __shared__ int64_t s_off[kStages][kTile];
+    __shared__ int s_pos[kStages][kTile];
     __shared__ int s_lo1[RB], s_hi1[RB], s_lo2[RB], s_hi2[RB];
     __shared__ float s_m[RB], s_l[RB], s_corr[RB];
     __shared__ int s_stream[4];
+    __shared__ int s_count[kThreads / 32];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y;
@@ -103,41 +136,28 @@ attn_simt_kernel(const AttnParams p) {
         ve = min(max(ve, 0), kv_len);
     }
 
-    // Sparse: compact the valid, strictly ascending selected positions below the tail.
+    // Sparse: the selected list is ascending with -1 padding; its usable entries (0 <= x <
+    // tail) form a prefix, counted in parallel.  Order violations are flagged here and
+    // repeated entries are skipped when the positions are mapped.
     int tail = 0;
+    const int32_t *sel = nullptr;
     if (p.kind == SD_ATTN_SPARSE) {
         tail = min(max(__ldg(p.tail_begin + b), 0), kv_len);
-        if (warp == 0) {
-            const int32_t *sel = p.idx + ((int64_t)b * kv.h_kv + g) * p.k_sel;
-            int count = 0, prev = -1;
-            for (int base = 0; base < p.k_sel; base += 32) {
-                const int e = base + lane;
-                const int x = e < p.k_sel ? __ldg(sel + e) : -1;
-                const bool in = x >= 0 && x < tail;
-                int pm = in ? x : -1;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int y = __shfl_up_sync(0xffffffffu, pm, o);
-                    if (lane >= o) pm = max(pm, y);
-                }
-                int before = __shfl_up_sync(0xffffffffu, pm, 1);
-                if (lane == 0) before = -1;
-                before = max(before, prev);
-                const bool keep = in && x > before;
-                if (in && !keep) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
-                const unsigned m = __ballot_sync(0xffffffffu, keep);
-                if (keep) s_sel[count + __popc(m & ((1u << lane) - 1u))] = x;
-                count += __popc(m);
-                prev = max(prev, __shfl_sync(0xffffffffu, pm, 31));
-            }
-            if (lane == 0) {
-                s_stream[0] = 0;
-                s_stream[1] = count;
-                s_stream[2] = tail;
-                s_stream[3] = kv_len - tail;
+        sel = p.idx + ((int64_t)b * kv.h_kv + g) * p.k_sel;
+        int cnt = 0;
+        for (int e = tid; e < p.k_sel; e += kThreads) {
+            const int x = __ldg(sel + e);
+            const bool use = x >= 0 && x < tail;
+            cnt += use ? 1 : 0;
+            if (use && e > 0) {
+                const int prev = __ldg(sel + e - 1);
+                if (prev >= x || prev < 0) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
             }
         }
-    } else if (tid == 0) {
+        cnt = __reduce_add_sync(0xffffffffu, cnt);
+        if (lane == 0) s_count[warp] = cnt;
+    }
+    if (tid == 0 && p.kind != SD_ATTN_SPARSE) {
         int s0 = 0, len0 = 0, s1 = 0, len1 = 0;
         if (p.kind == SD_ATTN_VERIFY) {
             len0 = kv_len;
@@ -199,11 +219,64 @@ attn_simt_kernel(const AttnParams p) {
         s_q[r][d] = val * p.scale_log2;
     }
     __syncthreads();
+    if (p.kind == SD_ATTN_SPARSE && tid == 0) {
+        int k_eff = 0;
+        for (int w2 = 0; w2 < kThreads / 32; ++w2) k_eff += s_count[w2];
+        s_stream[0] = 0;
+        s_stream[1] = k_eff;
+        s_stream[2] = tail;
+        s_stream[3] = kv_len - tail;
+    }
+    __syncthreads();
 
     const int s0 = s_stream[0], len0 = s_stream[1], s1 = s_stream[2], len1 = s_stream[3];
     const int64_t P = (int64_t)len0 + len1;
     const int c0 = (int)(P * split / p.n_splits), c1 = (int)(P * (split + 1) / p.n_splits);
+    const int n_tiles = (c1 - c0 + kTile - 1) / kTile;
     const bool sparse = p.kind == SD_ATTN_SPARSE;
+
+    // Physical position and element offset of every slot of tile u (threads < kTile).
+    auto map_tile = [&](int u) {
+        const int pl = c0 + u * kTile + tid;
+        int j = -1;
+        int64_t off = -1;
+        if (pl < c1) {
+            if (pl < len0) {
+                if (sparse) {
+                    j = __ldg(sel + pl);
+                    if (pl > 0 && __ldg(sel + pl - 1) >= j) j = -1;  // repeated: skip
+                } else {
+                    j = s0 + pl;
+                }
+            } else {
+                j = s1 + (pl - len0);
+            }
+            if (j >= 0 && j < kv_len) {
+                off = kv_row_offset(kv, b, g, j, p.dev_err);
+                if (off < 0) j = -1;
+            } else {
+                j = -1;
+            }
+        }
+        s_pos[u % kStages][tid] = j;
+        s_off[u % kStages][tid] = j >= 0 ? off : -1;
+    };
+    // Asynchronous copies of the K and V rows of tile u.
+    auto issue_tile = [&](int u) {
+        const int st = u % kStages;
+        const uint32_t kdst = smem_u32(s_kv) + st * 2 * C::TILEB;
+        const uint32_t vdst = kdst + C::TILEB;
+        const char *kbase = reinterpret_cast<const char *>(kv.k);
+        const char *vbase = reinterpret_cast<const char *>(kv.v);
+        for (int e = tid; e < kTile * C::CH; e += kThreads) {
+            const int row = e / C::CH, ch = e % C::CH;
+            const int64_t off = s_off[st][row];
+            if (off < 0) continue;
+            const uint32_t d = row * C::ROWB + ((ch ^ (row & C::SWZ)) << 4);
+            cp_async16(kdst + d, kbase + off * C::ESZ + ch * 16);
+            cp_async16(vdst + d, vbase + off * C::ESZ + ch * 16);
+        }
+    };
 
     float acc[RB][EPL];
 #pragma unroll
@@ -211,76 +284,81 @@ attn_simt_kernel(const AttnParams p) {
 #pragma unroll
         for (int e = 0; e < EPL; ++e) acc[r][e] = 0.f;
 
-    for (int t0 = c0; t0 < c1; t0 += kTile) {
-        // ---- scores: one position per thread, all RB rows ----
-        const int pl = t0 + tid;
-        int j = -1;
-        int64_t off = -1;
-        if (pl < c1) {
-            j = pl < len0 ? (sparse ? s_sel[pl] : s0 + pl) : s1 + (pl - len0);
-            off = kv_row_offset(kv, b, g, j, p.dev_err);
-            if (off < 0) j = -1;
-        }
-        s_off[tid] = j >= 0 ? off : -1;
-        float2 sc[RB];
+    for (int u = 0; u < kStages - 1; ++u) {
+        if (u < n_tiles && tid < kTile) map_tile(u);
+        __syncthreads();
+        if (u < n_tiles) issue_tile(u);
+        cp_async_commit();
+    }
+
+    for (int t = 0; t < n_tiles; ++t) {
+        const int u = t + kStages - 1;
+        if (u < n_tiles && tid < kTile) map_tile(u);
+        cp_async_wait<kStages - 2>();
+        __syncthreads();
+        if (u < n_tiles) issue_tile(u);
+        cp_async_commit();
+        const int st = t % kStages;
+        const uint8_t *ktile = s_kv + st * 2 * C::TILEB;
+        const uint8_t *vtile = ktile + C::TILEB;
+
+        // ---- scores: two threads per position, RB/2 rows each ----
+        {
+            const int prow = tid % kTile, half = tid / kTile;
+            const int j = s_pos[st][prow];
+            float2 sc[RH];
 #pragma unroll
-        for (int r = 0; r < RB; ++r) sc[r] = make_float2(0.f, 0.f);
-        if (j >= 0) {
-            const char *krow = reinterpret_cast<const char *>(kv.k) + off * ESZ;
+            for (int r = 0; r < RH; ++r) sc[r] = make_float2(0.f, 0.f);
+            if (j >= 0) {
+                const uint8_t *krow = ktile + prow * C::ROWB;
 #pragma unroll
-            for (int c = 0; c < NCHUNK; c += 4) {
-                uint4 raw[4];
+                for (int ch = 0; ch < C::CH; ++ch) {
+                    const uint4 raw =
+                        *reinterpret_cast<const uint4 *>(krow + ((ch ^ (prow & C::SWZ)) << 4));
+                    float f[CHK::kElems];
+                    CHK::to_float(raw, f);
+                    const int e0 = ch * CHK::kElems;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) raw[u] = ldg_stream16(krow + (c + u) * 16);
+                    for (int r = 0; r < RH; ++r) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    float f[CH::kElems];
-                    CH::to_float(raw[u], f);
-                    const int e0 = (c + u) * CH::kElems;
-#pragma unroll
-                    for (int r = 0; r < RB; ++r) {
-#pragma unroll
-                        for (int e = 0; e < CH::kElems; e += 4) {
-                            const float4 qv = *reinterpret_cast<const float4 *>(&s_q[r][e0 + e]);
-                            sc[r] = __ffma2_rn(make_float2(qv.x, qv.y), make_float2(f[e], f[e + 1]),
-                                               sc[r]);
+                        for (int e = 0; e < CHK::kElems; e += 4) {
+                            const float4 qv =
+                                *reinterpret_cast<const float4 *>(&s_q[half * RH + r][e0 + e]);
+                            sc[r] = __ffma2_rn(make_float2(qv.x, qv.y),
+                                               make_float2(f[e], f[e + 1]), sc[r]);
                             sc[r] = __ffma2_rn(make_float2(qv.z, qv.w),
                                                make_float2(f[e + 2], f[e + 3]), sc[r]);
                         }
                     }
                 }
             }
-        }
 #pragma unroll
-        for (int r = 0; r < RB; ++r) {
-            const bool ok = j >= 0 && ((j >= s_lo1[r] && j <= s_hi1[r]) ||
-                                       (j >= s_lo2[r] && j <= s_hi2[r]));
-            s_s[r][tid] = ok ? sc[r].x + sc[r].y : -INFINITY;
+            for (int r = 0; r < RH; ++r) {
+                const int rr = half * RH + r;
+                const bool ok = j >= 0 && ((j >= s_lo1[rr] && j <= s_hi1[rr]) ||
+                                           (j >= s_lo2[rr] && j <= s_hi2[rr]));
+                s_s[rr][prow] = ok ? sc[r].x + sc[r].y : -INFINITY;
+            }
         }
         __syncthreads();
 
         // ---- online softmax: one warp per row ----
-        for (int r = warp; r < RB; r += 4) {
-            float v[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) v[c] = s_s[r][lane + 32 * c];
-            const float tmax = warp_max(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
+        for (int r = warp; r < RB; r += kThreads / 32) {
+            float v0 = s_s[r][lane], v1 = s_s[r][lane + 32];
+            const float tmax = warp_max(fmaxf(v0, v1));
             const float m_old = s_m[r];
             const float m_new = fmaxf(m_old, tmax);
             float corr = 1.f, sum = 0.f;
             if (m_new != -INFINITY) {
                 corr = exp2f(m_old - m_new);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    v[c] = exp2f(v[c] - m_new);
-                    sum += v[c];
-                }
+                v0 = exp2f(v0 - m_new);
+                v1 = exp2f(v1 - m_new);
+                sum = v0 + v1;
             } else {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) v[c] = 0.f;
+                v0 = v1 = 0.f;
             }
-#pragma unroll
-            for (int c = 0; c < 4; ++c) s_p[lane + 32 * c][r] = v[c];
+            s_p[lane][r] = v0;
+            s_p[lane + 32][r] = v1;
             sum = warp_sum(sum);
             if (lane == 0) {
                 s_l[r] = s_l[r] * corr + sum;
@@ -297,61 +375,63 @@ attn_simt_kernel(const AttnParams p) {
 #pragma unroll
             for (int e = 0; e < EPL; ++e) acc[r][e] *= cr;
         }
-        const char *vbase = reinterpret_cast<const char *>(kv.v);
-        for (int t = warp; t < kTile; t += 4 * 8) {
-            float vf[8][EPL];
-            bool have[8];
+        {
+            constexpr int LANEB = EPL * C::ESZ;  // bytes per lane in a V row
+            const int lb = lane * LANEB;
+#pragma unroll 2
+            for (int t0 = warp; t0 < kTile; t0 += 4 * 4) {
+                float vf[4][EPL];
+                bool have[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int tt = t + 4 * u;
-                const int64_t o = tt < kTile ? s_off[tt] : -1;
-                have[u] = o >= 0;
-                if (have[u]) {
-                    const char *src = vbase + (o + lane * EPL) * ESZ;
+                for (int u4 = 0; u4 < 4; ++u4) {
+                    const int pp = t0 + 4 * u4;
+                    have[u4] = s_pos[st][pp] >= 0;
+                    const uint8_t *src = vtile + pp * C::ROWB +
+                                         ((((lb >> 4) ^ (pp & C::SWZ)) << 4) | (lb & 15));
                     if (BF16) {
                         if (EPL == 4) {
-                            const uint2 w2 = __ldg(reinterpret_cast<const uint2 *>(src));
-                            vf[u][0] = bf16_lo(w2.x);
-                            vf[u][1] = bf16_hi(w2.x);
-                            vf[u][2] = bf16_lo(w2.y);
-                            vf[u][3] = bf16_hi(w2.y);
+                            const uint2 w2 = *reinterpret_cast<const uint2 *>(src);
+                            vf[u4][0] = bf16_lo(w2.x);
+                            vf[u4][1] = bf16_hi(w2.x);
+                            vf[u4][2] = bf16_lo(w2.y);
+                            vf[u4][3] = bf16_hi(w2.y);
                         } else {
-                            const uint32_t w1 = __ldg(reinterpret_cast<const uint32_t *>(src));
-                            vf[u][0] = bf16_lo(w1);
-                            vf[u][1] = bf16_hi(w1);
+                            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(src);
+                            vf[u4][0] = bf16_lo(w1);
+                            vf[u4][1] = bf16_hi(w1);
                         }
                     } else {
                         if (EPL == 4) {
-                            const float4 f4 = __ldg(reinterpret_cast<const float4 *>(src));
-                            vf[u][0] = f4.x;
-                            vf[u][1] = f4.y;
-                            vf[u][2] = f4.z;
-                            vf[u][3] = f4.w;
+                            const float4 f4 = *reinterpret_cast<const float4 *>(src);
+                            vf[u4][0] = f4.x;
+                            vf[u4][1] = f4.y;
+                            vf[u4][2] = f4.z;
+                            vf[u4][3] = f4.w;
                         } else {
-                            const float2 f2 = __ldg(reinterpret_cast<const float2 *>(src));
-                            vf[u][0] = f2.x;
-                            vf[u][1] = f2.y;
+                            const float2 f2 = *reinterpret_cast<const float2 *>(src);
+                            vf[u4][0] = f2.x;
+                            vf[u4][1] = f2.y;
                         }
                     }
                 }
-            }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (!have[u]) continue;
-                const int tt = t + 4 * u;
+                for (int u4 = 0; u4 < 4; ++u4) {
+                    if (!have[u4]) continue;
+                    const int pp = t0 + 4 * u4;
 #pragma unroll
-                for (int r4 = 0; r4 < RB; r4 += 4) {
-                    const float4 pv = *reinterpret_cast<const float4 *>(&s_p[tt][r4]);
-                    const float pr[4] = {pv.x, pv.y, pv.z, pv.w};
+                    for (int r4 = 0; r4 < RB; r4 += 4) {
+                        const float4 pv = *reinterpret_cast<const float4 *>(&s_p[pp][r4]);
+                        const float pr[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                        for (int q = 0; q < 4; ++q) {
 #pragma unroll
-                        for (int e = 0; e < EPL; e += 2) {
-                            float2 a = make_float2(acc[r4 + q][e], acc[r4 + q][e + 1]);
-                            a = __ffma2_rn(make_float2(pr[q], pr[q]),
-                                           make_float2(vf[u][e], vf[u][e + 1]), a);
-                            acc[r4 + q][e] = a.x;
-                            acc[r4 + q][e + 1] = a.y;
+                            for (int e = 0; e < EPL; e += 2) {
+                                float2 a = make_float2(acc[r4 + q][e], acc[r4 + q][e + 1]);
+                                a = __ffma2_rn(make_float2(pr[q], pr[q]),
+                                               make_float2(vf[u4][e], vf[u4][e + 1]), a);
+                                acc[r4 + q][e] = a.x;
+                                acc[r4 + q][e + 1] = a.y;
+                            }
                         }
                     }
                 }
@@ -359,10 +439,12 @@ attn_simt_kernel(const AttnParams p) {
         }
         __syncthreads();
     }
+    cp_async_wait<0>();
 
-    // ---- sum the four warps' partial outputs in a fixed order ----
-    float *s_o = &s_s[0][0];  // [RB][D]
-    for (int w = 0; w < 4; ++w) {
+    // ---- sum the four warps' partial outputs in a fixed order (into s_q) ----
+    float *s_o = &s_q[0][0];  // [RB][D]
+    __syncthreads();
+    for (int w = 0; w < kThreads / 32; ++w) {
         if (warp == w) {
 #pragma unroll
             for (int r = 0; r < RB; ++r)
@@ -399,6 +481,7 @@ attn_simt_kernel(const AttnParams p) {
 }
 
 // Combine the splits of every (row, head): O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+// One warp per (row, head); lanes read the splits' statistics in parallel.
 template <bool BF16, int D>
 __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
     constexpr int EPL = D / 32;
@@ -407,24 +490,51 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
     const int row = (int)(gw / p.h_q), h = (int)(gw % p.h_q);
     const int total = __ldg(p.q_start + p.batch);
     if (row >= total || row >= p.rows_cap) return;
-    float M = -INFINITY;
-    for (int s = 0; s < p.n_splits; ++s)
-        M = fmaxf(M, p.ws_ml[(((int64_t)s * p.rows_cap + row) * p.h_q + h) * 2]);
-    float den = 0.f, o[EPL];
+    const int64_t stride = (int64_t)p.rows_cap * p.h_q;  // between splits, in (row, head) units
+    const int64_t rh = (int64_t)row * p.h_q + h;
+    float o[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) o[e] = 0.f;
+    float M = -INFINITY;
+    for (int s = lane; s < p.n_splits; s += 32) M = fmaxf(M, p.ws_ml[(s * stride + rh) * 2]);
+    M = warp_max(M);
+    float den = 0.f;
     if (M != -INFINITY) {
-        for (int s = 0; s < p.n_splits; ++s) {
-            const int64_t base = ((int64_t)s * p.rows_cap + row) * p.h_q + h;
-            const float m = p.ws_ml[base * 2], l = p.ws_ml[base * 2 + 1];
-            if (m == -INFINITY) continue;
-            const float w = exp2f(m - M);
-            den += w * l;
+        for (int s0 = 0; s0 < p.n_splits; s0 += 32) {
+            const int s = s0 + lane;
+            float w = 0.f, l = 0.f;
+            if (s < p.n_splits) {
+                const float m = p.ws_ml[(s * stride + rh) * 2];
+                l = p.ws_ml[(s * stride + rh) * 2 + 1];
+                w = m == -INFINITY ? 0.f : exp2f(m - M);
+            }
+            den += warp_sum(w * l);
+            const int n = min(32, p.n_splits - s0);
+            int i = 0;
+            for (; i + 4 <= n; i += 4) {
+                float ov[4][EPL];
+                float wv[4];
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) o[e] += w * p.ws_o[base * D + lane * EPL + e];
+                for (int k = 0; k < 4; ++k) {
+                    wv[k] = __shfl_sync(0xffffffffu, w, i + k);
+                    const float *src = p.ws_o + ((s0 + i + k) * stride + rh) * D + lane * EPL;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) ov[k][e] = src[e];
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) o[e] += wv[k] * ov[k][e];
+            }
+            for (; i < n; ++i) {
+                const float wk = __shfl_sync(0xffffffffu, w, i);
+                const float *src = p.ws_o + ((s0 + i) * stride + rh) * D + lane * EPL;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) o[e] += wk * src[e];
+            }
         }
     }
-    const int64_t oi = ((int64_t)row * p.h_q + h) * D + lane * EPL;
+    const int64_t oi = rh * D + lane * EPL;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
         const float val = den > 0.f ? o[e] / den : 0.f;
@@ -437,12 +547,14 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
 
 template <bool BF16, int D, int RB>
 cudaError_t launch_simt_t(const AttnParams &p, const AttnPlan &plan, cudaStream_t s) {
-    const size_t dyn = p.kind == SD_ATTN_SPARSE ? (size_t)p.k_sel * sizeof(int) : 0;
+    const size_t dyn = SimtCfg<BF16, D>::DYN;
     auto kern = attn_simt_kernel<BF16, D, RB>;
-    if (dyn > 16 * 1024) {
+    static bool attr_set = false;
+    if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)dyn);
         if (e != cudaSuccess) return e;
+        attr_set = true;
     }
     dim3 grid(p.n_splits * plan.n_rowblocks, p.kv.h_kv, p.batch);
     kern<<<grid, kThreads, dyn, s>>>(p);

@@ -222,6 +222,75 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+// All 128 fp32 columns [taddr, taddr+128) of this thread's TMEM lane, load + wait in one
+// statement.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
+    uint32_t r[128];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,"
+        "%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,"
+        "%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,"
+        "%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,"
+        "%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,"
+        "%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,"
+        "%126,%127}, [%128];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
+          "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+          "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
+          "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
+          "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]),
+          "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]),
+          "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]),
+          "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]),
+          "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]),
+          "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]),
+          "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]),
+          "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]),
+          "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]),
+          "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]),
+          "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]),
+          "=r"(r[127])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 64 packed columns to this thread's TMEM lane, store + wait in one statement.
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,"
+        "%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,"
+        "%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]),
+        "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]),
+        "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]),
+        "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]),
+        "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+        : "memory");
+}
+
+// 2^x with the hardware approximation (relative error ~2^-22; P is rounded to bf16 anyway).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&p);
@@ -438,6 +507,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         const int r = warp * 32 + lane;
         const bool row_ok = r < R;
         const int limit = kv_len - n_q + (row_ok ? r / G : 0);
+        const int warp_limit = kv_len - n_q + (warp * 32) / G;  // smallest limit in this warp
         const float sl2 = p.scale_log2;
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
         float m_used = -INFINITY, l = 0.f;
@@ -452,62 +522,72 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             }
             tc_after();
             const uint32_t s_addr = lane_base + sb * kTile;
-            float v[32];
+            float v[kTile];
+            tmem_ld128(s_addr, v);
+            // Interior tiles (every position visible to every row of this warp) skip masking.
+            const bool interior = p0 + kTile - 1 <= warp_limit;
             float mx = -INFINITY;
+            if (interior) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                tmem_ld32(s_addr + c * 32, v);
+                for (int e = 0; e < kTile; ++e) mx = fmaxf(mx, v[e]);
+                mx *= sl2;
+            } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const bool ok = row_ok && p0 + c * 32 + e <= limit;
-                    mx = fmaxf(mx, ok ? v[e] * sl2 : -INFINITY);
+                for (int e = 0; e < kTile; ++e) {
+                    if (!(row_ok && p0 + e <= limit)) v[e] = -INFINITY;
+                    mx = fmaxf(mx, v[e]);
                 }
+                mx = mx == -INFINITY ? -INFINITY : mx * sl2;
             }
             const bool grow = mx > m_used + kRescaleLog2;
             const bool rescale_o = grow && m_used != -INFINITY;
             if (__any_sync(FULL, rescale_o)) {
-                // O holds tiles < t: wait for the last P.V, then rescale O in TMEM.
+                // O holds tiles < t: wait for the P.V of tile t-1, then rescale O in TMEM.
+                // S_t was committed after the P.V of tile t-2 and the P.V of tile t needs this
+                // warp's arrival, so o_done is in phase t-1 or t: its parity test is exact.
                 const bool done = mbar_wait(BAR(OD), (t - 1) & 1, abort_flag, p.dev_err);
                 if (!__all_sync(FULL, done)) {
                     ok_run = false;
                     break;
                 }
                 tc_after();
-                const float corr = rescale_o ? exp2f(m_used - mx) : 1.f;
+                const float corr = rescale_o ? ex2(m_used - mx) : 1.f;
+                float o[32];
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    tmem_ld32(lane_base + kColO + c * 32, v);
+                    tmem_ld32(lane_base + kColO + c * 32, o);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] *= corr;
-                    tmem_st32(lane_base + kColO + c * 32, v);
+                    for (int e = 0; e < 32; ++e) o[e] *= corr;
+                    tmem_st32(lane_base + kColO + c * 32, o);
                 }
                 l *= corr;
             }
             if (grow) m_used = mx;
-            float sum = 0.f;
-            const bool live = m_used != -INFINITY;
+            // P = 2^(s*scale - m): masked entries are -inf and give exactly 0.
+            const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+            const float keep = m_used == -INFINITY ? 0.f : 1.f;
+            float sum0 = 0.f, sum1 = 0.f;
+            uint32_t pk[kTile / 2];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                tmem_ld32(s_addr + c * 32, v);
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const bool ok0 = live && row_ok && p0 + c * 32 + e <= limit;
-                    const bool ok1 = live && row_ok && p0 + c * 32 + e + 1 <= limit;
-                    const float a = ok0 ? exp2f(fmaf(v[e], sl2, -m_used)) : 0.f;
-                    const float bb = ok1 ? exp2f(fmaf(v[e + 1], sl2, -m_used)) : 0.f;
-                    sum += a + bb;
-                    pk[e >> 1] = pack_bf16(a, bb);
-                }
-                tmem_st16(s_addr + c * 16, pk);
+            for (int e = 0; e < kTile; e += 2) {
+                const float a = ex2(fmaf(v[e], sl2, neg_m)) * keep;
+                const float bb = ex2(fmaf(v[e + 1], sl2, neg_m)) * keep;
+                sum0 += a;
+                sum1 += bb;
+                pk[e >> 1] = pack_bf16(a, bb);
             }
+            tmem_st64(s_addr, pk);
+            const float sum = sum0 + sum1;
             l += sum;
             tc_before();
             mbar_arrive(BAR(PF + sb));
         }
         // ---- epilogue ----
+        // Wait on the one-shot drain barrier (committed after the last P.V), not on the
+        // per-tile o_done barrier: here only the P.V of tiles < n_my - 2 is known to be
+        // complete, so o_done could be two phases behind and its parity test would pass early.
         bool done = ok_run;
-        if (ok_run && n_my > 0) done = mbar_wait(BAR(OD), (n_my - 1) & 1, abort_flag, p.dev_err);
+        if (ok_run && n_my > 0) done = mbar_wait(BAR(DR), 0, abort_flag, p.dev_err);
         const bool read_o = __all_sync(FULL, done) && n_my > 0;
         tc_after();
         const bool have = read_o && m_used != -INFINITY;

@@ -39,7 +39,7 @@ hsr_kernel(const uint16_t *emb, const uint16_t *hid, int n_rows, int d_model, co
     float acc[NR];
 #pragma unroll
     for (int r = 0; r < NR; ++r) acc[r] = 0.f;
-    constexpr int U = 4;
+    constexpr int U = 14;  // 14 x 16 bytes per lane in flight
     for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
         uint4 wv[U];
 #pragma unroll

@@ -28,15 +28,30 @@ AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, in
     if (max_stream < 1) max_stream = 1;
     plan.max_kv_len = (int)(max_stream < (1LL << 30) ? max_stream : (1LL << 30));
     plan.tensor_core = tc_supported(kind, dtype, head_dim, rows);
-    // CUDA-core decomposition: about eight resident-CTA slots' worth of work per SM.
+    // CUDA-core decomposition: 64-position tiles, a 3-stage K/V ring of 3*2*64 rows in
+    // shared memory; two CTAs fit per SM when the ring is at most 96 KB.  Choose the split
+    // count whose CTAs fill whole waves best, with at least two tiles per CTA and a penalty
+    // for the per-CTA set-up and the merge.
     plan.rows_per_block = rows <= 8 ? 8 : 16;
     plan.n_rowblocks = (rows + plan.rows_per_block - 1) / plan.rows_per_block;
     {
+        const int esz = dtype == SD_BF16 ? 2 : 4;
+        const long long ring = 3LL * 2 * 64 * head_dim * esz;
+        const long long slots = (long long)sms * (ring <= 96 * 1024 ? 2 : 1);
         const long long units = (long long)batch * h_kv * plan.n_rowblocks;
-        long long splits = (8LL * sms + units - 1) / units;
-        const long long by_len = (max_stream + 255) / 256;
-        if (splits > by_len) splits = by_len;
-        plan.simt_splits = (int)(splits < 1 ? 1 : (splits > 512 ? 512 : splits));
+        const long long tiles = (max_stream + 63) / 64;
+        double best = -1.0;
+        plan.simt_splits = 1;
+        for (long long s = 1; s <= 256; ++s) {
+            if (s > 1 && tiles / s < 2) break;
+            const long long ctas = units * s;
+            const long long waves = (ctas + slots - 1) / slots;
+            const double score = (double)ctas / (double)(waves * slots) - 0.01 * (double)s;
+            if (score > best) {
+                best = score;
+                plan.simt_splits = (int)s;
+            }
+        }
     }
     // Tensor-core decomposition: one CTA per SM; pick the split count whose CTAs fill whole
     // waves best, keeping at least two 128-position tiles per CTA.

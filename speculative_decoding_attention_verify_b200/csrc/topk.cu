@@ -9,7 +9,8 @@
 //    8-bit digits, shared-memory histograms) finds the k-th largest key T exactly; then one
 //    pass in position order keeps every key > T and the first (k - #greater) keys == T, so
 //    equal scores go to the lower position, and block-wide prefix sums write the kept
-//    positions in ascending order.
+//    positions in ascending order.  When the keys fit in shared memory (up to 26,624) they are
+//    loaded once and the select touches shared memory only.
 #include "sd_internal.h"
 
 namespace sd {
@@ -74,20 +75,17 @@ __global__ void __launch_bounds__(kScoreThreads) topk_score_kernel(const TopkPar
         unsigned long long key = 0ull;
         if (off >= 0) {
             const char *row = reinterpret_cast<const char *>(p.kv.k) + off * ESZ;
+            uint4 raw[NCHUNK];  // the whole row in flight at once
+#pragma unroll
+            for (int c = 0; c < NCHUNK; ++c) raw[c] = ldg_stream16(row + c * 16);
             double acc = 0.0;
 #pragma unroll
-            for (int c = 0; c < NCHUNK; c += 4) {
-                uint4 raw[4];
+            for (int c = 0; c < NCHUNK; ++c) {
+                float f[CH::kElems];
+                CH::to_float(raw[c], f);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) raw[u] = ldg_stream16(row + (c + u) * 16);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    float f[CH::kElems];
-                    CH::to_float(raw[u], f);
-#pragma unroll
-                    for (int e = 0; e < CH::kElems; ++e)
-                        acc = fma((double)f[e], s_qbar[(c + u) * CH::kElems + e], acc);
-                }
+                for (int e = 0; e < CH::kElems; ++e)
+                    acc = fma((double)f[e], s_qbar[c * CH::kElems + e], acc);
             }
             key = score_key(acc);
         }
@@ -185,6 +183,84 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(const TopkP
     }
 }
 
+// Selection with every key in shared memory (up to kSmemKeys): the keys are loaded once,
+// coalesced; thread t then owns the contiguous candidates [t*kpt, t*kpt + kpt).  The eight
+// radix passes touch shared memory only, and the compaction needs a single block-wide scan
+// because each thread's candidates are contiguous.
+constexpr int kSmemKeys = 26624;  // 208 KB of keys
+
+__global__ void __launch_bounds__(kSelectThreads) topk_select_smem_kernel(const TopkParams p) {
+    extern __shared__ unsigned long long s_keys[];
+    __shared__ int s_hist[256];
+    __shared__ int s_warp[32];
+    __shared__ unsigned long long s_prefix;
+    __shared__ int s_remaining;
+    const int b = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
+    int32_t *out = p.idx_out + ((int64_t)b * p.kv.h_kv + g) * p.k;
+    const int last = __ldg(p.q_start + b + 1) - 1;
+    if (last < __ldg(p.q_start + b)) {
+        for (int e = tid; e < p.k; e += kSelectThreads) out[e] = -1;
+        return;
+    }
+    int cb, n;
+    cand_range(p, b, cb, n);
+    const unsigned long long *keys = p.keys + ((int64_t)b * p.kv.h_kv + g) * p.max_cand;
+    if (n <= p.k) {
+        for (int e = tid; e < p.k; e += kSelectThreads) out[e] = e < n ? cb + e : -1;
+        return;
+    }
+    for (int e = tid; e < n; e += kSelectThreads) s_keys[e] = keys[e];
+    const int kpt = (n + kSelectThreads - 1) / kSelectThreads;
+    const int first = tid * kpt;
+    const int mine = max(0, min(kpt, n - first));  // keys owned by this thread
+    const unsigned long long *my = s_keys + first;
+    unsigned long long prefix = 0ull, mask = 0ull;
+    int remaining = p.k;
+    for (int digit = 7; digit >= 0; --digit) {
+        const int shift = digit * 8;
+        if (tid < 256) s_hist[tid] = 0;
+        __syncthreads();
+        for (int i = 0; i < mine; ++i) {
+            const unsigned long long kk = my[i];
+            if ((kk & mask) == prefix) atomicAdd(&s_hist[(int)((kk >> shift) & 255ull)], 1);
+        }
+        __syncthreads();
+        const int c = tid < 256 ? s_hist[255 - tid] : 0;
+        int total;
+        const int incl = block_inclusive_scan(c, s_warp, total);
+        if (tid < 256 && incl >= remaining && incl - c < remaining) {
+            s_prefix = prefix | ((unsigned long long)(255 - tid) << shift);
+            s_remaining = remaining - (incl - c);
+        }
+        __syncthreads();
+        prefix = s_prefix;
+        remaining = s_remaining;
+        mask |= 255ull << shift;
+    }
+    const unsigned long long T = prefix;
+    // keys > T are all kept; the first `remaining` keys == T in position order are kept
+    int eq = 0, gt = 0;
+    for (int i = 0; i < mine; ++i) {
+        eq += my[i] == T ? 1 : 0;
+        gt += my[i] > T ? 1 : 0;
+    }
+    int eq_total;
+    const int eq_before = block_inclusive_scan(eq, s_warp, eq_total) - eq;
+    int eq_left = max(0, min(eq, remaining - eq_before));  // equal keys this thread keeps
+    const int keep_n = gt + eq_left;
+    int keep_total;
+    int pos = block_inclusive_scan(keep_n, s_warp, keep_total) - keep_n;
+    for (int i = 0; i < mine; ++i) {
+        const unsigned long long kk = my[i];
+        bool keep = kk > T;
+        if (kk == T && eq_left > 0) {
+            keep = true;
+            --eq_left;
+        }
+        if (keep) out[pos++] = cb + first + i;
+    }
+}
+
 template <bool BF16, int D>
 cudaError_t launch_score_t(const TopkParams &p, cudaStream_t s) {
     dim3 grid(p.n_splits, p.kv.h_kv, p.batch);
@@ -207,7 +283,20 @@ cudaError_t launch_topk(const TopkParams &p, cudaStream_t s) {
         e = bf ? launch_score_t<true, 64>(p, s) : launch_score_t<false, 64>(p, s);
     if (e != cudaSuccess) return e;
     dim3 grid(p.kv.h_kv, p.batch);
-    topk_select_kernel<<<grid, kSelectThreads, 0, s>>>(p);
+    if (p.max_cand <= kSmemKeys) {
+        const size_t dyn = (size_t)p.max_cand * sizeof(unsigned long long);
+        static bool attr_set = false;
+        if (!attr_set) {
+            e = cudaFuncSetAttribute(topk_select_smem_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)(kSmemKeys * sizeof(unsigned long long)));
+            if (e != cudaSuccess) return e;
+            attr_set = true;
+        }
+        topk_select_smem_kernel<<<grid, kSelectThreads, dyn, s>>>(p);
+    } else {
+        topk_select_kernel<<<grid, kSelectThreads, 0, s>>>(p);
+    }
     return cudaGetLastError();
 }
 

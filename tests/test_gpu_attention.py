@@ -210,3 +210,21 @@ def test_sparse_unsorted_indices_set_flag():
                            dev.int32(w.l_vis), 100, dev_err=flag)
     torch.cuda.synchronize()
     assert flag.item() & sd.SD_DEVERR_INDEX
+
+
+@pytest.mark.parametrize("l_vis,l_txt,batch", [(300, 40, 7), (1500, 100, 5), (700, 33, 9)])
+def test_verify_short_chunks_repeated(l_vis, l_txt, batch):
+    """Short sequences split into CTAs of one to three tiles, run repeatedly: every run must
+    match the oracle and be bitwise identical (catches pipeline races in the epilogue)."""
+    w = gen.make_attn_workload(4, l_vis=l_vis, l_txt=l_txt, batch=batch)
+    kv, q = dev.kv_cache(w), dev.verify_queries(w)
+    ref = oracle.verify_attention(w.h_q, w.q_verify, w.q_verify_start, oracle.cache_from_workload(w))
+    first = None
+    for _ in range(12):
+        out = sd.sd_verify_attention(q, kv)
+        _assert_close(out, ref, w.dtype, "short chunks")
+        bits = out.view(torch.int16).clone()
+        if first is None:
+            first = bits
+        else:
+            assert torch.equal(first, bits)
