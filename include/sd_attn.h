@@ -212,7 +212,7 @@ SD_API sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd
  *     y[r][o] = sum_i W[o][i] emb[r][i] + sum_i W[o][d_model+i] hid[r][i] (+ bias[o])
  * emb, hid: [n_rows][d_model]; W: [d_model][2*d_model] (out x in); bias: [d_model] or NULL;
  * y: [n_rows][d_model].  All bf16; fp32 accumulation.  The concatenation is never
- * materialised.  1 <= n_rows <= 16; d_model a multiple of 8; pointers 16-byte aligned.
+ * materialised.  1 <= n_rows <= 16; d_model a multiple of 16; emb, hid and W 16-byte aligned.
  */
 SD_API sd_status sd_hsr_project(const void *emb, const void *hid, int32_t n_rows, int32_t d_model,
                          const void *weight, const void *bias, void *y, void *stream);

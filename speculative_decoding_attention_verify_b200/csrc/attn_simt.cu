@@ -13,51 +13,22 @@
 // K and V rows of 64-position tiles are copied with 16-byte cp.async into a 3-stage
 // shared-memory ring (rows gathered through the position map, chunks XOR-swizzled so that
 // both the row-per-thread and the lanes-over-head_dim reads are conflict-free), so the copies
-// of the next two tiles overlap the arithmetic of the current one.  Per tile: two threads per
-// position score it against half of the RB rows each (packed fp32 FMA, query rows broadcast
-// from shared memory); one warp per row updates the running max / sum (online softmax, base
-// 2); then each warp accumulates P.V over a quarter of the positions with lanes spread over
-// head_dim.  The warps' partial outputs are summed in a fixed order (deterministic).  With
+// of the next two tiles overlap the arithmetic of the current one.  Per tile (256 threads,
+// 64 positions): four threads per position score it against a quarter of the RB rows each
+// (packed fp32 FMA, query rows broadcast from shared memory); one warp per row updates the
+// running max / sum (online softmax, base 2); then each warp accumulates P.V over an eighth
+// of the positions with lanes spread over head_dim.  The warps' partial outputs are summed in a fixed order (deterministic).  With
 // one split the normalised output is written directly; otherwise the unnormalised partial and
 // its (max, sum) go to the workspace and attn_merge_kernel combines the splits by their
 // log-sum-exp.
-#include "sd_internal.h"
+#include "attn_stream.cuh"
 
 namespace sd {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kTile = 64;    // positions per tile
 constexpr int kStages = 3;  // cp.async ring depth
-
-// Positions of one row's text-anchored window: the last W positions j <= limit outside
-// [vb, ve), as up to two ranges [lo1, hi1] and [lo2, hi2] (a range with lo > hi is empty).
-__device__ __forceinline__ void window_ranges(int limit, int vb, int ve, int W, int &lo1,
-                                              int &hi1, int &lo2, int &hi2) {
-    lo2 = 1;
-    hi2 = 0;
-    if (vb >= ve) vb = ve = 0;
-    if (limit < 0 || W <= 0) {
-        lo1 = 1;
-        hi1 = 0;
-        return;
-    }
-    if (limit >= ve) {  // row above the visual span
-        lo1 = max(ve, limit - W + 1);
-        hi1 = limit;
-        const int rem = W - (hi1 - lo1 + 1);
-        if (rem > 0 && vb > 0) {
-            hi2 = vb - 1;
-            lo2 = max(0, vb - rem);
-        }
-    } else if (limit >= vb) {  // row inside the span: only positions below it
-        hi1 = vb - 1;
-        lo1 = max(0, vb - W);
-    } else {  // row below the span
-        hi1 = limit;
-        lo1 = max(0, limit - W + 1);
-    }
-}
 
 template <bool BF16, int D>
 struct SimtCfg {
@@ -91,9 +62,11 @@ __global__ void __launch_bounds__(kThreads)
 attn_simt_kernel(const AttnParams p) {
     using C = SimtCfg<BF16, D>;
     using CHK = Chunk<BF16>;
-    constexpr int EPL = D / 32;  // head_dim elements per lane in the P.V phase
-    constexpr int RH = RB / 2;   // rows per thread in the score phase
-    static_assert(RB % 8 == 0 && kThreads == 2 * kTile, "tile shapes");
+    constexpr int EPL = D / 32;                  // head_dim elements per lane in the P.V phase
+    constexpr int PARTS = kThreads / kTile;       // threads sharing one position's scores
+    constexpr int RH = RB / PARTS;                // rows per thread in the score phase
+    constexpr int NW = kThreads / 32;
+    static_assert(RB % PARTS == 0 && RH % 2 == 0 && kThreads % kTile == 0, "tile shapes");
 
     extern __shared__ __align__(128) uint8_t s_kv[];  // [stage][K | V][kTile][ROWB]
     __shared__ __align__(16) float s_q[RB][D];         // pre-scaled rows; output buffer at the end
@@ -103,8 +76,7 @@ attn_simt_kernel(const AttnParams p) {
     __shared__ int s_pos[kStages][kTile];
     __shared__ int s_lo1[RB], s_hi1[RB], s_lo2[RB], s_hi2[RB];
     __shared__ float s_m[RB], s_l[RB], s_corr[RB];
-    __shared__ int s_stream[4];
-    __shared__ int s_count[kThreads / 32];
+    __shared__ int s_stream[4 + kThreads / 32];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y;
@@ -122,82 +94,13 @@ attn_simt_kernel(const AttnParams p) {
         return;
     }
 
-    // Visual span / window (text-anchored only).
-    int vb = 0, ve = 0, W = 0;
-    if (p.kind == SD_ATTN_TEXT_ANCHORED) {
-        vb = __ldg(p.vis_begin + b);
-        ve = __ldg(p.vis_end + b);
-        W = __ldg(p.window + b);
-        if (vb > ve) {
-            if (tid == 0) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
-            vb = ve = 0;
-        }
-        vb = min(max(vb, 0), kv_len);
-        ve = min(max(ve, 0), kv_len);
-    }
-
-    // Sparse: the selected list is ascending with -1 padding; its usable entries (0 <= x <
-    // tail) form a prefix, counted in parallel.  Order violations are flagged here and
-    // repeated entries are skipped when the positions are mapped.
-    int tail = 0;
-    const int32_t *sel = nullptr;
-    if (p.kind == SD_ATTN_SPARSE) {
-        tail = min(max(__ldg(p.tail_begin + b), 0), kv_len);
-        sel = p.idx + ((int64_t)b * kv.h_kv + g) * p.k_sel;
-        int cnt = 0;
-        for (int e = tid; e < p.k_sel; e += kThreads) {
-            const int x = __ldg(sel + e);
-            const bool use = x >= 0 && x < tail;
-            cnt += use ? 1 : 0;
-            if (use && e > 0) {
-                const int prev = __ldg(sel + e - 1);
-                if (prev >= x || prev < 0) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
-            }
-        }
-        cnt = __reduce_add_sync(0xffffffffu, cnt);
-        if (lane == 0) s_count[warp] = cnt;
-    }
-    if (tid == 0 && p.kind != SD_ATTN_SPARSE) {
-        int s0 = 0, len0 = 0, s1 = 0, len1 = 0;
-        if (p.kind == SD_ATTN_VERIFY) {
-            len0 = kv_len;
-        } else {
-            // Lowest position any row of this sequence may see (windows slide up with rows).
-            int lowest = kv_len;
-            for (int i = 0; i < n_q; ++i) {
-                int lo1, hi1, lo2, hi2;
-                window_ranges(kv_len - n_q + i, vb, ve, W, lo1, hi1, lo2, hi2);
-                if (lo2 <= hi2) lowest = min(lowest, lo2);
-                if (lo1 <= hi1) lowest = min(lowest, lo1);
-            }
-            if (vb < ve && lowest < vb) {
-                s0 = lowest;
-                len0 = vb - lowest;
-                s1 = ve;
-            } else {
-                s1 = (vb < ve && lowest >= vb) ? max(lowest, ve) : lowest;
-            }
-            len1 = max(0, kv_len - s1);
-        }
-        s_stream[0] = s0;
-        s_stream[1] = len0;
-        s_stream[2] = s1;
-        s_stream[3] = len1;
-    }
+    const StreamInfo si = stream_setup<kThreads>(p, b, g, n_q, kv_len, s_stream);
 
     // Per-row allowed ranges, running statistics and the pre-scaled query rows.
     if (tid < RB) {
-        const int r = tid, lr = rb * RB + r;
-        int lo1 = 1, hi1 = 0, lo2 = 1, hi2 = 0;
-        if (lr < R) {
-            const int limit = kv_len - n_q + lr / G;
-            if (p.kind == SD_ATTN_TEXT_ANCHORED) {
-                window_ranges(limit, vb, ve, W, lo1, hi1, lo2, hi2);
-            } else {
-                lo1 = 0;
-                hi1 = limit;
-            }
-        }
+        const int r = tid;
+        int lo1, hi1, lo2, hi2;
+        row_ranges(p, si, rb * RB + r, R, n_q, kv_len, lo1, hi1, lo2, hi2);
         s_lo1[r] = lo1;
         s_hi1[r] = hi1;
         s_lo2[r] = lo2;
@@ -219,44 +122,19 @@ attn_simt_kernel(const AttnParams p) {
         s_q[r][d] = val * p.scale_log2;
     }
     __syncthreads();
-    if (p.kind == SD_ATTN_SPARSE && tid == 0) {
-        int k_eff = 0;
-        for (int w2 = 0; w2 < kThreads / 32; ++w2) k_eff += s_count[w2];
-        s_stream[0] = 0;
-        s_stream[1] = k_eff;
-        s_stream[2] = tail;
-        s_stream[3] = kv_len - tail;
-    }
-    __syncthreads();
-
-    const int s0 = s_stream[0], len0 = s_stream[1], s1 = s_stream[2], len1 = s_stream[3];
+    const int len0 = si.len0, len1 = si.len1;
     const int64_t P = (int64_t)len0 + len1;
     const int c0 = (int)(P * split / p.n_splits), c1 = (int)(P * (split + 1) / p.n_splits);
     const int n_tiles = (c1 - c0 + kTile - 1) / kTile;
-    const bool sparse = p.kind == SD_ATTN_SPARSE;
 
     // Physical position and element offset of every slot of tile u (threads < kTile).
     auto map_tile = [&](int u) {
         const int pl = c0 + u * kTile + tid;
-        int j = -1;
+        int j = pl < c1 ? stream_position(p, si, pl, kv_len) : -1;
         int64_t off = -1;
-        if (pl < c1) {
-            if (pl < len0) {
-                if (sparse) {
-                    j = __ldg(sel + pl);
-                    if (pl > 0 && __ldg(sel + pl - 1) >= j) j = -1;  // repeated: skip
-                } else {
-                    j = s0 + pl;
-                }
-            } else {
-                j = s1 + (pl - len0);
-            }
-            if (j >= 0 && j < kv_len) {
-                off = kv_row_offset(kv, b, g, j, p.dev_err);
-                if (off < 0) j = -1;
-            } else {
-                j = -1;
-            }
+        if (j >= 0) {
+            off = kv_row_offset(kv, b, g, j, p.dev_err);
+            if (off < 0) j = -1;
         }
         s_pos[u % kStages][tid] = j;
         s_off[u % kStages][tid] = j >= 0 ? off : -1;
@@ -302,9 +180,9 @@ attn_simt_kernel(const AttnParams p) {
         const uint8_t *ktile = s_kv + st * 2 * C::TILEB;
         const uint8_t *vtile = ktile + C::TILEB;
 
-        // ---- scores: two threads per position, RB/2 rows each ----
+        // ---- scores: PARTS threads per position, RH rows each ----
         {
-            const int prow = tid % kTile, half = tid / kTile;
+            const int prow = tid % kTile, half = tid / kTile;  // half: which RH-row slice
             const int j = s_pos[st][prow];
             float2 sc[RH];
 #pragma unroll
@@ -343,7 +221,7 @@ attn_simt_kernel(const AttnParams p) {
         __syncthreads();
 
         // ---- online softmax: one warp per row ----
-        for (int r = warp; r < RB; r += kThreads / 32) {
+        for (int r = warp; r < RB; r += NW) {
             float v0 = s_s[r][lane], v1 = s_s[r][lane + 32];
             const float tmax = warp_max(fmaxf(v0, v1));
             const float m_old = s_m[r];
@@ -368,7 +246,7 @@ attn_simt_kernel(const AttnParams p) {
         }
         __syncthreads();
 
-        // ---- P.V: warp w takes positions w, w+4, ...; lanes spread over head_dim ----
+        // ---- P.V: warp w takes positions w, w+NW, ...; lanes spread over head_dim ----
 #pragma unroll
         for (int r = 0; r < RB; ++r) {
             const float cr = s_corr[r];
@@ -379,12 +257,12 @@ attn_simt_kernel(const AttnParams p) {
             constexpr int LANEB = EPL * C::ESZ;  // bytes per lane in a V row
             const int lb = lane * LANEB;
 #pragma unroll 2
-            for (int t0 = warp; t0 < kTile; t0 += 4 * 4) {
+            for (int t0 = warp; t0 < kTile; t0 += NW * 4) {
                 float vf[4][EPL];
                 bool have[4];
 #pragma unroll
                 for (int u4 = 0; u4 < 4; ++u4) {
-                    const int pp = t0 + 4 * u4;
+                    const int pp = t0 + NW * u4;
                     have[u4] = s_pos[st][pp] >= 0;
                     const uint8_t *src = vtile + pp * C::ROWB +
                                          ((((lb >> 4) ^ (pp & C::SWZ)) << 4) | (lb & 15));
@@ -417,7 +295,7 @@ attn_simt_kernel(const AttnParams p) {
 #pragma unroll
                 for (int u4 = 0; u4 < 4; ++u4) {
                     if (!have[u4]) continue;
-                    const int pp = t0 + 4 * u4;
+                    const int pp = t0 + NW * u4;
 #pragma unroll
                     for (int r4 = 0; r4 < RB; r4 += 4) {
                         const float4 pv = *reinterpret_cast<const float4 *>(&s_p[pp][r4]);
@@ -441,10 +319,10 @@ attn_simt_kernel(const AttnParams p) {
     }
     cp_async_wait<0>();
 
-    // ---- sum the four warps' partial outputs in a fixed order (into s_q) ----
+    // ---- sum the warps' partial outputs in a fixed order (into s_q) ----
     float *s_o = &s_q[0][0];  // [RB][D]
     __syncthreads();
-    for (int w = 0; w < kThreads / 32; ++w) {
+    for (int w = 0; w < NW; ++w) {
         if (warp == w) {
 #pragma unroll
             for (int r = 0; r < RB; ++r)

@@ -7,7 +7,8 @@
 //   warps 0-3  softmax: TMEM lane r holds query row r (rows ordered (i, h), h fastest; rows
 //              R..127 are padding and never read back)
 //   warp 4     TMA producer: K and V tiles of 128 positions (128-byte swizzle) into a
-//              3-4 stage shared-memory ring (contiguous caches: one 4-D box per half of
+//              3-4 stage shared-memory ring (a stage's K is released once S is computed, its V
+//              once P.V is) (contiguous caches: one 4-D box per half of
 //              head_dim; paged caches: one box per 16-position page)
 //   warp 5     MMA issuer (one elected thread) and TMEM owner
 // Per tile t (double-buffered S in TMEM):
@@ -49,7 +50,7 @@ struct Cfg {
     static constexpr int kStages = D == 128 ? 3 : 4;
     static constexpr int kQBytes = kRows * D * 2;
     static constexpr int kBarOffset = kQBytes + kStages * 2 * kTileBytes;
-    static constexpr int kSmem = kBarOffset + 256 + 1024;  // barriers + alignment slack
+    static constexpr int kSmem = kBarOffset + 256 + 1024;  // barriers (<= 4S+8 words) + slack
 };
 
 // ---------------------------------------------------------------- PTX wrappers ------------
@@ -284,6 +285,12 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64
         : "memory");
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // 2^x with the hardware approximation (relative error ~2^-22; P is rounded to bf16 anyway).
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -314,12 +321,14 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     uint8_t *sQ = smem;
     uint8_t *sKV = smem + C::kQBytes;  // stage s: K at s*2*tile, V at s*2*tile + tile
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
-    // barrier slots: k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_done, drain
+    // barrier slots: k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_full[2],
+    // o_done, drain.  A stage's K half is released as soon as S = Q K^T is computed, its V
+    // half once P.V is, so the next K copy starts a softmax earlier.
     const uint32_t bar0 = saddr(bars);
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    const int KF = 0, VF = S, KE = 2 * S, SF = 3 * S, PF = 3 * S + 2, OD = 3 * S + 4,
-              DR = 3 * S + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * S + 6);
+    const int KF = 0, VF = S, KE = 2 * S, VE = 3 * S, SF = 4 * S, PF = 4 * S + 2, OD = 4 * S + 4,
+              DR = 4 * S + 5;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * S + 6);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -353,6 +362,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             mbar_init(BAR(KF + s), 1);
             mbar_init(BAR(VF + s), 1);
             mbar_init(BAR(KE + s), 1);
+            mbar_init(BAR(VE + s), 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(BAR(SF + s), 1);
@@ -388,21 +398,13 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     if (warp == kProducerWarp) {
         // ---------------------------------------------------------- TMA producer ----------
         if (lane == 0) {
+            int pages[kTile / kPageSize];
             for (int t = 0; t < n_my; ++t) {
                 const int s = t % S, use = t / S;
-                if (t >= S && !mbar_wait(BAR(KE + s), (use - 1) & 1, abort_flag, p.dev_err)) break;
                 const int p0 = (tile_lo + t) * kTile;
                 const uint32_t dK = saddr(sKV + (size_t)s * 2 * C::kTileBytes);
                 const uint32_t dV = dK + C::kTileBytes;
-                mbar_arrive_tx(BAR(KF + s), C::kTileBytes);
-                mbar_arrive_tx(BAR(VF + s), C::kTileBytes);
-                if (!PAGED) {
-#pragma unroll
-                    for (int h = 0; h < C::kHalves; ++h) {
-                        tma_load_4d(dK + h * kHalfBytes, &maps.k, BAR(KF + s), h * 64, p0, g, b);
-                        tma_load_4d(dV + h * kHalfBytes, &maps.v, BAR(VF + s), h * 64, p0, g, b);
-                    }
-                } else {
+                if (PAGED) {
                     for (int pg = 0; pg < kTile / kPageSize; ++pg) {
                         const int pos = p0 + pg * kPageSize;
                         int page = kv.num_pages;  // out of range: zero-filled box
@@ -414,14 +416,29 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                             else
                                 set_dev_err(p.dev_err, SD_DEVERR_PAGE);
                         }
-#pragma unroll
-                        for (int h = 0; h < C::kHalves; ++h) {
-                            const uint32_t o = h * kHalfBytes + pg * kPageSize * 128;
-                            tma_load_4d(dK + o, &maps.k, BAR(KF + s), h * 64, 0, g, page);
-                            tma_load_4d(dV + o, &maps.v, BAR(VF + s), h * 64, 0, g, page);
-                        }
+                        pages[pg] = page;
                     }
                 }
+                for (int half = 0; half < 2; ++half) {  // K, then V
+                    const int full = half == 0 ? KF : VF, empty = half == 0 ? KE : VE;
+                    const uint32_t dst = half == 0 ? dK : dV;
+                    const CUtensorMap *map = half == 0 ? &maps.k : &maps.v;
+                    if (t >= S && !mbar_wait(BAR(empty + s), (use - 1) & 1, abort_flag, p.dev_err))
+                        break;
+                    mbar_arrive_tx(BAR(full + s), C::kTileBytes);
+                    if (!PAGED) {
+#pragma unroll
+                        for (int h = 0; h < C::kHalves; ++h)
+                            tma_load_4d(dst + h * kHalfBytes, map, BAR(full + s), h * 64, p0, g, b);
+                    } else {
+                        for (int pg = 0; pg < kTile / kPageSize; ++pg)
+#pragma unroll
+                            for (int h = 0; h < C::kHalves; ++h)
+                                tma_load_4d(dst + h * kHalfBytes + pg * kPageSize * 128, map,
+                                            BAR(full + s), h * 64, 0, g, pages[pg]);
+                    }
+                }
+                if (*abort_flag) break;
             }
         }
     } else if (warp == kMmaWarp) {
@@ -449,6 +466,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                            idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(BAR(SF + sb));
+                mma_commit(BAR(KE + s));
                 issued = true;
             }
             __syncwarp();
@@ -485,7 +503,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                     mma_ts(tmem + kColO, tmem + sb * kTile + kk * 8,
                            desc_mn_sw128(vb + kk * 2048, kHalfBytes), idesc_pv,
                            (t > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(BAR(KE + s));
+                mma_commit(BAR(VE + s));
                 mma_commit(BAR(OD));
             }
             __syncwarp();
@@ -527,18 +545,14 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             // Interior tiles (every position visible to every row of this warp) skip masking.
             const bool interior = p0 + kTile - 1 <= warp_limit;
             float mx = -INFINITY;
-            if (interior) {
+            if (!interior) {
 #pragma unroll
-                for (int e = 0; e < kTile; ++e) mx = fmaxf(mx, v[e]);
-                mx *= sl2;
-            } else {
-#pragma unroll
-                for (int e = 0; e < kTile; ++e) {
+                for (int e = 0; e < kTile; ++e)
                     if (!(row_ok && p0 + e <= limit)) v[e] = -INFINITY;
-                    mx = fmaxf(mx, v[e]);
-                }
-                mx = mx == -INFINITY ? -INFINITY : mx * sl2;
             }
+#pragma unroll
+            for (int e = 0; e < kTile; e += 2) mx = max3(mx, v[e], v[e + 1]);
+            mx = mx == -INFINITY ? -INFINITY : mx * sl2;
             const bool grow = mx > m_used + kRescaleLog2;
             const bool rescale_o = grow && m_used != -INFINITY;
             if (__any_sync(FULL, rescale_o)) {
@@ -563,21 +577,21 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 l *= corr;
             }
             if (grow) m_used = mx;
-            // P = 2^(s*scale - m): masked entries are -inf and give exactly 0.
+            // P = 2^(s*scale - m).  Masked entries are -inf and give exactly 0; while no
+            // position of the row has been visible (m = -inf) every entry is masked.
             const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-            const float keep = m_used == -INFINITY ? 0.f : 1.f;
-            float sum0 = 0.f, sum1 = 0.f;
+            const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
+            float2 acc2 = make_float2(0.f, 0.f);
             uint32_t pk[kTile / 2];
 #pragma unroll
             for (int e = 0; e < kTile; e += 2) {
-                const float a = ex2(fmaf(v[e], sl2, neg_m)) * keep;
-                const float bb = ex2(fmaf(v[e + 1], sl2, neg_m)) * keep;
-                sum0 += a;
-                sum1 += bb;
-                pk[e >> 1] = pack_bf16(a, bb);
+                const float2 x = __ffma2_rn(make_float2(v[e], v[e + 1]), sc2, nm2);
+                const float2 pe = make_float2(ex2(x.x), ex2(x.y));
+                acc2 = __fadd2_rn(acc2, pe);
+                pk[e >> 1] = pack_bf16(pe.x, pe.y);
             }
             tmem_st64(s_addr, pk);
-            const float sum = sum0 + sum1;
+            const float sum = acc2.x + acc2.y;
             l += sum;
             tc_before();
             mbar_arrive(BAR(PF + sb));

@@ -1,93 +1,129 @@
 // Hidden-state-reuse projection: y = W [emb ; hid] (+ bias), bf16 in/out, fp32 accumulation.
 //
-// A weight-streaming GEMV with n_rows <= 16 right-hand sides: every weight row (2*d_model
-// bf16) is read from HBM exactly once per group of up to 4 input rows, with 16-byte loads,
-// one warp per output feature.  The input rows are copied once per CTA into shared memory as
-// the concatenation [emb ; hid] (the concatenation only ever exists in shared memory).
+// A weight-streaming GEMV with n_rows <= 16 right-hand sides, balanced so that every SM
+// streams the same number of weight bytes: one CTA per SM owns an even share of the output
+// features [r0, r1) and splits each weight row into four quarter-rows; its 16 warps take the
+// quarter-rows round-robin, two at a time (14 coalesced 16-byte loads per lane in flight), and
+// store one partial per (feature, quarter), which are summed in a fixed order (deterministic).
+// The input rows are copied once per CTA into shared memory as the concatenation
+// [emb ; hid] (the concatenation only ever exists there).  Weights are read once per group of
+// up to four input rows.
 #include "sd_internal.h"
 
 namespace sd {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;
+constexpr int kParts = 4;  // quarter-rows per weight row
 
 template <int NR>
 __global__ void __launch_bounds__(kWarps * 32)
 hsr_kernel(const uint16_t *emb, const uint16_t *hid, int n_rows, int d_model, const uint16_t *w,
-           const uint16_t *bias, uint16_t *y) {
-    extern __shared__ uint4 s_x4[];  // [NR][2*d_model] bf16, as 16-byte chunks
+           const uint16_t *bias, uint16_t *y, int max_rows_per_cta) {
+    extern __shared__ uint4 s_x4[];  // [NR][2*d_model] bf16 chunks, then [rows][kParts][NR] f32
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int r0 = blockIdx.y * NR;
-    const int nr = min(NR, n_rows - r0);
-    const int in_dim = 2 * d_model;
-    const int chunks = in_dim / 8;  // 16-byte chunks per concatenated row
-    for (int e = tid; e < NR * chunks; e += kWarps * 32) {
-        const int r = e / chunks, c = e % chunks;
+    const int g0 = blockIdx.y * NR;
+    const int nr = min(NR, n_rows - g0);
+    const int cpr = 2 * d_model / 8;    // 16-byte chunks per weight row
+    const int cpp = cpr / kParts;       // chunks per quarter-row
+    const int r0 = (int)((int64_t)d_model * blockIdx.x / gridDim.x);
+    const int r1 = (int)((int64_t)d_model * (blockIdx.x + 1) / gridDim.x);
+    float *s_part = reinterpret_cast<float *>(s_x4 + NR * cpr);
+    for (int e = tid; e < NR * cpr; e += kWarps * 32) {
+        const int r = e / cpr, c = e % cpr;
         uint4 v = make_uint4(0, 0, 0, 0);
         if (r < nr) {
             const int col = c * 8;
-            const uint16_t *src = col < d_model ? emb + (int64_t)(r0 + r) * d_model + col
-                                                : hid + (int64_t)(r0 + r) * d_model + (col - d_model);
+            const uint16_t *src = col < d_model ? emb + (int64_t)(g0 + r) * d_model + col
+                                                : hid + (int64_t)(g0 + r) * d_model + (col - d_model);
             v = *reinterpret_cast<const uint4 *>(src);
         }
         s_x4[e] = v;
     }
     __syncthreads();
-    const int o = blockIdx.x * kWarps + warp;
-    if (o >= d_model) return;
-    const uint16_t *wrow = w + (int64_t)o * in_dim;
-    float acc[NR];
+    const int items = (r1 - r0) * kParts;
+    const uint4 *wbase = reinterpret_cast<const uint4 *>(w) + (int64_t)r0 * cpr;
+    for (int it0 = warp; it0 < items; it0 += 2 * kWarps) {
+        const int it1 = it0 + kWarps;  // second item of the pair (may not exist)
+        float part[2][NR];
 #pragma unroll
-    for (int r = 0; r < NR; ++r) acc[r] = 0.f;
-    constexpr int U = 14;  // 14 x 16 bytes per lane in flight
-    for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
-        uint4 wv[U];
+        for (int k = 0; k < 2; ++k)
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int c = c0 + 32 * u;
-            wv[u] = c < chunks ? ldg_stream16(wrow + c * 8) : make_uint4(0, 0, 0, 0);
+            for (int r = 0; r < NR; ++r) part[k][r] = 0.f;
+        for (int c0 = lane; c0 < cpp; c0 += 32 * 7) {
+            uint4 wv[2][7];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int it = k == 0 ? it0 : it1;
+#pragma unroll
+                for (int u = 0; u < 7; ++u) {
+                    const int c = c0 + 32 * u;
+                    wv[k][u] = (it < items && c < cpp)
+                                   ? ldg_stream16(wbase + (int64_t)(it / kParts) * cpr +
+                                                  (it % kParts) * cpp + c)
+                                   : make_uint4(0, 0, 0, 0);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int it = k == 0 ? it0 : it1;
+                if (it >= items) break;
+#pragma unroll
+                for (int u = 0; u < 7; ++u) {
+                    const int c = c0 + 32 * u;
+                    if (c >= cpp) break;
+                    float wf[8];
+                    Chunk<true>::to_float(wv[k][u], wf);
+                    const int col = (it % kParts) * cpp + c;
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) {
+                        float xf[8];
+                        Chunk<true>::to_float(s_x4[r * cpr + col], xf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) part[k][r] = fmaf(wf[e], xf[e], part[k][r]);
+                    }
+                }
+            }
         }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int c = c0 + 32 * u;
-            if (c >= chunks) break;
-            float wf[8];
-            Chunk<true>::to_float(wv[u], wf);
+        for (int k = 0; k < 2; ++k) {
+            const int it = k == 0 ? it0 : it1;
 #pragma unroll
             for (int r = 0; r < NR; ++r) {
-                float xf[8];
-                Chunk<true>::to_float(s_x4[r * chunks + c], xf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[r] = fmaf(wf[e], xf[e], acc[r]);
+                const float sum = warp_sum(part[k][r]);
+                if (lane == 0 && it < items) s_part[(it * NR) + r] = sum;
             }
         }
     }
+    __syncthreads();
+    for (int e = tid; e < nr * (r1 - r0); e += kWarps * 32) {
+        const int r = e / (r1 - r0), i = e % (r1 - r0);
+        float val = 0.f;
 #pragma unroll
-    for (int r = 0; r < NR; ++r) {
-        const float s = warp_sum(acc[r]);
-        if (lane == 0 && r < nr) {
-            float val = s;
-            if (bias) val += __uint_as_float((uint32_t)bias[o] << 16);
-            y[(int64_t)(r0 + r) * d_model + o] = (uint16_t)f32_to_bf16_bits(val);
-        }
+        for (int q = 0; q < kParts; ++q) val += s_part[((i * kParts + q) * NR) + r];
+        if (bias) val += __uint_as_float((uint32_t)bias[r0 + i] << 16);
+        y[(int64_t)(g0 + r) * d_model + r0 + i] = (uint16_t)f32_to_bf16_bits(val);
     }
 }
 
 template <int NR>
 cudaError_t launch_hsr_t(const void *emb, const void *hid, int n_rows, int d_model, const void *w,
                          const void *bias, void *y, cudaStream_t s) {
-    const size_t smem = (size_t)NR * 2 * d_model * sizeof(uint16_t);
+    const int ctas = min(device_sm_count(), d_model);
+    const int max_rows = (d_model + ctas - 1) / ctas;
+    const size_t smem = (size_t)NR * 2 * d_model * sizeof(uint16_t) +
+                        (size_t)max_rows * kParts * NR * sizeof(float);
     auto kern = hsr_kernel<NR>;
     if (smem > 48 * 1024) {
         cudaError_t e =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    dim3 grid((d_model + kWarps - 1) / kWarps, (n_rows + NR - 1) / NR);
+    dim3 grid(ctas, (n_rows + NR - 1) / NR);
     kern<<<grid, kWarps * 32, smem, s>>>(
         reinterpret_cast<const uint16_t *>(emb), reinterpret_cast<const uint16_t *>(hid), n_rows,
         d_model, reinterpret_cast<const uint16_t *>(w), reinterpret_cast<const uint16_t *>(bias),
-        reinterpret_cast<uint16_t *>(y));
+        reinterpret_cast<uint16_t *>(y), max_rows);
     return cudaGetLastError();
 }
 

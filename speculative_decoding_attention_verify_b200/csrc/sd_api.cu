@@ -319,21 +319,32 @@ sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd_kv_des
     p.idx_out = idx_out;
     p.keys = reinterpret_cast<unsigned long long *>(workspace);
     p.dev_err = dev_err;
+    // Scoring CTAs stream 128-candidate tiles through a 3-stage ring (two CTAs per SM for
+    // bf16, d=128); choose the split count whose CTAs fill whole waves best, with at least four
+    // tiles per CTA.
     const int sms = device_sm_count();
     const long long units = (long long)batch * kv->h_kv;
-    long long splits = (4LL * sms + units - 1) / units;
-    const long long by_len = ((long long)max_cand + 1023) / 1024;
-    if (splits > by_len) splits = by_len;
-    if (splits < 1) splits = 1;
-    if (splits > 1024) splits = 1024;
-    p.n_splits = (int)splits;
+    const long long slots = (long long)sms * (kv->dtype == SD_BF16 && kv->head_dim == 128 ? 2 : 1);
+    const long long tiles = ((long long)max_cand + 127) / 128;
+    double best = -1.0;
+    p.n_splits = 1;
+    for (long long s = 1; s <= 1024; ++s) {
+        if (s > 1 && tiles / s < 4) break;
+        const long long ctas = units * s;
+        const long long waves = (ctas + slots - 1) / slots;
+        const double score = (double)ctas / (double)(waves * slots) - 0.005 * (double)s;
+        if (score > best) {
+            best = score;
+            p.n_splits = (int)s;
+        }
+    }
     return cuda_status(launch_topk(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sd_status sd_hsr_project(const void *emb, const void *hid, int32_t n_rows, int32_t d_model,
                          const void *weight, const void *bias, void *y, void *stream) {
-    if (!emb || !hid || !weight || !y || n_rows < 1 || n_rows > 16 || d_model < 8 ||
-        d_model % 8 != 0 || d_model > (1 << 20))
+    if (!emb || !hid || !weight || !y || n_rows < 1 || n_rows > 16 || d_model < 16 ||
+        d_model % 16 != 0 || d_model > (1 << 20))
         return SD_ERR_INVALID_ARG;
     const uintptr_t a = reinterpret_cast<uintptr_t>(emb) | reinterpret_cast<uintptr_t>(hid) |
                         reinterpret_cast<uintptr_t>(weight);

@@ -1,8 +1,9 @@
 // Top-K KV selection per (sequence, KV head).
 //
 // 1. topk_score_kernel: grid (splits, KV heads, sequences).  The group's last query rows are
-//    summed once in fp64 (qbar); every candidate key row is streamed with 16-byte loads and
-//    dotted with qbar in fp64 (bf16 x bf16 products are exact in fp64, and the sum of the
+//    summed once in fp64 (qbar); candidate key rows are staged through a 3-stage cp.async ring
+//    with coalesced 16-byte copies, and each thread dots one row with qbar in fp64 (four
+//    independent accumulation chains) (bf16 x bf16 products are exact in fp64, and the sum of the
 //    group's dot products equals qbar . k up to fp64 rounding).  The score is stored as an
 //    order-preserving 64-bit key (larger score -> larger key; -0 == +0; NaN lowest).
 // 2. topk_select_kernel: one CTA per (sequence, KV head).  An MSB-first radix select (eight
@@ -16,7 +17,7 @@
 namespace sd {
 namespace {
 
-constexpr int kScoreThreads = 256;
+constexpr int kScoreThreads = 128;
 constexpr int kSelectThreads = 1024;
 
 __device__ __forceinline__ unsigned long long score_key(double x) {
@@ -41,56 +42,111 @@ __device__ __forceinline__ void cand_range(const TopkParams &p, int b, int &cb, 
     if (bad && threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
 }
 
+constexpr int kScoreTile = 128;   // candidates per staged tile (one per thread)
+constexpr int kScoreStages = 3;   // cp.async ring depth
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <bool BF16, int D>
 __global__ void __launch_bounds__(kScoreThreads) topk_score_kernel(const TopkParams p) {
     using CH = Chunk<BF16>;
     constexpr int ESZ = BF16 ? 2 : 4;
-    constexpr int NCHUNK = D * ESZ / 16;
+    constexpr int ROWB = D * ESZ;
+    constexpr int NCHUNK = ROWB / 16;
+    constexpr int SWZ = NCHUNK < 16 ? NCHUNK - 1 : 15;
+    static_assert(kScoreThreads == kScoreTile, "one candidate per thread");
+    extern __shared__ __align__(128) uint8_t s_ring[];  // [stage][kScoreTile][ROWB]
     __shared__ double s_qbar[D];
+    __shared__ int64_t s_off[kScoreStages][kScoreTile];
+    const int tid = threadIdx.x;
     const int b = blockIdx.z, g = blockIdx.y, split = blockIdx.x;
     const int last = __ldg(p.q_start + b + 1) - 1;
     if (last < __ldg(p.q_start + b)) {
-        if (threadIdx.x == 0 && split == 0) set_dev_err(p.dev_err, SD_DEVERR_SHAPE);
+        if (tid == 0 && split == 0) set_dev_err(p.dev_err, SD_DEVERR_SHAPE);
         return;
     }
     int cb, n;
     cand_range(p, b, cb, n);
-    if (threadIdx.x < D) {
+    for (int e = tid; e < D; e += kScoreThreads) {
         double acc = 0.0;
         for (int h = g * p.group; h < (g + 1) * p.group; ++h) {
-            const int64_t off = ((int64_t)last * p.h_q + h) * D + threadIdx.x;
+            const int64_t off = ((int64_t)last * p.h_q + h) * D + e;
             const float qf = BF16 ? __uint_as_float((uint32_t)__ldg(
                                         reinterpret_cast<const unsigned short *>(p.q) + off) << 16)
                                   : __ldg(reinterpret_cast<const float *>(p.q) + off);
             acc += (double)qf;
         }
-        s_qbar[threadIdx.x] = acc;
+        s_qbar[e] = acc;
     }
-    __syncthreads();
     unsigned long long *keys = p.keys + ((int64_t)b * p.kv.h_kv + g) * p.max_cand;
     const int t_begin = (int)((int64_t)n * split / p.n_splits);
     const int t_end = (int)((int64_t)n * (split + 1) / p.n_splits);
-    for (int t = t_begin + threadIdx.x; t < t_end; t += kScoreThreads) {
-        const int64_t off = kv_row_offset(p.kv, b, g, cb + t, p.dev_err);
-        unsigned long long key = 0ull;
-        if (off >= 0) {
-            const char *row = reinterpret_cast<const char *>(p.kv.k) + off * ESZ;
-            uint4 raw[NCHUNK];  // the whole row in flight at once
-#pragma unroll
-            for (int c = 0; c < NCHUNK; ++c) raw[c] = ldg_stream16(row + c * 16);
-            double acc = 0.0;
-#pragma unroll
-            for (int c = 0; c < NCHUNK; ++c) {
-                float f[CH::kElems];
-                CH::to_float(raw[c], f);
-#pragma unroll
-                for (int e = 0; e < CH::kElems; ++e)
-                    acc = fma((double)f[e], s_qbar[c * CH::kElems + e], acc);
-            }
-            key = score_key(acc);
+    const int n_tiles = (t_end - t_begin + kScoreTile - 1) / kScoreTile;
+    const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(s_ring));
+    const char *kbase = reinterpret_cast<const char *>(p.kv.k);
+
+    auto map_tile = [&](int u) {
+        const int t = t_begin + u * kScoreTile + tid;
+        s_off[u % kScoreStages][tid] = t < t_end ? kv_row_offset(p.kv, b, g, cb + t, p.dev_err) : -1;
+    };
+    auto issue_tile = [&](int u) {  // coalesced: consecutive threads take consecutive chunks
+        const int st = u % kScoreStages;
+        for (int e = tid; e < kScoreTile * NCHUNK; e += kScoreThreads) {
+            const int row = e / NCHUNK, ch = e % NCHUNK;
+            const int64_t off = s_off[st][row];
+            if (off < 0) continue;
+            cp_async16(ring + (st * kScoreTile + row) * ROWB + ((ch ^ (row & SWZ)) << 4),
+                       kbase + off * ESZ + ch * 16);
         }
-        keys[t] = key;
+    };
+    for (int u = 0; u < kScoreStages - 1; ++u) {
+        if (u < n_tiles) map_tile(u);
+        __syncthreads();
+        if (u < n_tiles) issue_tile(u);
+        cp_async_commit();
     }
+    for (int t = 0; t < n_tiles; ++t) {
+        const int u = t + kScoreStages - 1;
+        if (u < n_tiles) map_tile(u);
+        cp_async_wait<kScoreStages - 2>();
+        __syncthreads();
+        if (u < n_tiles) issue_tile(u);
+        cp_async_commit();
+        const int st = t % kScoreStages;
+        const int cand = t_begin + t * kScoreTile + tid;
+        if (cand < t_end) {
+            unsigned long long key = 0ull;
+            if (s_off[st][tid] >= 0) {
+                const uint8_t *rp = s_ring + (st * kScoreTile + tid) * ROWB;
+                double a[4] = {0.0, 0.0, 0.0, 0.0};  // independent chains
+#pragma unroll
+                for (int ch = 0; ch < NCHUNK; ++ch) {
+                    const uint4 raw =
+                        *reinterpret_cast<const uint4 *>(rp + ((ch ^ (tid & SWZ)) << 4));
+                    float f[CH::kElems];
+                    CH::to_float(raw, f);
+#pragma unroll
+                    for (int e = 0; e < CH::kElems; ++e)
+                        a[e & 3] = fma((double)f[e], s_qbar[ch * CH::kElems + e], a[e & 3]);
+                }
+                key = score_key((a[0] + a[1]) + (a[2] + a[3]));
+            }
+            keys[cand] = key;
+        }
+        __syncthreads();
+    }
+    cp_async_wait<0>();
 }
 
 // Inclusive block-wide prefix sum of one int per thread (kSelectThreads threads).
@@ -263,8 +319,16 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_smem_kernel(const 
 
 template <bool BF16, int D>
 cudaError_t launch_score_t(const TopkParams &p, cudaStream_t s) {
+    const int dyn = kScoreStages * kScoreTile * D * (BF16 ? 2 : 4);
+    auto kern = topk_score_kernel<BF16, D>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
     dim3 grid(p.n_splits, p.kv.h_kv, p.batch);
-    topk_score_kernel<BF16, D><<<grid, kScoreThreads, 0, s>>>(p);
+    kern<<<grid, kScoreThreads, dyn, s>>>(p);
     return cudaGetLastError();
 }
 

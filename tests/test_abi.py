@@ -101,6 +101,7 @@ def test_other_entry_points_validate_on_the_host():
     assert lib.sd_hsr_project(ctypes.c_void_p(0x7f0000001002), P, 1, 3584, P, None, P,
                               None) == sd.SD_ERR_INVALID_ARG
     assert lib.sd_hsr_project(P, P, 1, 3580, P, None, P, None) == sd.SD_ERR_INVALID_ARG
+    assert lib.sd_hsr_project(P, P, 1, 3592, P, None, P, None) == sd.SD_ERR_INVALID_ARG
     # acceptance: out_stride too small, missing workspace
     assert lib.sd_accept_greedy(P, P, P, 2, 7, 1000, P, P, 7, P, 1 << 20, None,
                                 None) == sd.SD_ERR_INVALID_ARG
