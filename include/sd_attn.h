@@ -258,6 +258,30 @@ SD_API sd_status sd_accept_sample(const float *tgt_logits, const float *draft_lo
                            int32_t *near_boundary, void *workspace, size_t workspace_bytes,
                            int32_t *dev_err, void *stream);
 
+/*
+ * Verify attention without any allocation (no counterpart in the papers: it exists for callers
+ * that cannot allocate device memory at call time, such as a serving engine whose paged KV pool
+ * has taken all free HBM, or a host program that only holds device pointers handed to it by
+ * another runtime; cudaMalloc there would fail, shrink the pool, or synchronise the device).
+ *
+ * Computes exactly what sd_verify_attention computes, with the same arguments minus the
+ * workspace: the split-KV partials go to a scratch array of SD_VERIFY_NOALLOC_SCRATCH_BYTES
+ * that the library holds in device memory of each device it runs on.  A call whose workspace
+ * (sd_attention_workspace_size with SD_ATTN_VERIFY) exceeds that size returns
+ * SD_ERR_WORKSPACE and launches nothing.  Nothing in the scratch needs to start at zero.
+ *
+ * The first call on a device looks up the scratch's address (and may load the module that
+ * holds it), so make it before any stream capture.  Calls that may overlap on one device
+ * (different streams or host threads without ordering between them) share the scratch and
+ * race; calls on one stream are safe.  Errors: as sd_verify_attention; SD_ERR_UNSUPPORTED if
+ * the current device ordinal is 64 or more; SD_ERR_CUDA if the address lookup fails.
+ */
+#define SD_VERIFY_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+SD_API sd_status sd_verify_attention_noalloc(const sd_q_desc *q, const void *q_data,
+                                      const sd_kv_desc *kv, int32_t batch, void *out,
+                                      int32_t *dev_err, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

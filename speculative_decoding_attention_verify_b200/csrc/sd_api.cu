@@ -199,6 +199,25 @@ long long stream_hint(sd_attn_kind kind, const sd_q_desc *q, long long extra) {
 
 }  // namespace
 
+namespace sd {
+
+// Validation and plan of a verify call, for entry points that supply their own workspace.
+sd_status verify_plan(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv, int batch,
+                      const void *out, AttnPlan *plan) {
+    if (!q_data || !out) return SD_ERR_INVALID_ARG;
+    return check_attention(SD_ATTN_VERIFY, q, kv, batch, q ? q->max_kv_len : 0, plan);
+}
+
+// Launch of a verify call planned by verify_plan, on a workspace of at least plan.ws_bytes.
+sd_status verify_run(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv, int batch,
+                     void *out, const AttnPlan &plan, void *workspace, int32_t *dev_err,
+                     void *stream) {
+    AttnParams p = base_params(SD_ATTN_VERIFY, q, q_data, kv, batch, out, plan, workspace, dev_err);
+    return run_attention(p, plan, stream);
+}
+
+}  // namespace sd
+
 extern "C" {
 
 const char *sd_status_string(sd_status s) {

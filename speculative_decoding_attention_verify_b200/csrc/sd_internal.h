@@ -108,4 +108,12 @@ size_t accept_workspace_bytes(int batch, int max_gamma, int vocab, int *n_chunks
 cudaError_t launch_accept_greedy(const AcceptParams &p, cudaStream_t s);
 cudaError_t launch_accept_sample(const AcceptParams &p, cudaStream_t s);
 
+// Verify attention split into validation/plan and launch, for entry points that supply their
+// own workspace (defined with the other entry points).
+sd_status verify_plan(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv, int batch,
+                      const void *out, AttnPlan *plan);
+sd_status verify_run(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv, int batch,
+                     void *out, const AttnPlan &plan, void *workspace, int32_t *dev_err,
+                     void *stream);
+
 }  // namespace sd

@@ -51,7 +51,10 @@ class sd_q_desc(ctypes.Structure):
 EXPORTS = ("sd_status_string", "sd_version", "sd_attention_workspace_size", "sd_verify_attention",
            "sd_text_anchored_attention", "sd_sparse_attention", "sd_topk_workspace_size",
            "sd_topk_select", "sd_hsr_project", "sd_accept_workspace_size", "sd_accept_greedy",
-           "sd_accept_sample")
+           "sd_accept_sample", "sd_verify_attention_noalloc")
+
+# Size of the library's fixed scratch used by sd_verify_attention_noalloc.
+SD_VERIFY_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def lib():
@@ -79,6 +82,7 @@ def lib():
                 h.sd_accept_greedy.argtypes = [P, P, P, I32, I32, I32, P, P, I32, P, SZ, P, P]
                 h.sd_accept_sample.argtypes = [P, P, P, P, P, P, I32, I32, I32, P, P, I32, P, P, SZ,
                                                P, P]
+                h.sd_verify_attention_noalloc.argtypes = [P, P, P, I32, P, P, P]
                 for name in EXPORTS[2:]:
                     getattr(h, name).restype = ctypes.c_int
                 _LIB = h
@@ -201,6 +205,17 @@ def sd_verify_attention(q: Queries, kv: KVCache, out=None, workspace=None, dev_e
     _check(lib().sd_verify_attention(ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc),
                                      kv.batch, _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
                                      _stream(stream)), "sd_verify_attention")
+    return out
+
+
+def sd_verify_attention_noalloc(q: Queries, kv: KVCache, out: torch.Tensor, dev_err=None,
+                                stream=None) -> torch.Tensor:
+    """sd_verify_attention on the library's fixed scratch: the C call allocates nothing, so the
+    caller passes ``out``.  Raises SdError (SD_ERR_WORKSPACE) when the call's workspace exceeds
+    SD_VERIFY_NOALLOC_SCRATCH_BYTES."""
+    _check(lib().sd_verify_attention_noalloc(ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc),
+                                             kv.batch, _ptr(out), _ptr(dev_err), _stream(stream)),
+           "sd_verify_attention_noalloc")
     return out
 
 
