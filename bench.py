@@ -86,7 +86,8 @@ def recorded_traffic():
 # ---------------------------------------------------------------- algorithmic bytes --------
 
 def cycle_bytes(w, lens_draft, topk):
-    """Bytes the method must move in one step, per call kind (SURVEY-style formulas)."""
+    """Bytes the method must move in one step, per call kind (algorithmic bytes: every operand
+    the step reads or writes once; scratch is not credited)."""
     d, hk, hq, s = w.d, w.h_kv, w.h_q, 2
     row = hk * d * 2 * s  # K and V of one position, all KV heads
     L = w.n_seq

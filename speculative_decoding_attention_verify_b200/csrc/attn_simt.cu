@@ -370,24 +370,25 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
     if (row >= total || row >= p.rows_cap) return;
     const int64_t stride = (int64_t)p.rows_cap * p.h_q;  // between splits, in (row, head) units
     const int64_t rh = (int64_t)row * p.h_q + h;
+    const int n_splits = p.n_splits;
     float o[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) o[e] = 0.f;
     float M = -INFINITY;
-    for (int s = lane; s < p.n_splits; s += 32) M = fmaxf(M, p.ws_ml[(s * stride + rh) * 2]);
+    for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, p.ws_ml[(s * stride + rh) * 2]);
     M = warp_max(M);
     float den = 0.f;
     if (M != -INFINITY) {
-        for (int s0 = 0; s0 < p.n_splits; s0 += 32) {
+        for (int s0 = 0; s0 < n_splits; s0 += 32) {
             const int s = s0 + lane;
             float w = 0.f, l = 0.f;
-            if (s < p.n_splits) {
+            if (s < n_splits) {
                 const float m = p.ws_ml[(s * stride + rh) * 2];
                 l = p.ws_ml[(s * stride + rh) * 2 + 1];
                 w = m == -INFINITY ? 0.f : exp2f(m - M);
             }
             den += warp_sum(w * l);
-            const int n = min(32, p.n_splits - s0);
+            const int n = min(32, n_splits - s0);
             int i = 0;
             for (; i + 4 <= n; i += 4) {
                 float ov[4][EPL];

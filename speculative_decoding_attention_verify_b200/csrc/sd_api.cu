@@ -147,6 +147,7 @@ AttnParams base_params(sd_attn_kind kind, const sd_q_desc *q, const void *q_data
     p.h_q = q->h_q;
     p.group = q->h_q / kv->h_kv;
     p.max_q_rows = q->max_q_rows;
+    p.max_kv_len = q->max_kv_len;
     p.rows_cap = batch * q->max_q_rows;
     const float scale = q->softmax_scale > 0.f ? q->softmax_scale
                                                : (float)(1.0 / sqrt((double)kv->head_dim));
@@ -295,7 +296,7 @@ sd_status sd_sparse_attention(const sd_q_desc *q, const void *q_data, const sd_k
     sd_status st = check_attention(SD_ATTN_SPARSE, q, kv, batch,
                                    stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail), &plan);
     if (st != SD_OK) return st;
-    plan.tensor_core = false;  // the sparse gather always runs on the CUDA-core engine
+    plan.tensor_core = false;  // the sparse gather runs on the CUDA-core engine
     if (plan.ws_bytes > workspace_bytes || (plan.ws_bytes && !workspace)) return SD_ERR_WORKSPACE;
     AttnParams p = base_params(SD_ATTN_SPARSE, q, q_data, kv, batch, out, plan, workspace, dev_err);
     p.idx = idx;

@@ -18,6 +18,7 @@ struct AttnParams {
     int h_q;
     int group;       // h_q / h_kv
     int max_q_rows;  // host hint
+    int max_kv_len;  // host hint: upper bound of every kv_len
     int rows_cap;    // batch * max_q_rows: rows addressable in the split workspace
     float scale_log2;  // softmax_scale * log2(e)
     const void *q;

@@ -17,7 +17,7 @@
 namespace sd {
 namespace {
 
-constexpr int kScoreThreads = 128;
+constexpr int kScoreThreads = 256;  // two threads per candidate of a tile
 constexpr int kSelectThreads = 1024;
 
 __device__ __forceinline__ unsigned long long score_key(double x) {
@@ -42,7 +42,7 @@ __device__ __forceinline__ void cand_range(const TopkParams &p, int b, int &cb, 
     if (bad && threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
 }
 
-constexpr int kScoreTile = 128;   // candidates per staged tile (one per thread)
+constexpr int kScoreTile = 128;   // candidates per staged tile
 constexpr int kScoreStages = 3;   // cp.async ring depth
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kScoreThreads) topk_score_kernel(const TopkPar
     constexpr int ROWB = D * ESZ;
     constexpr int NCHUNK = ROWB / 16;
     constexpr int SWZ = NCHUNK < 16 ? NCHUNK - 1 : 15;
-    static_assert(kScoreThreads == kScoreTile, "one candidate per thread");
+    static_assert(kScoreThreads == 2 * kScoreTile, "two threads per candidate");
     extern __shared__ __align__(128) uint8_t s_ring[];  // [stage][kScoreTile][ROWB]
     __shared__ double s_qbar[D];
     __shared__ int64_t s_off[kScoreStages][kScoreTile];
@@ -97,8 +97,11 @@ __global__ void __launch_bounds__(kScoreThreads) topk_score_kernel(const TopkPar
     const char *kbase = reinterpret_cast<const char *>(p.kv.k);
 
     auto map_tile = [&](int u) {
-        const int t = t_begin + u * kScoreTile + tid;
-        s_off[u % kScoreStages][tid] = t < t_end ? kv_row_offset(p.kv, b, g, cb + t, p.dev_err) : -1;
+        if (tid < kScoreTile) {
+            const int t = t_begin + u * kScoreTile + tid;
+            s_off[u % kScoreStages][tid] =
+                t < t_end ? kv_row_offset(p.kv, b, g, cb + t, p.dev_err) : -1;
+        }
     };
     auto issue_tile = [&](int u) {  // coalesced: consecutive threads take consecutive chunks
         const int st = u % kScoreStages;
@@ -124,26 +127,28 @@ __global__ void __launch_bounds__(kScoreThreads) topk_score_kernel(const TopkPar
         if (u < n_tiles) issue_tile(u);
         cp_async_commit();
         const int st = t % kScoreStages;
-        const int cand = t_begin + t * kScoreTile + tid;
-        if (cand < t_end) {
-            unsigned long long key = 0ull;
-            if (s_off[st][tid] >= 0) {
-                const uint8_t *rp = s_ring + (st * kScoreTile + tid) * ROWB;
-                double a[4] = {0.0, 0.0, 0.0, 0.0};  // independent chains
+        // thread pair (2c, 2c+1) scores candidate c of the tile: each takes half of the row
+        const int c = tid >> 1, half = tid & 1;
+        const int cand = t_begin + t * kScoreTile + c;
+        const bool valid = s_off[st][c] >= 0;
+        double a[4] = {0.0, 0.0, 0.0, 0.0};  // independent chains
+        if (cand < t_end && valid) {
+            const uint8_t *rp = s_ring + (st * kScoreTile + c) * ROWB;
 #pragma unroll
-                for (int ch = 0; ch < NCHUNK; ++ch) {
-                    const uint4 raw =
-                        *reinterpret_cast<const uint4 *>(rp + ((ch ^ (tid & SWZ)) << 4));
-                    float f[CH::kElems];
-                    CH::to_float(raw, f);
+            for (int k = 0; k < NCHUNK / 2; ++k) {
+                const int ch = half * (NCHUNK / 2) + k;
+                const uint4 raw = *reinterpret_cast<const uint4 *>(rp + ((ch ^ (c & SWZ)) << 4));
+                float f[CH::kElems];
+                CH::to_float(raw, f);
 #pragma unroll
-                    for (int e = 0; e < CH::kElems; ++e)
-                        a[e & 3] = fma((double)f[e], s_qbar[ch * CH::kElems + e], a[e & 3]);
-                }
-                key = score_key((a[0] + a[1]) + (a[2] + a[3]));
+                for (int e = 0; e < CH::kElems; ++e)
+                    a[e & 3] = fma((double)f[e], s_qbar[ch * CH::kElems + e], a[e & 3]);
             }
-            keys[cand] = key;
         }
+        const double part = (a[0] + a[1]) + (a[2] + a[3]);
+        const double other = __shfl_xor_sync(0xffffffffu, part, 1);
+        if (half == 0 && cand < t_end)
+            keys[cand] = valid ? score_key(part + other) : 0ull;  // first half + second half
         __syncthreads();
     }
     cp_async_wait<0>();

@@ -38,6 +38,11 @@ VERIFY_CASES = [
     (3, dict(layers=2, l_vis=2500, l_txt=300)),                # gamma 8: R = 63 rows
     (4, dict(l_vis=1500, l_txt=100, batch=5)),                 # paged, ragged gammas, NaN page tails
     (4, {}),                                                   # C4 full: 8 sequences up to 34.8k
+    (0, dict(dtype="bf16")),                                   # d=64, G=4: R = 20 (tensor cores)
+    (0, dict(dtype="bf16", l_vis=3000, l_txt=77, gamma=7)),    # d=64: R = 32 rows, ragged tail
+    (4, dict(l_vis=1500, l_txt=100, batch=5, gamma=2)),        # paged ragged, R = 21
+    (2, dict(layers=48, l_vis=600, l_txt=50, gamma=1)),        # 192 (sequence, KV head) units
+    (1, dict(l_vis=40, l_txt=9, gamma=3)),                     # a single tile
 ]
 
 
@@ -71,14 +76,28 @@ def test_verify_gamma0_equals_single_token_decode():
     _assert_close(out, ref, w.dtype, "gamma0")
 
 
-def test_verify_split_count_does_not_change_the_result():
+def test_verify_engines_and_schedules_agree():
+    """The same call under looser (still valid) host hints: a larger max_q_rows plans 56 rows
+    per KV head instead of 21; a larger max_kv_len plans another split of the positions.  All
+    must match the oracle."""
     w = gen.make_attn_workload(1, l_vis=6000, l_txt=200, gamma=2)
     kv = dev.kv_cache(w)
-    a = sd.sd_verify_attention(dev.verify_queries(w), kv)
-    q_small_hint = dev.queries(w.q_verify, w.q_verify_start, w.dtype, 256)  # forces one split
-    b = sd.sd_verify_attention(q_small_hint, kv)
-    diff = (a.float() - b.float()).abs().max().item()
-    assert diff <= 2e-2
+    ref = oracle.verify_attention(w.h_q, w.q_verify, w.q_verify_start, oracle.cache_from_workload(w))
+    n = int(w.kv_len_verify.max())
+    base = dev.verify_queries(w)
+    variants = {
+        "default": base,
+        "rows8": sd.Queries(base.q, base.q_start, max_q_rows=8, max_kv_len=n),
+        "len4x": sd.Queries(base.q, base.q_start, max_q_rows=base.desc.max_q_rows,
+                            max_kv_len=4 * n),
+    }
+    outs = {}
+    for name, q in variants.items():
+        outs[name] = sd.sd_verify_attention(q, kv)
+        _assert_close(outs[name], ref, w.dtype, name)
+    for name in ("rows8", "len4x"):
+        diff = (outs[name].float() - outs["default"].float()).abs().max().item()
+        assert diff <= 2e-2, name
 
 
 def test_verify_is_deterministic():
@@ -89,8 +108,9 @@ def test_verify_is_deterministic():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-def test_verify_bad_page_sets_flag_without_fault():
-    w = gen.make_attn_workload(4, l_vis=500, l_txt=40, batch=2)
+@pytest.mark.parametrize("gamma", [None, 2])   # R = 56 and R = 21 rows per KV head
+def test_verify_bad_page_sets_flag_without_fault(gamma):
+    w = gen.make_attn_workload(4, l_vis=500, l_txt=40, batch=2, gamma=gamma)
     bt = w.block_table.copy()
     bt[1, 3] = w.num_pages + 5  # out of the pool
     kv = dev.kv_cache(w)
@@ -128,6 +148,8 @@ TA_CASES = [
     (2, dict(layers=4, l_vis=3000), {}),
     (4, dict(l_vis=2000, l_txt=300, batch=6), {}),
     (4, {}, {}),
+    (0, dict(dtype="bf16", l_vis=2000, l_txt=500), dict(window=300)),     # d=64 tensor cores
+    (2, dict(layers=40, l_vis=2000, l_txt=900), dict(vis=(100, 1500), window=1000)),
 ]
 
 
@@ -167,6 +189,8 @@ SPARSE_CASES = [
     (3, dict(layers=3, l_vis=5000, l_txt=600), 2),
     (4, dict(l_vis=3000, l_txt=200, batch=5), 0),
     (4, {}, 1),
+    (0, dict(dtype="bf16", l_vis=2000, l_txt=100), 3),                     # d=64
+    (2, dict(layers=40, l_vis=3000, l_txt=300), 5),                        # 160 units
 ]
 
 
