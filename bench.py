@@ -62,14 +62,14 @@ def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "speculative_decoding_attention_verify_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.startswith("attn_") or name in ("sd_common.cuh", "sd_internal.h"):
+        if name.startswith("attn_") or name in ("sd_common.cuh", "sd_internal.h", "tc_ptx.cuh"):
             h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:12]
 
 
 def recorded_traffic():
     """DRAM bytes per verify launch from the committed ncu summary, if the kernel is unchanged."""
-    path = os.path.join(ROOT, "profiles", "verify_attention_c2_ncu.md")
+    path = os.path.join(ROOT, "profiles", "verify_attention_c3_ncu.md")
     try:
         text = open(path).read()
     except OSError:
@@ -163,11 +163,13 @@ class Cycle:
         mk = lambda n: torch.empty(max(int(n), 16), dtype=torch.uint8, device=device)
         self.ws_verify = mk(sd.sd_attention_workspace_size(sd.SD_ATTN_VERIFY, self.q_verify,
                                                            self.kv_verify))
-        self.ws_sparse = mk(sd.sd_attention_workspace_size(sd.SD_ATTN_SPARSE, self.q_draft[-1],
-                                                           self.kv_draft[-1]))
+        self.ws_sparse = mk(sd.sd_sparse_workspace_size(self.q_draft[-1], self.kv_draft[-1],
+                                                        w.topk, self.max_tail))
         self.ws_ta = mk(sd.sd_attention_workspace_size(sd.SD_ATTN_TEXT_ANCHORED, self.q_draft[-1],
                                                        self.kv_draft[-1]))
         self.ws_topk = mk(sd.sd_topk_workspace_size(self.kv_verify, int(w.l_vis.max()), w.topk))
+        # the top-K rows are staged once per cycle and read by every draft step
+        self.sel = mk(sd.sd_sparse_selection_size(self.kv_draft[0], w.topk))
         self.ws_acc = mk(sd.sd_accept_workspace_size(1, g, aw.vocab))
         self.n_acc_g = torch.empty(1, dtype=torch.int32, device=device)
         self.out_g = torch.empty((1, g + 1), dtype=torch.int32, device=device)
@@ -177,21 +179,36 @@ class Cycle:
         self.bytes = cycle_bytes(w, self.lens_draft, w.topk)
         self.verify_events = []
 
-    def launches_per_step(self):
-        merge = lambda ws: 1 if ws.numel() > 16 else 0
+    def launches_per_step(self, graph=None):
+        """Kernels one step launches: counted from the captured CUDA graph (kernel nodes; every
+        kernel of the step is libsdattn's), else an upper bound from the call structure."""
+        if graph is not None:
+            try:
+                from cuda.bindings import runtime as rt
+                h = rt.cudaGraph_t(init_value=int(graph.raw_cuda_graph()))
+                err, _, n = rt.cudaGraphGetNodes(h, 0)
+                err2, nodes, n = rt.cudaGraphGetNodes(h, n)
+                if err == rt.cudaError_t.cudaSuccess and err2 == rt.cudaError_t.cudaSuccess:
+                    kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+                    return sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel)
+            except Exception:  # noqa: BLE001 - fall back to the structural count
+                pass
         g = self.gamma
-        return (2 + g * (1 + merge(self.ws_sparse)) + g + g * (1 + merge(self.ws_ta)) +
-                (1 + merge(self.ws_verify)) + 2 + 4)
+        # top-K (score, select), staging; per draft step sparse (attention, merge), HSR,
+        # text-anchored (attention, merge); verify (attention, merge); greedy (2); sampling (4)
+        return 2 + 1 + g * 2 + g + g * 2 + 2 + 2 + 4
 
     def step(self, stream=None, time_verify=False):
         sd = self.sd
         sd.sd_topk_select(self.q_verify, self.kv_verify, self.cand_b, self.cand_e,
                           int(self.w.l_vis.max()), self.topk, idx_out=self.idx,
                           workspace=self.ws_topk, stream=stream)
+        sd.sd_sparse_stage(self.kv_draft[0], self.idx, self.tail, selection=self.sel,
+                           stream=stream)
         for t in range(self.gamma):
-            sd.sd_sparse_attention(self.q_draft[t], self.kv_draft[t], self.idx, self.tail,
-                                   self.max_tail, out=self.o_draft[t], workspace=self.ws_sparse,
-                                   stream=stream)
+            sd.sd_sparse_attention_staged(self.q_draft[t], self.kv_draft[t], self.sel, self.topk,
+                                          self.tail, self.max_tail, out=self.o_draft[t],
+                                          workspace=self.ws_sparse, stream=stream)
             sd.sd_hsr_project(self.emb[t], self.hid, self.W, out=self.y, stream=stream)
             sd.sd_text_anchored_attention(self.q_draft[t], self.kv_draft[t], self.vis_b,
                                           self.vis_e, self.win, int(self.w.window.max()),
@@ -429,7 +446,7 @@ def run_ours(args):
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": host.h2d_bytes, "d2h_bytes_per_step": host.d2h_bytes,
                     "ms_per_step": round(e2e_ms / args.steps, 4)},
-            "gpu_launches": cyc.launches_per_step() * args.steps,
+            "gpu_launches": cyc.launches_per_step(graph) * args.steps,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }

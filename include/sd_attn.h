@@ -134,8 +134,9 @@ SD_API const char *sd_status_string(sd_status s);
 SD_API int32_t sd_version(void);
 
 /*
- * Workspace bytes an attention call of `kind` needs for these descriptors (host hints only;
- * device arrays are not read).  A call may be given more.  *bytes may be 0.
+ * Workspace bytes a verify or text-anchored call needs for these descriptors (host hints only;
+ * device arrays are not read).  A call may be given more.  *bytes may be 0.  SD_ATTN_SPARSE is
+ * rejected (SD_ERR_INVALID_ARG): its size depends on k, see sd_sparse_workspace_size.
  */
 SD_API sd_status sd_attention_workspace_size(sd_attn_kind kind, const sd_q_desc *q,
                                       const sd_kv_desc *kv, int32_t batch, size_t *bytes);
@@ -171,6 +172,15 @@ SD_API sd_status sd_text_anchored_attention(const sd_q_desc *q, const void *q_da
                                      void *stream);
 
 /*
+ * Workspace bytes of sd_sparse_attention with these descriptors, k list entries and the
+ * max_tail hint (host values only).  For bf16 caches it includes the staging of the selected
+ * rows: batch * h_kv * k * head_dim * 2 bytes for K and as much for V, plus their positions.
+ */
+SD_API sd_status sd_sparse_workspace_size(const sd_q_desc *q, const sd_kv_desc *kv,
+                                          int32_t batch, int32_t k, int32_t max_tail,
+                                          size_t *bytes);
+
+/*
  * Sparse draft attention [StD "Metodologia"]: the sparse model attends only to the selected
  * top-K KV entries plus the dense tail.  For row i of sequence b and KV head g the allowed
  * set is ({idx[b][g][0..k)} U [tail_begin[b], limit]) restricted to j <= limit,
@@ -178,12 +188,45 @@ SD_API sd_status sd_text_anchored_attention(const sd_q_desc *q, const void *q_da
  * entries are padding and ignored; entries >= tail_begin are covered by the tail; a
  * non-ascending list sets SD_DEVERR_INDEX and repeated entries are skipped.
  * tail_begin: device int32 [batch].  max_tail: host hint >= kv_len[b] - tail_begin[b].
+ * bf16 caches: the kept entries' K and V rows are first copied, in list order, into the
+ * workspace, and the tensor-core kernel streams that compact run and the tail.  The workspace
+ * (sd_sparse_workspace_size) must not be shared with a call in flight.
  */
 SD_API sd_status sd_sparse_attention(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
                               int32_t batch, const int32_t *idx, int32_t k,
                               const int32_t *tail_begin, int32_t max_tail, void *out,
                               void *workspace, size_t workspace_bytes, int32_t *dev_err,
                               void *stream);
+
+/*
+ * Staged sparse selection [StD "Metodologia": the top-K KV entries are chosen once and reused
+ * by every draft step].  sd_sparse_stage copies, for every (sequence, KV head), the K and V
+ * rows of the entries of idx that sd_sparse_attention would use (0 <= x < tail_begin[b], not
+ * equal to the entry before; a non-ascending list sets SD_DEVERR_INDEX) into `selection`,
+ * in list order, with their positions and counts.  sd_sparse_attention_staged then computes
+ * exactly what sd_sparse_attention computes for that idx, reading the staged rows instead of
+ * gathering them again; the selection stays valid while idx, tail_begin and the selected cache
+ * rows are unchanged (the draft steps of one cycle append only to the tail).
+ *
+ * selection: device memory of sd_sparse_selection_size bytes, 256-byte aligned, owned by the
+ * caller.  k must be the same in the three calls.  bf16 caches, head_dim 64 or 128 and at most
+ * 128 rows per KV head; otherwise SD_ERR_UNSUPPORTED (use sd_sparse_attention).  The staged
+ * attention's workspace: sd_attention_workspace_size is not used; pass
+ * sd_sparse_workspace_size(...) bytes or more.
+ */
+SD_API sd_status sd_sparse_selection_size(const sd_kv_desc *kv, int32_t batch, int32_t k,
+                                          size_t *bytes);
+
+SD_API sd_status sd_sparse_stage(const sd_kv_desc *kv, int32_t batch, const int32_t *idx,
+                                 int32_t k, const int32_t *tail_begin, void *selection,
+                                 size_t selection_bytes, int32_t *dev_err, void *stream);
+
+SD_API sd_status sd_sparse_attention_staged(const sd_q_desc *q, const void *q_data,
+                                            const sd_kv_desc *kv, int32_t batch,
+                                            const void *selection, int32_t k,
+                                            const int32_t *tail_begin, int32_t max_tail,
+                                            void *out, void *workspace, size_t workspace_bytes,
+                                            int32_t *dev_err, void *stream);
 
 /*
  * Workspace for sd_topk_select.  max_cand: host hint >= cand_end[b] - cand_begin[b].

@@ -92,8 +92,18 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     // The unit's position stream as at most two runs [s0, s0+len0) and [s1, s1+len1) (verify:
     // [0, kv_len); text-anchored: the non-visual positions from the lowest windowed one).  Each
     // run is tiled from a0 (a1): its start, or the page boundary below it for paged caches.
-    const StreamInfo si = stream_setup<kThreads>(p, b, g, n_q, kv_len, s_stream);
-    const int a0 = PAGED ? (si.s0 & ~(kPageSize - 1)) : si.s0;
+    // Sparse: run 0 is the compacted selection [0, k_eff) in its own buffer, run 1 the tail.
+    const bool sparse = p.kind == SD_ATTN_SPARSE;
+    StreamInfo si{};
+    if (sparse) {
+        si.s0 = 0;
+        si.len0 = __ldg(p.k_eff + b * kv.h_kv + g);
+        si.s1 = min(max(__ldg(p.tail_begin + b), 0), kv_len);
+        si.len1 = kv_len - si.s1;
+    } else {
+        si = stream_setup<kThreads>(p, b, g, n_q, kv_len, s_stream);
+    }
+    const int a0 = (PAGED && !sparse) ? (si.s0 & ~(kPageSize - 1)) : si.s0;
     const int a1 = PAGED ? (si.s1 & ~(kPageSize - 1)) : si.s1;
     const int nt0 = si.len0 > 0 ? (si.s0 + si.len0 - a0 + kTile - 1) / kTile : 0;
     const int nt1 = si.len1 > 0 ? (si.s1 + si.len1 - a1 + kTile - 1) / kTile : 0;
@@ -157,9 +167,11 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             for (int t = 0; t < n_my; ++t) {
                 const int s = t % S, use = t / S;
                 const int p0 = tile_start(tile_lo + t);
+                // compacted sparse selection: its own contiguous buffer
+                const bool cmp = sparse && tile_lo + t < nt0;
                 const uint32_t dK = saddr(sKV + (size_t)s * 2 * C::kTileBytes);
                 const uint32_t dV = dK + C::kTileBytes;
-                if (PAGED) {
+                if (PAGED && !cmp) {
                     for (int pg = 0; pg < kTile / kPageSize; ++pg) {
                         const int pos = p0 + pg * kPageSize;
                         int page = kv.num_pages;  // out of range: zero-filled box
@@ -177,11 +189,12 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 for (int half = 0; half < 2; ++half) {  // K, then V
                     const int full = half == 0 ? KF : VF, empty = half == 0 ? KE : VE;
                     const uint32_t dst = half == 0 ? dK : dV;
-                    const CUtensorMap *map = half == 0 ? &maps.k : &maps.v;
+                    const CUtensorMap *map = cmp ? (half == 0 ? &maps.k2 : &maps.v2)
+                                                 : (half == 0 ? &maps.k : &maps.v);
                     if (t >= S && !mbar_wait(BAR(empty + s), (use - 1) & 1, abort_flag, p.dev_err))
                         break;
                     mbar_arrive_tx(BAR(full + s), C::kTileBytes);
-                    if (!PAGED) {
+                    if (!PAGED || cmp) {
 #pragma unroll
                         for (int h = 0; h < C::kHalves; ++h)
                             tma_load_4d(dst + h * kHalfBytes, map, BAR(full + s), h * 64, p0, g, b);
@@ -240,7 +253,10 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             // V rows past the end of the sequence may hold anything (NaN included): zero
             // them so that 0 * V cannot poison O.
             uint8_t *vs = sKV + (size_t)s * 2 * C::kTileBytes + C::kTileBytes;
-            const int valid = min(kTile, kv_len - tile_start(tile_lo + t));
+            // (rows past the run's end in its tensor: the sequence end, or the compacted count)
+            const int tt = tile_lo + t;
+            const int run_hi = tt < nt0 ? si.s0 + si.len0 : si.s1 + si.len1;
+            const int valid = max(0, min(kTile, run_hi - tile_start(tt)));
             if (valid < kTile) {
                 const int nchunk = (kTile - valid) * 8;  // 16-byte chunks per half
                 for (int h = 0; h < C::kHalves; ++h)
@@ -297,6 +313,12 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 w2 = (uint32_t)(y2 - x2);
             }
         }
+        // Sparse: every selected position is below the tail; when the tail starts at or below
+        // the smallest row limit + 1, every row sees the whole selection, else the compacted
+        // positions are tested one by one.
+        const bool sel_all = !sparse || si.s1 <= kv_len - n_q + 1;
+        const uint32_t row_ok_u = row_ok ? 1u : 0u;
+        const int32_t *cpos = sparse ? p.cpos + ((int64_t)b * kv.h_kv + g) * p.k_cap : nullptr;
         const float sl2 = p.scale_log2;
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
         float m_used = -INFINITY, l = 0.f;
@@ -319,20 +341,40 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             tmem_ld128(s_addr, v);
             // Interior tiles (inside the run and visible in full to every row of this warp)
             // skip masking.
+            // (tiles of the compacted selection are in list coordinates: the positions are
+            // cpos[...], all below the tail)
+            const bool cmp = sparse && tt < nt0;
             const bool in_run = p0 >= seg_lo && p0 + kTile <= seg_hi;
             const uint32_t d1 = (uint32_t)p0 - lo1, d2 = (uint32_t)p0 - lo2;
-            const bool whole = !row_ok || (w1 >= kTile - 1 && d1 <= w1 - (kTile - 1)) ||
-                               (w2 >= kTile - 1 && d2 <= w2 - (kTile - 1));
+            const bool whole = !row_ok || (cmp ? sel_all
+                                               : ((w1 >= kTile - 1 && d1 <= w1 - (kTile - 1)) ||
+                                                  (w2 >= kTile - 1 && d2 <= w2 - (kTile - 1))));
             const bool interior = __all_sync(FULL, in_run && whole);
             float mx = -INFINITY;
             if (!interior) {
                 const uint32_t seg_w = (uint32_t)(seg_hi - seg_lo);
+                if (!cmp) {
 #pragma unroll
-                for (int e = 0; e < kTile; ++e) {
-                    const uint32_t j = (uint32_t)(p0 + e);
-                    const uint32_t vis = (j - (uint32_t)seg_lo < seg_w) &
-                                         ((j - lo1 <= w1) | (j - lo2 <= w2));
-                    v[e] = vis ? v[e] : -INFINITY;
+                    for (int e = 0; e < kTile; ++e) {
+                        const uint32_t j = (uint32_t)(p0 + e);
+                        const uint32_t vis = (j - (uint32_t)seg_lo < seg_w) &
+                                             ((j - lo1 <= w1) | (j - lo2 <= w2));
+                        v[e] = vis ? v[e] : -INFINITY;
+                    }
+                } else if (sel_all) {
+#pragma unroll
+                    for (int e = 0; e < kTile; ++e) {
+                        const uint32_t vis = ((uint32_t)(p0 + e) < seg_w) & row_ok_u;
+                        v[e] = vis ? v[e] : -INFINITY;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < kTile; ++e) {
+                        const bool in = p0 + e < (int)seg_w;
+                        const uint32_t j = in ? (uint32_t)__ldg(cpos + p0 + e) : 0u;
+                        const uint32_t vis = (uint32_t)in & (j - lo1 <= w1);
+                        v[e] = vis ? v[e] : -INFINITY;
+                    }
                 }
             }
 #pragma unroll
@@ -531,12 +573,25 @@ bool encode_kv_maps(const AttnParams &p, int max_kv_len, TcMaps *maps) {
     CUresult rv = enc(&maps->v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(kv.v), dims,
                       strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return rk == CUDA_SUCCESS && rv == CUDA_SUCCESS;
+    if (rk != CUDA_SUCCESS || rv != CUDA_SUCCESS) return false;
+    if (p.kind != SD_ATTN_SPARSE) return true;
+    // compacted selection [batch][h_kv][k_cap][d]
+    const cuuint64_t kc = (cuuint64_t)(p.k_cap > 0 ? p.k_cap : 1);
+    const cuuint64_t cdims[4] = {d, kc, (cuuint64_t)kv.h_kv, (cuuint64_t)p.batch};
+    const cuuint64_t cstr[3] = {d * 2, kc * d * 2, (cuuint64_t)kv.h_kv * kc * d * 2};
+    const cuuint32_t cbox[4] = {64, kTile, 1, 1};
+    CUresult ck = enc(&maps->k2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.ck, cdims, cstr, cbox, elem,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult cv = enc(&maps->v2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.cv, cdims, cstr, cbox, elem,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return ck == CUDA_SUCCESS && cv == CUDA_SUCCESS;
 }
 
 bool tc_supported(int kind, int dtype, int head_dim, int rows) {
-    return (kind == SD_ATTN_VERIFY || kind == SD_ATTN_TEXT_ANCHORED) && dtype == SD_BF16 &&
-           (head_dim == 64 || head_dim == 128) && rows >= 1 && rows <= kRows;
+    return dtype == SD_BF16 && (head_dim == 64 || head_dim == 128) && rows >= 1 &&
+           rows <= kRows;  // every kind (sparse through the compacted selection)
 }
 
 cudaError_t launch_attention_tc(const AttnParams &p, const AttnPlan &plan, cudaStream_t s) {

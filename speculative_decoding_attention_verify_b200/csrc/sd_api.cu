@@ -53,20 +53,20 @@ AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, in
             }
         }
     }
-    // Tensor-core decomposition: one CTA per SM; pick the split count whose CTAs fill whole
-    // waves best, keeping at least two 128-position tiles per CTA.
+    // Tensor-core decomposition: one CTA per SM.  Modelled time of split count s: waves x
+    // (per-CTA start-up and drain, about three tiles' worth, + tiles per CTA); the smallest wins.
     plan.tc_splits = 1;
     if (plan.tensor_core) {
         const long long units = (long long)batch * h_kv;
         const long long tiles = (max_stream + 127) / 128;
-        double best = -1.0;
+        long long best = -1;
         for (long long s = 1; s <= 64; ++s) {
             if (s > 1 && tiles / s < 2) break;
             const long long ctas = units * s;
             const long long waves = (ctas + sms - 1) / sms;
-            const double score = (double)ctas / (double)(waves * sms) - 0.003 * (double)s;
-            if (score > best) {
-                best = score;
+            const long long t = waves * (3 + (tiles + s - 1) / s);
+            if (best < 0 || t < best) {
+                best = t;
                 plan.tc_splits = (int)s;
             }
         }
@@ -186,6 +186,40 @@ sd_status run_attention(AttnParams p, const AttnPlan &plan, void *stream) {
     return cuda_status(e);
 }
 
+// A staged sparse selection: K, V [batch][h_kv][k_cap][d] bf16, positions [batch][h_kv][k_cap]
+// and per-unit counts, from offset `base`; each region 256-byte aligned.
+struct SelLayout {
+    size_t ck, cv, cpos, k_eff, end;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+SelLayout sel_layout(size_t base, const sd_kv_desc *kv, int batch, int k) {
+    SelLayout l{};
+    const size_t units = (size_t)batch * kv->h_kv, kc = (size_t)(k > 0 ? k : 1);
+    l.ck = up256(base);
+    l.cv = l.ck + up256(units * kc * kv->head_dim * 2);
+    l.cpos = l.cv + up256(units * kc * kv->head_dim * 2);
+    l.k_eff = l.cpos + up256(units * kc * 4);
+    l.end = l.k_eff + up256(units * 4);
+    return l;
+}
+
+void set_selection(AttnParams &p, void *base, const SelLayout &l, int k) {
+    char *w = static_cast<char *>(base);
+    p.ck = w + l.ck;
+    p.cv = w + l.cv;
+    p.cpos = reinterpret_cast<int32_t *>(w + l.cpos);
+    p.k_eff = reinterpret_cast<int32_t *>(w + l.k_eff);
+    p.k_cap = k > 0 ? k : 1;
+}
+
+// Workspace bytes of sd_sparse_attention: the split partials, plus a staged selection when
+// the tensor-core path is planned.
+size_t sparse_ws_bytes(const AttnPlan &plan, const sd_kv_desc *kv, int batch, int k) {
+    return plan.tensor_core ? sel_layout(plan.ws_bytes, kv, batch, k).end : plan.ws_bytes;
+}
+
 long long stream_hint(sd_attn_kind kind, const sd_q_desc *q, long long extra) {
     if (kind == SD_ATTN_TEXT_ANCHORED) {
         const long long w = extra + q->max_q_rows - 1;
@@ -237,8 +271,8 @@ int32_t sd_version(void) { return 100; }
 sd_status sd_attention_workspace_size(sd_attn_kind kind, const sd_q_desc *q,
                                       const sd_kv_desc *kv, int32_t batch, size_t *bytes) {
     if (!bytes || !q || !kv) return SD_ERR_INVALID_ARG;
-    if (kind != SD_ATTN_VERIFY && kind != SD_ATTN_TEXT_ANCHORED && kind != SD_ATTN_SPARSE)
-        return SD_ERR_INVALID_ARG;
+    // (sparse calls also stage the selected rows: see sd_sparse_workspace_size)
+    if (kind != SD_ATTN_VERIFY && kind != SD_ATTN_TEXT_ANCHORED) return SD_ERR_INVALID_ARG;
     if (kv->h_kv < 1 || q->h_q < 1 || q->h_q % kv->h_kv || batch < 1 || q->max_q_rows < 1)
         return SD_ERR_INVALID_ARG;
     if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
@@ -283,6 +317,20 @@ sd_status sd_text_anchored_attention(const sd_q_desc *q, const void *q_data,
     return run_attention(p, plan, stream);
 }
 
+sd_status sd_sparse_workspace_size(const sd_q_desc *q, const sd_kv_desc *kv, int32_t batch,
+                                   int32_t k, int32_t max_tail, size_t *bytes) {
+    if (!bytes || !q || !kv || k < 0 || k > (1 << 16) || max_tail < 0) return SD_ERR_INVALID_ARG;
+    if (kv->h_kv < 1 || q->h_q < 1 || q->h_q % kv->h_kv || batch < 1 || q->max_q_rows < 1 ||
+        q->max_kv_len < 1)
+        return SD_ERR_INVALID_ARG;
+    if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
+    const AttnPlan plan = plan_attention(SD_ATTN_SPARSE, kv->dtype, kv->head_dim, q->h_q,
+                                         kv->h_kv, batch, q->max_q_rows,
+                                         stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail));
+    *bytes = sparse_ws_bytes(plan, kv, batch, k);
+    return SD_OK;
+}
+
 sd_status sd_sparse_attention(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
                               int32_t batch, const int32_t *idx, int32_t k,
                               const int32_t *tail_begin, int32_t max_tail, void *out,
@@ -296,13 +344,85 @@ sd_status sd_sparse_attention(const sd_q_desc *q, const void *q_data, const sd_k
     sd_status st = check_attention(SD_ATTN_SPARSE, q, kv, batch,
                                    stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail), &plan);
     if (st != SD_OK) return st;
-    plan.tensor_core = false;  // the sparse gather runs on the CUDA-core engine
-    if (plan.ws_bytes > workspace_bytes || (plan.ws_bytes && !workspace)) return SD_ERR_WORKSPACE;
+    const size_t need = sparse_ws_bytes(plan, kv, batch, k);
+    if (need > workspace_bytes || (need && !workspace)) return SD_ERR_WORKSPACE;
     AttnParams p = base_params(SD_ATTN_SPARSE, q, q_data, kv, batch, out, plan, workspace, dev_err);
     p.idx = idx;
     p.k_sel = k;
     p.tail_begin = tail_begin;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(q_data) | reinterpret_cast<uintptr_t>(out)) &
+                          15) == 0;
+    if (plan.tensor_core && aligned) {
+        // tensor-core path: stage the selected rows, then stream [selection ; tail]
+        set_selection(p, workspace, sel_layout(plan.ws_bytes, kv, batch, k), k);
+        const cudaError_t e = launch_sparse_compact(p, reinterpret_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return SD_ERR_CUDA;
+    } else {
+        plan.tensor_core = false;
+    }
     return run_attention(p, plan, stream);
+}
+
+sd_status sd_sparse_selection_size(const sd_kv_desc *kv, int32_t batch, int32_t k,
+                                   size_t *bytes) {
+    if (!bytes || !kv || batch < 1 || k < 0 || k > (1 << 16) || kv->h_kv < 1)
+        return SD_ERR_INVALID_ARG;
+    if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
+    *bytes = sel_layout(0, kv, batch, k).end;
+    return SD_OK;
+}
+
+sd_status sd_sparse_stage(const sd_kv_desc *kv, int32_t batch, const int32_t *idx, int32_t k,
+                          const int32_t *tail_begin, void *selection, size_t selection_bytes,
+                          int32_t *dev_err, void *stream) {
+    if (!tail_begin || k < 0 || (k > 0 && !idx) || k > (1 << 16) || batch < 1 || batch > 65535)
+        return SD_ERR_INVALID_ARG;
+    if (!kv_desc_ok(kv, batch)) return SD_ERR_INVALID_ARG;
+    if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
+    if (kv->dtype != SD_BF16) return SD_ERR_UNSUPPORTED;
+    const SelLayout l = sel_layout(0, kv, batch, k);
+    if (!selection || l.end > selection_bytes || (reinterpret_cast<uintptr_t>(selection) & 255))
+        return SD_ERR_WORKSPACE;
+    AttnParams p{};
+    p.kind = SD_ATTN_SPARSE;
+    p.kv = make_view(kv);
+    p.batch = batch;
+    p.idx = idx;
+    p.k_sel = k;
+    p.tail_begin = tail_begin;
+    p.dev_err = dev_err;
+    set_selection(p, selection, l, k);
+    return cuda_status(launch_sparse_compact(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sd_status sd_sparse_attention_staged(const sd_q_desc *q, const void *q_data,
+                                     const sd_kv_desc *kv, int32_t batch, const void *selection,
+                                     int32_t k, const int32_t *tail_begin, int32_t max_tail,
+                                     void *out, void *workspace, size_t workspace_bytes,
+                                     int32_t *dev_err, void *stream) {
+    if (!q || !q_data || !out || !tail_begin || !selection || k < 0 || max_tail < 0 ||
+        k > (1 << 16))
+        return SD_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(selection) & 255) ||
+        ((reinterpret_cast<uintptr_t>(q_data) | reinterpret_cast<uintptr_t>(out)) & 15))
+        return SD_ERR_INVALID_ARG;
+    AttnPlan plan;
+    sd_status st = check_attention(SD_ATTN_SPARSE, q, kv, batch,
+                                   stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail), &plan);
+    if (st != SD_OK) return st;
+    if (!plan.tensor_core) return SD_ERR_UNSUPPORTED;  // bf16, head_dim 64/128, <= 128 rows
+    if (plan.ws_bytes > workspace_bytes || (plan.ws_bytes && !workspace)) return SD_ERR_WORKSPACE;
+    AttnParams p = base_params(SD_ATTN_SPARSE, q, q_data, kv, batch, out, plan, workspace, dev_err);
+    p.k_sel = k;
+    p.tail_begin = tail_begin;
+    set_selection(p, const_cast<void *>(selection), sel_layout(0, kv, batch, k), k);
+    set_splits(p, plan.tc_splits);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_attention_tc(p, plan, s);
+    if (e == cudaErrorNotSupported) return SD_ERR_UNSUPPORTED;
+    if (e != cudaSuccess) return SD_ERR_CUDA;
+    if (p.n_splits > 1) e = launch_attention_merge(p, s);
+    return cuda_status(e);
 }
 
 sd_status sd_topk_workspace_size(const sd_kv_desc *kv, int32_t batch, int32_t max_cand,

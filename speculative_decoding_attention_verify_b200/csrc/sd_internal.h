@@ -32,6 +32,11 @@ struct AttnParams {
     const int32_t *idx;
     int k_sel;
     const int32_t *tail_begin;
+    // sparse, tensor-core path: the selected rows compacted per (sequence, KV head)
+    void *ck, *cv;     // [batch][h_kv][k_cap][head_dim] bf16
+    int32_t *cpos;     // [batch][h_kv][k_cap] their positions
+    int32_t *k_eff;    // [batch][h_kv] kept entries
+    int k_cap;
     // split-KV decomposition
     int n_splits;
     int n_rowblocks;
@@ -59,6 +64,7 @@ AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, in
 
 cudaError_t launch_attention_simt(const AttnParams &p, const AttnPlan &plan, cudaStream_t s);
 cudaError_t launch_attention_tc(const AttnParams &p, const AttnPlan &plan, cudaStream_t s);
+cudaError_t launch_sparse_compact(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_attention_merge(const AttnParams &p, cudaStream_t s);
 bool tc_supported(int kind, int dtype, int head_dim, int rows);
 

@@ -11,13 +11,17 @@ namespace sd {
 
 // TMA descriptors of the K and V caches: contiguous caches as (d, capacity, h_kv, batch) with
 // 64 x 128 boxes, paged caches as (d, 16, h_kv, pages) with 64 x 16 boxes; 128-byte swizzle.
+// k2 / v2 describe the compacted sparse selection (d, k_cap, h_kv, batch) when used.
 struct TcMaps {
     CUtensorMap k;
     CUtensorMap v;
+    CUtensorMap k2;
+    CUtensorMap v2;
 };
 
-// Encodes the maps of p.kv (bf16); false when the driver entry point is missing or the layout
-// cannot be described (the caller then uses another engine).
+// Encodes the maps of p.kv (bf16), and for sparse calls those of p.ck / p.cv; false when the
+// driver entry point is missing or a layout cannot be described (the caller then uses another
+// engine).
 bool encode_kv_maps(const AttnParams &p, int max_kv_len, TcMaps *maps);
 
 namespace tc {

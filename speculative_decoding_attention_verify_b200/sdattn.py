@@ -51,7 +51,8 @@ class sd_q_desc(ctypes.Structure):
 EXPORTS = ("sd_status_string", "sd_version", "sd_attention_workspace_size", "sd_verify_attention",
            "sd_text_anchored_attention", "sd_sparse_attention", "sd_topk_workspace_size",
            "sd_topk_select", "sd_hsr_project", "sd_accept_workspace_size", "sd_accept_greedy",
-           "sd_accept_sample", "sd_verify_attention_noalloc")
+           "sd_accept_sample", "sd_verify_attention_noalloc", "sd_sparse_workspace_size",
+           "sd_sparse_selection_size", "sd_sparse_stage", "sd_sparse_attention_staged")
 
 # Size of the library's fixed scratch used by sd_verify_attention_noalloc.
 SD_VERIFY_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -83,6 +84,11 @@ def lib():
                 h.sd_accept_sample.argtypes = [P, P, P, P, P, P, I32, I32, I32, P, P, I32, P, P, SZ,
                                                P, P]
                 h.sd_verify_attention_noalloc.argtypes = [P, P, P, I32, P, P, P]
+                h.sd_sparse_workspace_size.argtypes = [P, P, I32, I32, I32, ctypes.POINTER(SZ)]
+                h.sd_sparse_selection_size.argtypes = [P, I32, I32, ctypes.POINTER(SZ)]
+                h.sd_sparse_stage.argtypes = [P, I32, P, I32, P, P, SZ, P, P]
+                h.sd_sparse_attention_staged.argtypes = [P, P, P, I32, P, I32, P, I32, P, P, SZ,
+                                                         P, P]
                 for name in EXPORTS[2:]:
                     getattr(h, name).restype = ctypes.c_int
                 _LIB = h
@@ -234,11 +240,52 @@ def sd_text_anchored_attention(q: Queries, kv: KVCache, vis_begin, vis_end, wind
 def sd_sparse_attention(q: Queries, kv: KVCache, idx: torch.Tensor, tail_begin, max_tail: int,
                         out=None, workspace=None, dev_err=None, stream=None) -> torch.Tensor:
     out = _attn_out(q, out)
-    ws = _workspace(sd_attention_workspace_size(SD_ATTN_SPARSE, q, kv), q.q.device, workspace)
+    ws = _workspace(sd_sparse_workspace_size(q, kv, int(idx.shape[-1]), max_tail), q.q.device,
+                    workspace)
     _check(lib().sd_sparse_attention(
         ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(idx),
         int(idx.shape[-1]), _ptr(tail_begin), int(max_tail), _ptr(out), _ptr(ws), ws.numel(),
         _ptr(dev_err), _stream(stream)), "sd_sparse_attention")
+    return out
+
+
+def sd_sparse_workspace_size(q: Queries, kv: KVCache, k: int, max_tail: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().sd_sparse_workspace_size(ctypes.byref(q.desc), ctypes.byref(kv.desc), kv.batch,
+                                          int(k), int(max_tail), ctypes.byref(n)),
+           "sd_sparse_workspace_size")
+    return n.value
+
+
+def sd_sparse_selection_size(kv: KVCache, k: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().sd_sparse_selection_size(ctypes.byref(kv.desc), kv.batch, int(k),
+                                          ctypes.byref(n)), "sd_sparse_selection_size")
+    return n.value
+
+
+def sd_sparse_stage(kv: KVCache, idx: torch.Tensor, tail_begin, selection=None, dev_err=None,
+                    stream=None) -> torch.Tensor:
+    """Stages the selected rows of idx [batch][h_kv][k]; returns the selection buffer."""
+    k = int(idx.shape[-1])
+    if selection is None:
+        selection = torch.empty(max(sd_sparse_selection_size(kv, k), 16), dtype=torch.uint8,
+                                device=kv.k.device)
+    _check(lib().sd_sparse_stage(ctypes.byref(kv.desc), kv.batch, _ptr(idx), k, _ptr(tail_begin),
+                                 _ptr(selection), selection.numel(), _ptr(dev_err),
+                                 _stream(stream)), "sd_sparse_stage")
+    return selection
+
+
+def sd_sparse_attention_staged(q: Queries, kv: KVCache, selection: torch.Tensor, k: int,
+                               tail_begin, max_tail: int, out=None, workspace=None, dev_err=None,
+                               stream=None) -> torch.Tensor:
+    out = _attn_out(q, out)
+    ws = _workspace(sd_sparse_workspace_size(q, kv, k, max_tail), q.q.device, workspace)
+    _check(lib().sd_sparse_attention_staged(
+        ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(selection),
+        int(k), _ptr(tail_begin), int(max_tail), _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
+        _stream(stream)), "sd_sparse_attention_staged")
     return out
 
 

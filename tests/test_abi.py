@@ -54,6 +54,26 @@ def _verify(q, kv, batch=2, ws_bytes=0, ws=None):
                                         ws_bytes, None, None)
 
 
+def test_sparse_workspace_query_includes_the_staged_selection():
+    q, kv = _descs(max_q=1, max_kv=30000)
+    n = ctypes.c_size_t(0)
+    assert sd.lib().sd_attention_workspace_size(sd.SD_ATTN_SPARSE, ctypes.byref(q),
+                                                ctypes.byref(kv), 28,
+                                                ctypes.byref(n)) == sd.SD_ERR_INVALID_ARG
+    assert sd.lib().sd_sparse_workspace_size(ctypes.byref(q), ctypes.byref(kv), 28, 1024, 1100,
+                                             ctypes.byref(n)) == sd.SD_OK
+    staged = 28 * 4 * 1024 * 128 * 2 * 2  # compact K and V, bf16
+    assert n.value >= staged
+    m = ctypes.c_size_t(0)
+    assert sd.lib().sd_sparse_workspace_size(ctypes.byref(q), ctypes.byref(kv), 28, 512, 1100,
+                                             ctypes.byref(m)) == sd.SD_OK
+    assert m.value < n.value
+    # too small a workspace is rejected before any launch
+    assert sd.lib().sd_sparse_attention(ctypes.byref(q), FAKE, ctypes.byref(kv), 28, FAKE, 1024,
+                                        FAKE, 1100, FAKE, FAKE, n.value - 1, None,
+                                        None) == sd.SD_ERR_WORKSPACE
+
+
 def test_workspace_query_and_undersized_workspace_is_rejected():
     q, kv = _descs()
     n = ctypes.c_size_t(0)

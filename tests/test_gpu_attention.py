@@ -224,6 +224,47 @@ def test_sparse_with_every_candidate_equals_dense():
     _assert_close(dense, ref, w.dtype, "dense")
 
 
+@pytest.mark.parametrize("cfg,kw", [(1, dict(l_vis=4000, l_txt=300)),
+                                    (3, dict(layers=3, l_vis=5000, l_txt=600)),
+                                    (4, dict(l_vis=3000, l_txt=200, batch=5))])
+def test_sparse_staged_selection_reused_across_draft_steps(cfg, kw):
+    """One staged selection serves every draft step (the tail grows, the selection does not);
+    each step matches the oracle and the unstaged call."""
+    w = gen.make_attn_workload(cfg, **kw)
+    idx = _oracle_topk(w, w.kv_len_verify, w.topk)
+    tail = w.l_vis.astype(np.int32)
+    kv0 = dev.kv_cache(w, kv_len=w.kv_len_draft(0))
+    sel = sd.sd_sparse_stage(kv0, dev.int32(idx), dev.int32(tail))
+    for step in range(int(w.gamma.min())):  # steps every sequence drafts
+        lens = w.kv_len_draft(step)
+        kv = dev.kv_cache(w, kv_len=lens)
+        q = dev.draft_queries(w, step)
+        max_tail = int((lens - tail).max())
+        out = sd.sd_sparse_attention_staged(q, kv, sel, w.topk, dev.int32(tail), max_tail)
+        ref = oracle.sparse_attention(w.h_q, w.q_draft[step], np.arange(w.n_seq + 1),
+                                      oracle.cache_from_workload(w, kv_len=lens), idx, tail)
+        _assert_close(out, ref, w.dtype, f"staged cfg{cfg} step {step}")
+        direct = sd.sd_sparse_attention(q, kv, dev.int32(idx), dev.int32(tail), max_tail)
+        assert (out.float() - direct.float()).abs().max().item() <= TOL[w.dtype]
+
+
+@pytest.mark.parametrize("tail_back", [1, 3, 40])
+def test_sparse_multi_row_tail_above_row_limits(tail_back):
+    """Several rows per sequence with the tail starting above the lowest rows' causal limit:
+    some selected positions are then invisible to some rows (the positions are checked one by
+    one)."""
+    w = gen.make_attn_workload(1, l_vis=3000, l_txt=200, gamma=4)
+    kv, q = dev.kv_cache(w), dev.verify_queries(w)
+    kv_len = int(w.kv_len_verify[0])
+    tail = np.array([kv_len - tail_back], np.int32)
+    cache = oracle.cache_from_workload(w)
+    idx, _ = oracle.topk_select(w.h_q, w.q_verify, w.q_verify_start, cache,
+                                np.zeros(1, np.int32), tail, 256)
+    out = sd.sd_sparse_attention(q, kv, dev.int32(idx), dev.int32(tail), tail_back)
+    ref = oracle.sparse_attention(w.h_q, w.q_verify, w.q_verify_start, cache, idx, tail)
+    _assert_close(out, ref, w.dtype, f"sparse multi-row tail_back={tail_back}")
+
+
 def test_sparse_unsorted_indices_set_flag():
     w = gen.make_attn_workload(0)
     lens = w.kv_len_draft(0)
