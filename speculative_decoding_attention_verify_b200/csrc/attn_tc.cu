@@ -54,9 +54,17 @@ struct Cfg {
 
 // ---------------------------------------------------------------- the kernel --------------
 
-template <int D, bool PAGED>
+// NCP row copies: with R <= 128 / NCP rows per KV head, the rows are placed NCP times in the
+// 128 MMA rows (copy c in rows [c * 128/NCP, (c+1) * 128/NCP)) and softmax warp w, of copy
+// c = w / (4 / NCP), handles the columns [c * 128/NCP, (c+1) * 128/NCP) of every tile: the
+// exponentials of a tile are spread over four warps (and their SM sub-partitions) instead of
+// one or two.  Each copy keeps its own running max, sum and output rows; the copies are
+// merged in shared memory at the end.
+template <int D, bool PAGED, int NCP>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
+    constexpr int RPC = kRows / NCP;  // rows per copy
+    constexpr int NC = kTile / NCP;   // columns per softmax warp
     using C = Cfg<D>;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -71,8 +79,8 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     const uint32_t bar0 = saddr(bars);
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
     const int KF = 0, VF = S, KE = 2 * S, VE = 3 * S, SF = 4 * S, PF = 4 * S + 2, OD = 4 * S + 4,
-              DR = 4 * S + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * S + 6);
+              DR = 4 * S + 5, QF = 4 * S + 6;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * S + 7);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *s_stream = reinterpret_cast<int *>(tmem_slot + 2);  // stream set-up scratch
 
@@ -84,7 +92,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     const int n_q = __ldg(p.q_start + b + 1) - q0;
     const int kv_len = __ldg(kv.kv_len + b);
     const int R = n_q * G;
-    if (n_q < 1 || R > kRows || n_q > p.max_q_rows || q0 + n_q > p.rows_cap || kv_len < n_q ||
+    if (n_q < 1 || R > RPC || n_q > p.max_q_rows || q0 + n_q > p.rows_cap || kv_len < n_q ||
         (PAGED && kv_len > kv.max_pages * kPageSize)) {
         if (tid == 0 && n_q != 0) set_dev_err(p.dev_err, SD_DEVERR_SHAPE);
         return;
@@ -113,7 +121,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     const int tile_lo = (int)((int64_t)n_tiles * split / p.n_splits);
     const int tile_hi = (int)((int64_t)n_tiles * (split + 1) / p.n_splits);
     const int n_my = tile_hi - tile_lo;
-    const int n_active = (R + 31) / 32;  // softmax warps holding real rows
+    const int n_active = NCP > 1 ? 4 : (R + 31) / 32;  // softmax warps holding real rows
 
     if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -135,14 +143,21 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         }
         mbar_init(BAR(OD), 1);
         mbar_init(BAR(DR), 1);
+        mbar_init(BAR(QF), 128);  // Q in shared memory (warps 0-3)
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // Q rows into shared memory in the 128-byte swizzled K-major layout (rows >= R are zero).
+    tc_before();
+    __syncthreads();
+    tc_after();
+    const uint32_t tmem = *tmem_slot;
+    // Q rows into shared memory in the 128-byte swizzled K-major layout: MMA row rr holds query
+    // row rr % RPC of the group (zero past R).  Loaded after the producer has started its first
+    // copies; the MMA issuer waits for it before the first S = Q K^T.
     if (warp < 4) {
         constexpr int CPR = D / 8;  // 16-byte chunks per row
         for (int e = tid; e < kRows * CPR; e += 128) {
-            const int r = e / CPR, c = e % CPR;
+            const int rr = e / CPR, c = e % CPR, r = rr % RPC;
             uint4 val = make_uint4(0, 0, 0, 0);
             if (r < R) {
                 const int64_t off = ((int64_t)(q0 + r / G) * p.h_q + g * G + r % G) * D + c * 8;
@@ -150,15 +165,12 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                     reinterpret_cast<const unsigned short *>(p.q) + off));
             }
             const int half = c >> 3, cc = c & 7;
-            *reinterpret_cast<uint4 *>(sQ + half * kHalfBytes + r * 128 + ((cc ^ (r & 7)) << 4)) =
+            *reinterpret_cast<uint4 *>(sQ + half * kHalfBytes + rr * 128 + ((cc ^ (rr & 7)) << 4)) =
                 val;
         }
         fence_async_smem();
+        mbar_arrive(BAR(QF));
     }
-    tc_before();
-    __syncthreads();
-    tc_after();
-    const uint32_t tmem = *tmem_slot;
 
     if (warp == kProducerWarp) {
         // ---------------------------------------------------------- TMA producer ----------
@@ -240,7 +252,16 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             __syncwarp();
             return true;
         };
-        bool alive = n_my > 0 ? issue_qk(0) : true;
+        bool alive = true;
+        if (n_my > 0) {
+            bool qok = true;
+            if (lane == 0) qok = mbar_wait(BAR(QF), 0, abort_flag, p.dev_err);
+            alive = __shfl_sync(0xffffffffu, qok ? 1 : 0, 0) != 0;
+            if (alive) {
+                fence_async_smem();
+                alive = issue_qk(0);
+            }
+        }
         for (int t = 0; alive && t < n_my; ++t) {
             const int s = t % S, use = t / S, sb = t & 1;
             if (t + 1 < n_my && !issue_qk(t + 1)) break;
@@ -293,7 +314,9 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         // tcgen05.ld / st are warp-collective: every lane executes them, row validity only
         // selects values, and decisions that gate them are made warp-uniform by votes.
         const unsigned FULL = 0xffffffffu;
-        const int r = warp * 32 + lane;
+        const int cp = NCP > 1 ? warp / (4 / NCP) : 0;  // this warp's row copy
+        const int c0 = cp * NC;                         // its first tile column
+        const int r = warp * 32 + lane - cp * RPC;      // its row
         const bool row_ok = r < R;
         const int limit = kv_len - n_q + (row_ok ? r / G : 0);
         // The row's visible positions as two ranges: visible(j) <=> j - lo1 <= w1 or
@@ -337,48 +360,49 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             }
             tc_after();
             const uint32_t s_addr = lane_base + sb * kTile;
-            float v[kTile];
-            tmem_ld128(s_addr, v);
+            float v[NC];
+            tmem_ld_cols<NC>(s_addr + c0, v);
+            const int q0p = p0 + c0;  // stream coordinate of this warp's first column
             // Interior tiles (inside the run and visible in full to every row of this warp)
             // skip masking.
             // (tiles of the compacted selection are in list coordinates: the positions are
             // cpos[...], all below the tail)
             const bool cmp = sparse && tt < nt0;
-            const bool in_run = p0 >= seg_lo && p0 + kTile <= seg_hi;
-            const uint32_t d1 = (uint32_t)p0 - lo1, d2 = (uint32_t)p0 - lo2;
+            const bool in_run = q0p >= seg_lo && q0p + NC <= seg_hi;
+            const uint32_t d1 = (uint32_t)q0p - lo1, d2 = (uint32_t)q0p - lo2;
             const bool whole = !row_ok || (cmp ? sel_all
-                                               : ((w1 >= kTile - 1 && d1 <= w1 - (kTile - 1)) ||
-                                                  (w2 >= kTile - 1 && d2 <= w2 - (kTile - 1))));
+                                               : ((w1 >= NC - 1 && d1 <= w1 - (NC - 1)) ||
+                                                  (w2 >= NC - 1 && d2 <= w2 - (NC - 1))));
             const bool interior = __all_sync(FULL, in_run && whole);
             float mx = -INFINITY;
             if (!interior) {
                 const uint32_t seg_w = (uint32_t)(seg_hi - seg_lo);
                 if (!cmp) {
 #pragma unroll
-                    for (int e = 0; e < kTile; ++e) {
-                        const uint32_t j = (uint32_t)(p0 + e);
+                    for (int e = 0; e < NC; ++e) {
+                        const uint32_t j = (uint32_t)(q0p + e);
                         const uint32_t vis = (j - (uint32_t)seg_lo < seg_w) &
                                              ((j - lo1 <= w1) | (j - lo2 <= w2));
                         v[e] = vis ? v[e] : -INFINITY;
                     }
                 } else if (sel_all) {
 #pragma unroll
-                    for (int e = 0; e < kTile; ++e) {
-                        const uint32_t vis = ((uint32_t)(p0 + e) < seg_w) & row_ok_u;
+                    for (int e = 0; e < NC; ++e) {
+                        const uint32_t vis = ((uint32_t)(q0p + e) < seg_w) & row_ok_u;
                         v[e] = vis ? v[e] : -INFINITY;
                     }
                 } else {
 #pragma unroll
-                    for (int e = 0; e < kTile; ++e) {
-                        const bool in = p0 + e < (int)seg_w;
-                        const uint32_t j = in ? (uint32_t)__ldg(cpos + p0 + e) : 0u;
+                    for (int e = 0; e < NC; ++e) {
+                        const bool in = q0p + e < (int)seg_w;
+                        const uint32_t j = in ? (uint32_t)__ldg(cpos + q0p + e) : 0u;
                         const uint32_t vis = (uint32_t)in & (j - lo1 <= w1);
                         v[e] = vis ? v[e] : -INFINITY;
                     }
                 }
             }
 #pragma unroll
-            for (int e = 0; e < kTile; e += 2) mx = max3(mx, v[e], v[e + 1]);
+            for (int e = 0; e < NC; e += 2) mx = max3(mx, v[e], v[e + 1]);
             mx = mx == -INFINITY ? -INFINITY : mx * sl2;
             const bool grow = mx > m_used + kRescaleLog2;
             const bool rescale_o = grow && m_used != -INFINITY;
@@ -409,15 +433,25 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
             const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
             float2 acc2 = make_float2(0.f, 0.f);
-            uint32_t pk[kTile / 2];
+            uint32_t pk[NC / 2];
 #pragma unroll
-            for (int e = 0; e < kTile; e += 2) {
+            for (int e = 0; e < NC; e += 2) {
                 const float2 x = __ffma2_rn(make_float2(v[e], v[e + 1]), sc2, nm2);
                 const float2 pe = make_float2(ex2(x.x), ex2(x.y));
                 acc2 = __fadd2_rn(acc2, pe);
                 pk[e >> 1] = pack_bf16(pe.x, pe.y);
             }
-            tmem_st64(s_addr, pk);
+            // P over S: the warp's NC columns are packed into NC/2 TMEM columns at c0/2; the
+            // other copies' columns of these rows are zero
+            uint32_t prow[kTile / 2];
+#pragma unroll
+            for (int i = 0; i < kTile / 2; ++i) prow[i] = 0u;
+#pragma unroll
+            for (int q = 0; q < NCP; ++q)
+                if (q == cp)
+#pragma unroll
+                    for (int i = 0; i < NC / 2; ++i) prow[q * (NC / 2) + i] = pk[i];
+            tmem_st64(s_addr, prow);
             const float sum = acc2.x + acc2.y;
             l += sum;
             tc_before();
@@ -434,17 +468,59 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         const bool have = read_o && m_used != -INFINITY;
         const int i = row_ok ? r / G : 0, h = g * G + (row_ok ? r % G : 0);
         const int row = q0 + i;
-        const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
+        float m_out = have ? m_used : -INFINITY, l_out = have ? l : 0.f;
+        float *s_o = nullptr;  // merged copies: [copy][RPC][D] scaled outputs (stage memory)
+        if constexpr (NCP > 1) {
+            // Merge the copies: M = max over copies, factors 2^(m_c - M), L = sum of scaled
+            // sums; each copy's O, scaled, goes to shared memory (the K/V ring is idle now) and
+            // copy 0 sums them in a fixed order.
+            float *s_m = reinterpret_cast<float *>(sKV);
+            float *s_l = s_m + kRows;
+            s_o = s_l + kRows;
+            s_m[cp * RPC + r] = m_out;
+            s_l[cp * RPC + r] = l_out;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            float M = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < NCP; ++q) M = fmaxf(M, s_m[q * RPC + r]);
+            float L = 0.f;
+#pragma unroll
+            for (int q = 0; q < NCP; ++q) {
+                const float mq = s_m[q * RPC + r];
+                L += mq == -INFINITY ? 0.f : ex2(mq - M) * s_l[q * RPC + r];
+            }
+            const float f = have ? ex2(m_used - M) : 0.f;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                float o[32];
+                if (read_o) tmem_ld32(lane_base + kColO + c * 32, o);
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    s_o[(cp * RPC + r) * D + c * 32 + e] = have ? o[e] * f : 0.f;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            m_out = M;
+            l_out = L;
+        }
+        const float inv = l_out > 0.f ? 1.f / l_out : 0.f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
             float o[32];
-            if (read_o) {
-                tmem_ld32(lane_base + kColO + c * 32, o);
-            }
+            if constexpr (NCP > 1) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                if (!have) o[e] = 0.f;
-            if (!row_ok) continue;
+                for (int e = 0; e < 32; ++e) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int q = 0; q < NCP; ++q) acc += s_o[(q * RPC + r) * D + c * 32 + e];
+                    o[e] = acc;
+                }
+            } else {
+                if (read_o) tmem_ld32(lane_base + kColO + c * 32, o);
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (!have) o[e] = 0.f;
+            }
+            if (!row_ok || cp != 0) continue;
             if (p.n_splits == 1) {
                 uint32_t pk[16];
 #pragma unroll
@@ -461,8 +537,8 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 for (int e = 0; e < 8; ++e)
                     dst[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
                 if (c == 0) {
-                    p.ws_ml[base * 2] = have ? m_used : -INFINITY;
-                    p.ws_ml[base * 2 + 1] = have ? l : 0.f;
+                    p.ws_ml[base * 2] = l_out > 0.f ? m_out : -INFINITY;
+                    p.ws_ml[base * 2 + 1] = l_out;
                 }
             }
         }
@@ -489,10 +565,9 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
 
 // ---------------------------------------------------------------- host side ---------------
 
-template <int D, bool PAGED>
-cudaError_t launch_t(const AttnParams &p, const AttnPlan &plan, const TcMaps &maps,
-                     cudaStream_t s) {
-    auto kern = attn_tc_kernel<D, PAGED>;
+template <int D, bool PAGED, int NCP>
+cudaError_t launch_t(const AttnParams &p, const TcMaps &maps, cudaStream_t s) {
+    auto kern = attn_tc_kernel<D, PAGED, NCP>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -597,10 +672,17 @@ bool tc_supported(int kind, int dtype, int head_dim, int rows) {
 cudaError_t launch_attention_tc(const AttnParams &p, const AttnPlan &plan, cudaStream_t s) {
     TcMaps maps;
     if (!encode_kv_maps(p, p.max_kv_len, &maps)) return cudaErrorNotSupported;
+    (void)plan;
     const bool paged = p.kv.page_size != 0;
-    if (p.kv.head_dim == 128)
-        return paged ? launch_t<128, true>(p, plan, maps, s) : launch_t<128, false>(p, plan, maps, s);
-    return paged ? launch_t<64, true>(p, plan, maps, s) : launch_t<64, false>(p, plan, maps, s);
+    // row copies: four when the planned rows per KV head fit in 32 (the draft steps); with more
+    // rows, two copies measured no faster than one
+    const int rows = p.group * p.max_q_rows;
+    const int ncp = rows <= 32 ? 4 : 1;
+#define SD_TC_LAUNCH(DD, PG)                                                   \
+    (ncp == 4 ? launch_t<DD, PG, 4>(p, maps, s) : launch_t<DD, PG, 1>(p, maps, s))
+    if (p.kv.head_dim == 128) return paged ? SD_TC_LAUNCH(128, true) : SD_TC_LAUNCH(128, false);
+    return paged ? SD_TC_LAUNCH(64, true) : SD_TC_LAUNCH(64, false);
+#undef SD_TC_LAUNCH
 }
 
 }  // namespace sd

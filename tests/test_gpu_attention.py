@@ -43,6 +43,8 @@ VERIFY_CASES = [
     (4, dict(l_vis=1500, l_txt=100, batch=5, gamma=2)),        # paged ragged, R = 21
     (2, dict(layers=48, l_vis=600, l_txt=50, gamma=1)),        # 192 (sequence, KV head) units
     (1, dict(l_vis=40, l_txt=9, gamma=3)),                     # a single tile
+    (1, dict(l_vis=3000, l_txt=100, gamma=11)),                # R = 84 rows: one row copy
+    (1, dict(l_vis=3000, l_txt=100, gamma=8)),                 # R = 63: two row copies
 ]
 
 

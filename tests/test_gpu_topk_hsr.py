@@ -92,7 +92,8 @@ def test_topk_offset_candidate_range_and_ties():
 
 
 @pytest.mark.parametrize("n,bias,d_model", [(1, False, 3584), (3, True, 3584), (16, True, 3584),
-                                            (2, False, 512)])
+                                            (2, False, 512), (4, True, 4096), (2, True, 4112),
+                                            (1, False, 16), (5, False, 64)])
 def test_hsr_matches_oracle(n, bias, d_model):
     hw = gen.make_hsr_workload(n=n, d_model=d_model, with_bias=bias)
     e = dev.tensor(hw.emb, gen.BF16)
@@ -103,3 +104,11 @@ def test_hsr_matches_oracle(n, bias, d_model):
     ref = oracle.hsr_project(hw.emb, hw.hid, hw.weight, hw.bias)
     err = np.abs(dev.to_numpy_f64(y) - ref).max()
     assert err <= 2e-2, err
+
+
+def test_hsr_is_deterministic():
+    hw = gen.make_hsr_workload(n=3, d_model=3584, with_bias=True)
+    e, h, W, b = (dev.tensor(a, gen.BF16) for a in (hw.emb, hw.hid, hw.weight, hw.bias))
+    y1 = sd.sd_hsr_project(e, h, W, b)
+    y2 = sd.sd_hsr_project(e, h, W, b)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
