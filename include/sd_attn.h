@@ -242,7 +242,8 @@ SD_API sd_status sd_topk_workspace_size(const sd_kv_desc *kv, int32_t batch, int
  * scale 1/sqrt(d) changes no rank and is not applied.  Scores are accumulated in fp64.  The k
  * highest scores are selected, equal scores going to the lower position, and written in
  * ascending position order to idx_out [batch][h_kv][k] (device int32); when fewer than k
- * candidates exist all of them are written and the rest is -1.
+ * candidates exist all of them are written and the rest is -1.  A key with an infinite or NaN
+ * element scores +inf, -inf or NaN as that sum does (NaN ranks below every other score).
  */
 SD_API sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
                          int32_t batch, const int32_t *cand_begin, const int32_t *cand_end,

@@ -459,12 +459,11 @@ sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd_kv_des
     p.idx_out = idx_out;
     p.keys = reinterpret_cast<unsigned long long *>(workspace);
     p.dev_err = dev_err;
-    // Scoring CTAs stream 128-candidate tiles through a 3-stage ring (two CTAs per SM for
-    // bf16, d=128); choose the split count whose CTAs fill whole waves best, with at least four
-    // tiles per CTA.
+    // Scoring CTAs stream 128-candidate spans through a shared-memory ring; choose the split
+    // count whose CTAs fill whole waves best, with at least four spans per CTA.
     const int sms = device_sm_count();
     const long long units = (long long)batch * kv->h_kv;
-    const long long slots = (long long)sms * (kv->dtype == SD_BF16 && kv->head_dim == 128 ? 2 : 1);
+    const long long slots = (long long)sms * topk_score_ctas_per_sm();
     const long long tiles = ((long long)max_cand + 127) / 128;
     double best = -1.0;
     p.n_splits = 1;

@@ -86,6 +86,7 @@ struct TopkParams {
     int32_t *dev_err;
 };
 size_t topk_workspace_bytes(int batch, int h_kv, int max_cand);
+int topk_score_ctas_per_sm();  // resident scoring CTAs per SM
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t s);
 
 // HSR projection.

@@ -1,11 +1,14 @@
 // Top-K KV selection per (sequence, KV head).
 //
 // 1. topk_score_kernel: grid (splits, KV heads, sequences).  The group's last query rows are
-//    summed once in fp64 (qbar); candidate key rows are staged through a 3-stage cp.async ring
-//    with coalesced 16-byte copies, and each thread dots one row with qbar in fp64 (four
-//    independent accumulation chains) (bf16 x bf16 products are exact in fp64, and the sum of the
+//    summed once in fp64 (qbar).  Candidate key rows are staged through a 4-stage cp.async
+//    ring in 64-row tiles with coalesced 16-byte copies (two CTAs per SM); four threads share
+//    a row, each holding its quarter of qbar in registers, and accumulate in fp64 (four
+//    independent chains per thread; bf16 x bf16 products are exact in fp64, and the sum of the
 //    group's dot products equals qbar . k up to fp64 rounding).  The score is stored as an
-//    order-preserving 64-bit key (larger score -> larger key; -0 == +0; NaN lowest).
+//    order-preserving 64-bit key (larger score -> larger key; -0 == +0; NaN lowest).  A
+//    non-finite score (the row holds an infinite or NaN element) is recomputed head by head,
+//    since the sum over heads and qbar . k can differ there.
 // 2. topk_select_kernel: one CTA per (sequence, KV head).  An MSB-first radix select (eight
 //    8-bit digits, shared-memory histograms) finds the k-th largest key T exactly; then one
 //    pass in position order keeps every key > T and the first (k - #greater) keys == T, so
@@ -17,7 +20,10 @@
 namespace sd {
 namespace {
 
-constexpr int kScoreThreads = 256;  // two threads per candidate of a tile
+constexpr int kRowThreads = 4;    // threads per candidate (each holds a quarter of qbar)
+constexpr int kScoreTile = 64;    // candidates per staged tile
+constexpr int kScoreThreads = kRowThreads * kScoreTile;
+constexpr int kScoreCtasPerSm = 2;
 constexpr int kSelectThreads = 1024;
 
 __device__ __forceinline__ unsigned long long score_key(double x) {
@@ -42,8 +48,9 @@ __device__ __forceinline__ void cand_range(const TopkParams &p, int b, int &cb, 
     if (bad && threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
 }
 
-constexpr int kScoreTile = 128;   // candidates per staged tile
-constexpr int kScoreStages = 3;   // cp.async ring depth
+// cp.async ring depth: 4 stages of 64 rows (bf16, d = 128: two CTAs x 48 KB ahead per SM),
+// 3 for fp32 rows
+constexpr int score_stages(int row_bytes) { return row_bytes >= 512 ? 3 : 4; }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -58,14 +65,58 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Shared-memory chunk slot of chunk ch of tile row `row`.  A quarter-warp (the unit of a
+// 16-byte shared load) covers two rows x four threads; thread j of a row reads chunks
+// j, j + 4, ...; flipping bit 2 of the slot on odd rows puts the two rows on disjoint bank
+// quads, and the copy side's eight consecutive chunks of one row stay distinct.
+__device__ __forceinline__ int score_swizzle(int ch, int row) { return ch ^ ((row & 1) << 2); }
+
+// Element e of query head h in row `row`.
 template <bool BF16, int D>
-__global__ void __launch_bounds__(kScoreThreads) topk_score_kernel(const TopkParams p) {
+__device__ __forceinline__ float query_elem(const void *q, int h_q, int row, int h, int e) {
+    const int64_t off = ((int64_t)row * h_q + h) * D + e;
+    return BF16 ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(q) +
+                                                  off) << 16)
+                : __ldg(reinterpret_cast<const float *>(q) + off);
+}
+
+// Part score (one thread's chunks) of a key row whose qbar score is not finite: the row holds
+// an infinite or NaN element (or the query does).  The score is then +inf, -inf or NaN, and
+// which one follows the group's own dot products (the sum over heads of q_h . k): qbar . k can
+// differ there (+inf against heads of both signs is NaN).  Rare, so it is recomputed head by
+// head, outside the scoring loop.
+template <bool BF16, int D>
+__device__ __noinline__ double nonfinite_part_score(const void *q, int h_q, int row, int h0,
+                                                    int h1, const uint8_t *rp, int c,
+                                                    int part) {
+    using CH = Chunk<BF16>;
+    constexpr int NCHUNK = D * (BF16 ? 2 : 4) / 16;
+    constexpr int QCH = NCHUNK / kRowThreads;
+    double t = 0.0;
+    for (int k = 0; k < QCH; ++k) {
+        const int ch = part + kRowThreads * k;
+        const uint4 raw = *reinterpret_cast<const uint4 *>(rp + (score_swizzle(ch, c) << 4));
+        float f[CH::kElems];
+        CH::to_float(raw, f);
+#pragma unroll
+        for (int e = 0; e < CH::kElems; ++e)
+            for (int h = h0; h < h1; ++h)
+                t = fma((double)query_elem<BF16, D>(q, h_q, row, h, ch * CH::kElems + e),
+                        (double)f[e], t);
+    }
+    return t;
+}
+
+template <bool BF16, int D>
+__global__ void __launch_bounds__(kScoreThreads, kScoreCtasPerSm) topk_score_kernel(const TopkParams p) {
     using CH = Chunk<BF16>;
     constexpr int ESZ = BF16 ? 2 : 4;
     constexpr int ROWB = D * ESZ;
     constexpr int NCHUNK = ROWB / 16;
-    constexpr int SWZ = NCHUNK < 16 ? NCHUNK - 1 : 15;
-    static_assert(kScoreThreads == 2 * kScoreTile, "two threads per candidate");
+    constexpr int QCH = NCHUNK / kRowThreads;  // chunks per thread
+    constexpr int QE = D / kRowThreads;        // elements per thread
+    constexpr int kScoreStages = score_stages(ROWB);
+    static_assert(kScoreThreads == kRowThreads * kScoreTile, "four threads per candidate");
     extern __shared__ __align__(128) uint8_t s_ring[];  // [stage][kScoreTile][ROWB]
     __shared__ double s_qbar[D];
     __shared__ int64_t s_off[kScoreStages][kScoreTile];
@@ -80,15 +131,21 @@ __global__ void __launch_bounds__(kScoreThreads) topk_score_kernel(const TopkPar
     cand_range(p, b, cb, n);
     for (int e = tid; e < D; e += kScoreThreads) {
         double acc = 0.0;
-        for (int h = g * p.group; h < (g + 1) * p.group; ++h) {
-            const int64_t off = ((int64_t)last * p.h_q + h) * D + e;
-            const float qf = BF16 ? __uint_as_float((uint32_t)__ldg(
-                                        reinterpret_cast<const unsigned short *>(p.q) + off) << 16)
-                                  : __ldg(reinterpret_cast<const float *>(p.q) + off);
-            acc += (double)qf;
-        }
+        for (int h = g * p.group; h < (g + 1) * p.group; ++h)
+            acc += (double)query_elem<BF16, D>(p.q, p.h_q, last, h, e);
         s_qbar[e] = acc;
     }
+    __syncthreads();
+    // thread quad (4c .. 4c+3) scores candidate c of a tile; thread 4c+j takes chunks
+    // j, j+4, ... of the row and holds their qbar elements in registers
+    const int c = tid / kRowThreads, quarter = tid % kRowThreads;
+    double qr[QE];
+#pragma unroll
+    for (int k = 0; k < QCH; ++k)
+#pragma unroll
+        for (int e = 0; e < CH::kElems; ++e)
+            qr[k * CH::kElems + e] = s_qbar[(quarter + kRowThreads * k) * CH::kElems + e];
+
     unsigned long long *keys = p.keys + ((int64_t)b * p.kv.h_kv + g) * p.max_cand;
     const int t_begin = (int)((int64_t)n * split / p.n_splits);
     const int t_end = (int)((int64_t)n * (split + 1) / p.n_splits);
@@ -105,11 +162,13 @@ __global__ void __launch_bounds__(kScoreThreads) topk_score_kernel(const TopkPar
     };
     auto issue_tile = [&](int u) {  // coalesced: consecutive threads take consecutive chunks
         const int st = u % kScoreStages;
-        for (int e = tid; e < kScoreTile * NCHUNK; e += kScoreThreads) {
+#pragma unroll
+        for (int i = 0; i < kScoreTile * NCHUNK / kScoreThreads; ++i) {
+            const int e = tid + i * kScoreThreads;
             const int row = e / NCHUNK, ch = e % NCHUNK;
             const int64_t off = s_off[st][row];
             if (off < 0) continue;
-            cp_async16(ring + (st * kScoreTile + row) * ROWB + ((ch ^ (row & SWZ)) << 4),
+            cp_async16(ring + (st * kScoreTile + row) * ROWB + (score_swizzle(ch, row) << 4),
                        kbase + off * ESZ + ch * 16);
         }
     };
@@ -127,28 +186,36 @@ __global__ void __launch_bounds__(kScoreThreads) topk_score_kernel(const TopkPar
         if (u < n_tiles) issue_tile(u);
         cp_async_commit();
         const int st = t % kScoreStages;
-        // thread pair (2c, 2c+1) scores candidate c of the tile: each takes half of the row
-        const int c = tid >> 1, half = tid & 1;
         const int cand = t_begin + t * kScoreTile + c;
-        const bool valid = s_off[st][c] >= 0;
+        const bool live = cand < t_end && s_off[st][c] >= 0;
+        const uint8_t *rp = s_ring + (st * kScoreTile + c) * ROWB;
         double a[4] = {0.0, 0.0, 0.0, 0.0};  // independent chains
-        if (cand < t_end && valid) {
-            const uint8_t *rp = s_ring + (st * kScoreTile + c) * ROWB;
+        if (live) {
 #pragma unroll
-            for (int k = 0; k < NCHUNK / 2; ++k) {
-                const int ch = half * (NCHUNK / 2) + k;
-                const uint4 raw = *reinterpret_cast<const uint4 *>(rp + ((ch ^ (c & SWZ)) << 4));
+            for (int k = 0; k < QCH; ++k) {
+                const int ch = quarter + kRowThreads * k;
+                const uint4 raw = *reinterpret_cast<const uint4 *>(rp + (score_swizzle(ch, c) << 4));
                 float f[CH::kElems];
                 CH::to_float(raw, f);
 #pragma unroll
                 for (int e = 0; e < CH::kElems; ++e)
-                    a[e & 3] = fma((double)f[e], s_qbar[ch * CH::kElems + e], a[e & 3]);
+                    a[e & 3] = fma((double)f[e], qr[k * CH::kElems + e], a[e & 3]);
             }
         }
-        const double part = (a[0] + a[1]) + (a[2] + a[3]);
-        const double other = __shfl_xor_sync(0xffffffffu, part, 1);
-        if (half == 0 && cand < t_end)
-            keys[cand] = valid ? score_key(part + other) : 0ull;  // first half + second half
+        double part = (a[0] + a[1]) + (a[2] + a[3]);
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);  // the same sum in all four threads
+        // converted elements carry infinities and NaNs into the score
+        const bool redo = live && !isfinite(part);
+        if (__any_sync(0xffffffffu, redo)) {
+            double r = redo ? nonfinite_part_score<BF16, D>(p.q, p.h_q, last, g * p.group,
+                                                            (g + 1) * p.group, rp, c, quarter)
+                            : 0.0;
+            r += __shfl_xor_sync(0xffffffffu, r, 1);
+            r += __shfl_xor_sync(0xffffffffu, r, 2);
+            if (redo) part = r;
+        }
+        if (quarter == 0 && cand < t_end) keys[cand] = live ? score_key(part) : 0ull;
         __syncthreads();
     }
     cp_async_wait<0>();
@@ -324,7 +391,7 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_smem_kernel(const 
 
 template <bool BF16, int D>
 cudaError_t launch_score_t(const TopkParams &p, cudaStream_t s) {
-    const int dyn = kScoreStages * kScoreTile * D * (BF16 ? 2 : 4);
+    const int dyn = score_stages(D * (BF16 ? 2 : 4)) * kScoreTile * D * (BF16 ? 2 : 4);
     auto kern = topk_score_kernel<BF16, D>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -338,6 +405,8 @@ cudaError_t launch_score_t(const TopkParams &p, cudaStream_t s) {
 }
 
 }  // namespace
+
+int topk_score_ctas_per_sm() { return kScoreCtasPerSm; }
 
 size_t topk_workspace_bytes(int batch, int h_kv, int max_cand) {
     return (size_t)batch * h_kv * (size_t)max_cand * sizeof(unsigned long long);

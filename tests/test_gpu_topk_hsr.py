@@ -88,6 +88,58 @@ def test_topk_offset_candidate_range_and_ties():
     assert _assert_same_sets(got, ref, gap) == 0
 
 
+def test_topk_special_key_values():
+    """Signed zeros, subnormals, the largest finite keys and non-finite keys score exactly.
+
+    Head 0 holds only subnormal keys (every score is then a sum of subnormal products), head 1
+    zeros and subnormals among normal keys, head 2 the largest finite bf16 values among normal
+    keys, head 3 a few +inf, -inf and NaN elements.  A non-finite element makes the score the
+    sum over the group's heads of +-inf products: +inf or -inf where every head's query agrees
+    in sign there (dimension 9 of group 3 is set to 1.0 in every head), NaN otherwise.
+    """
+    w = gen.make_attn_workload(1, l_vis=3000, l_txt=50)
+    rng = np.random.default_rng(11)
+    k = w.k.copy()
+    shape = k[0, 0, :3000].shape
+    sign = rng.integers(0, 2, size=shape).astype(np.uint16) << 15
+    sub = rng.integers(1, 128, size=shape).astype(np.uint16) | sign
+    k[0, 0, :3000] = sub
+    h1 = k[0, 1, :3000]
+    r = rng.random(shape)
+    h1[r < 0.2] = sub[r < 0.2]
+    h1[(r >= 0.2) & (r < 0.3)] = sign[(r >= 0.2) & (r < 0.3)]  # +0 / -0
+    h2 = k[0, 2, :3000]
+    big = rng.random(shape) < 0.01
+    h2[big] = np.uint16(0x7F7F) | sign[big]
+    h3 = k[0, 3, :3000]
+    PINF, NINF, QNAN = 0x7F80, 0xFF80, 0x7FC0
+    for pos, dim, val in ((100, 9, PINF), (1500, 9, PINF), (101, 9, NINF), (700, 60, PINF),
+                          (2000, 80, NINF), (2500, 4, QNAN), (2600, 9, PINF), (2600, 10, NINF)):
+        h3[pos, dim] = val
+    w.k = k
+    q = w.q_verify.copy()
+    last = int(w.q_verify_start[1]) - 1
+    q[last, 21:28, 9] = 0x3F80  # 1.0: every head of group 3 agrees in sign at dimension 9
+    w.q_verify = q
+    got, ref, gap = _run_topk(w, 200)
+    assert np.array_equal(got, ref)
+    sel3 = set(got[0, 3].tolist())
+    assert {100, 1500} <= sel3                       # +inf scores
+    assert not {101, 700, 2000, 2500, 2600} & sel3   # -inf or NaN scores
+
+
+def test_topk_huge_query_values():
+    """Queries near the top of the bf16 range: |qbar| reaches 7 * 2^126 in one dimension."""
+    w = gen.make_attn_workload(1, l_vis=3000, l_txt=50)
+    q = w.q_verify.copy()
+    last = int(w.q_verify_start[1]) - 1
+    q[last, :7, 3] = 0x7E80  # 2^126 in seven heads of group 0: the group sum is 7 * 2^126
+    q[last, 7:14, 5] = 0x7E00  # 2^125 in group 1
+    w.q_verify = q
+    got, ref, gap = _run_topk(w, 300)
+    assert _assert_same_sets(got, ref, gap) == 0
+
+
 # ---------------------------------------------------------------- HSR ----------------------
 
 
