@@ -37,8 +37,9 @@ constexpr int kRows = 128;            // MMA M
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kThreads = 6 * 32;
-constexpr uint32_t kTmemCols = 512;   // S0 [0,128) S1 [128,256) O [256, 256+D)
+constexpr uint32_t kTmemCols = 512;   // S0 [0,128) S1 [128,256) O [256,256+D) Q [384,384+D/2)
 constexpr uint32_t kColO = 256;
+constexpr uint32_t kColQ = 384;       // Q as packed bf16 pairs: the A operand of S = Q K^T
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kHalfBytes = kTile * 128;  // one 64-column half of a 128-row tile
 
@@ -47,8 +48,7 @@ struct Cfg {
     static constexpr int kHalves = D / 64;
     static constexpr int kTileBytes = kTile * D * 2;
     static constexpr int kStages = D == 128 ? 3 : 4;
-    static constexpr int kQBytes = kRows * D * 2;
-    static constexpr int kBarOffset = kQBytes + kStages * 2 * kTileBytes;
+    static constexpr int kBarOffset = kStages * 2 * kTileBytes;
     static constexpr int kSmem = kBarOffset + 256 + 1024;  // barriers (<= 4S+8 words) + slack
 };
 
@@ -70,8 +70,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQ = smem;
-    uint8_t *sKV = smem + C::kQBytes;  // stage s: K at s*2*tile, V at s*2*tile + tile
+    uint8_t *sKV = smem;  // stage s: K at s*2*tile, V at s*2*tile + tile
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
     // barrier slots: k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_full[2],
     // o_done, drain.  A stage's K half is released as soon as S = Q K^T is computed, its V
@@ -151,38 +150,59 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     __syncthreads();
     tc_after();
     const uint32_t tmem = *tmem_slot;
-    // Q rows into shared memory in the 128-byte swizzled K-major layout: MMA row rr holds query
-    // row rr % RPC of the group (zero past R).  Loaded after the producer has started its first
-    // copies; the MMA issuer waits for it before the first S = Q K^T.
+    // Q rows into TMEM columns [kColQ, kColQ + D/2) as packed bf16 pairs, the A operand of
+    // S = Q K^T (read by the tensor core from TMEM, not re-read from shared memory every
+    // tile): lane rr holds query row rr % RPC of the group (zero past R).  Each of warps 0-3
+    // writes its own 32 lanes, after the producer has started its first copies; the MMA
+    // issuer waits for it before the first S = Q K^T.
     if (warp < 4) {
-        constexpr int CPR = D / 8;  // 16-byte chunks per row
-        for (int e = tid; e < kRows * CPR; e += 128) {
-            const int rr = e / CPR, c = e % CPR, r = rr % RPC;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (r < R) {
-                const int64_t off = ((int64_t)(q0 + r / G) * p.h_q + g * G + r % G) * D + c * 8;
-                val = __ldg(reinterpret_cast<const uint4 *>(
-                    reinterpret_cast<const unsigned short *>(p.q) + off));
+        const int rr = warp * 32 + lane, r = rr % RPC;
+        uint32_t qv[D / 2];
+        if (r < R) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                reinterpret_cast<const unsigned short *>(p.q) +
+                ((int64_t)(q0 + r / G) * p.h_q + g * G + r % G) * D);
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) {
+                const uint4 x = __ldg(src + c);
+                qv[4 * c] = x.x;
+                qv[4 * c + 1] = x.y;
+                qv[4 * c + 2] = x.z;
+                qv[4 * c + 3] = x.w;
             }
-            const int half = c >> 3, cc = c & 7;
-            *reinterpret_cast<uint4 *>(sQ + half * kHalfBytes + rr * 128 + ((cc ^ (rr & 7)) << 4)) =
-                val;
+        } else {
+#pragma unroll
+            for (int c = 0; c < D / 2; ++c) qv[c] = 0u;
         }
-        fence_async_smem();
+        const uint32_t qaddr = tmem + ((uint32_t)(warp * 32) << 16) + kColQ;
+        if constexpr (D == 128) {
+            tmem_st64(qaddr, qv);
+        } else {
+            float qf[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) qf[c] = __uint_as_float(qv[c]);
+            tmem_st32(qaddr, qf);
+        }
+        tc_before();
         mbar_arrive(BAR(QF));
     }
 
+    int n_issued = 0;  // producer lanes: tiles whose copy this lane has issued
     if (warp == kProducerWarp) {
         // ---------------------------------------------------------- TMA producer ----------
-        if (lane == 0) {
+        // Lane 0 streams K, lane 1 streams V, each through its own half of the stage ring, so
+        // a K copy never waits behind the release of a V stage (which needs the P.V).
+        if (lane < 2) {
+            const int half = lane;
+            const int full = half == 0 ? KF : VF, empty = half == 0 ? KE : VE;
             int pages[kTile / kPageSize];
             for (int t = 0; t < n_my; ++t) {
                 const int s = t % S, use = t / S;
                 const int p0 = tile_start(tile_lo + t);
                 // compacted sparse selection: its own contiguous buffer
                 const bool cmp = sparse && tile_lo + t < nt0;
-                const uint32_t dK = saddr(sKV + (size_t)s * 2 * C::kTileBytes);
-                const uint32_t dV = dK + C::kTileBytes;
+                const uint32_t dst =
+                    saddr(sKV + (size_t)s * 2 * C::kTileBytes + (size_t)half * C::kTileBytes);
                 if (PAGED && !cmp) {
                     for (int pg = 0; pg < kTile / kPageSize; ++pg) {
                         const int pos = p0 + pg * kPageSize;
@@ -198,26 +218,23 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                         pages[pg] = page;
                     }
                 }
-                for (int half = 0; half < 2; ++half) {  // K, then V
-                    const int full = half == 0 ? KF : VF, empty = half == 0 ? KE : VE;
-                    const uint32_t dst = half == 0 ? dK : dV;
-                    const CUtensorMap *map = cmp ? (half == 0 ? &maps.k2 : &maps.v2)
-                                                 : (half == 0 ? &maps.k : &maps.v);
-                    if (t >= S && !mbar_wait(BAR(empty + s), (use - 1) & 1, abort_flag, p.dev_err))
-                        break;
-                    mbar_arrive_tx(BAR(full + s), C::kTileBytes);
-                    if (!PAGED || cmp) {
+                const CUtensorMap *map = cmp ? (half == 0 ? &maps.k2 : &maps.v2)
+                                             : (half == 0 ? &maps.k : &maps.v);
+                if (t >= S && !mbar_wait(BAR(empty + s), (use - 1) & 1, abort_flag, p.dev_err))
+                    break;
+                mbar_arrive_tx(BAR(full + s), C::kTileBytes);
+                if (!PAGED || cmp) {
+#pragma unroll
+                    for (int h = 0; h < C::kHalves; ++h)
+                        tma_load_4d(dst + h * kHalfBytes, map, BAR(full + s), h * 64, p0, g, b);
+                } else {
+                    for (int pg = 0; pg < kTile / kPageSize; ++pg)
 #pragma unroll
                         for (int h = 0; h < C::kHalves; ++h)
-                            tma_load_4d(dst + h * kHalfBytes, map, BAR(full + s), h * 64, p0, g, b);
-                    } else {
-                        for (int pg = 0; pg < kTile / kPageSize; ++pg)
-#pragma unroll
-                            for (int h = 0; h < C::kHalves; ++h)
-                                tma_load_4d(dst + h * kHalfBytes + pg * kPageSize * 128, map,
-                                            BAR(full + s), h * 64, 0, g, pages[pg]);
-                    }
+                            tma_load_4d(dst + h * kHalfBytes + pg * kPageSize * 128, map,
+                                        BAR(full + s), h * 64, 0, g, pages[pg]);
                 }
+                n_issued = t + 1;
                 if (*abort_flag) break;
             }
         }
@@ -228,21 +245,16 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         // tensor core computes it while the softmax warps work.
         const uint32_t idesc_qk = idesc_bf16(kTile, false);
         const uint32_t idesc_pv = idesc_bf16(D, true);
-        const uint32_t q_base = saddr(sQ);
         bool issued = false;
-        auto issue_qk = [&](int t) -> bool {
-            const int s = t % S, use = t / S, sb = t & 1;
+        auto issue_qk = [&](int t) {  // S = Q K^T of tile t (its K stage has landed)
+            const int s = t % S, sb = t & 1;
             const uint32_t kb = saddr(sKV + (size_t)s * 2 * C::kTileBytes);
-            bool ok = true;
-            if (lane == 0) ok = mbar_wait(BAR(KF + s), use & 1, abort_flag, p.dev_err);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) return false;
             tc_after();
             if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                    mma_ss(tmem + sb * kTile, desc_k_sw128(q_base + off), desc_k_sw128(kb + off),
+                    mma_ts(tmem + sb * kTile, tmem + kColQ + kk * 8, desc_k_sw128(kb + off),
                            idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(BAR(SF + sb));
@@ -250,27 +262,9 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 issued = true;
             }
             __syncwarp();
-            return true;
         };
-        bool alive = true;
-        if (n_my > 0) {
-            bool qok = true;
-            if (lane == 0) qok = mbar_wait(BAR(QF), 0, abort_flag, p.dev_err);
-            alive = __shfl_sync(0xffffffffu, qok ? 1 : 0, 0) != 0;
-            if (alive) {
-                fence_async_smem();
-                alive = issue_qk(0);
-            }
-        }
-        for (int t = 0; alive && t < n_my; ++t) {
-            const int s = t % S, use = t / S, sb = t & 1;
-            if (t + 1 < n_my && !issue_qk(t + 1)) break;
-            bool ok = true;
-            if (lane == 0)
-                ok = mbar_wait(BAR(PF + sb), (t >> 1) & 1, abort_flag, p.dev_err) &&
-                     mbar_wait(BAR(VF + s), use & 1, abort_flag, p.dev_err);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
+        auto issue_pv = [&](int t) {  // O += P V of tile t (its P and V stage are ready)
+            const int s = t % S, sb = t & 1;
             // V rows past the end of the sequence may hold anything (NaN included): zero
             // them so that 0 * V cannot poison O.
             uint8_t *vs = sKV + (size_t)s * 2 * C::kTileBytes + C::kTileBytes;
@@ -299,6 +293,56 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 mma_commit(BAR(OD));
             }
             __syncwarp();
+        };
+        bool alive = true;
+        if (n_my > 0) {
+            bool qok = true;
+            if (lane == 0)
+                qok = mbar_wait(BAR(QF), 0, abort_flag, p.dev_err) &&
+                      mbar_wait(BAR(KF), 0, abort_flag, p.dev_err);
+            alive = __shfl_sync(0xffffffffu, qok ? 1 : 0, 0) != 0;
+            if (alive) issue_qk(0);
+        }
+        for (int t = 0; alive && t < n_my; ++t) {
+            // S of tile t+1 and P.V of tile t, in whichever order their operands arrive (S
+            // first when both are ready, so the softmax warps get their next tile early).  S of
+            // t+1 overwrites the buffer of tile t-1, whose P.V was issued in the previous
+            // iteration, so either order is safe.
+            const int s = t % S, use = t / S, sb = t & 1;
+            const int s1 = (t + 1) % S, use1 = (t + 1) / S;
+            bool qk_done = t + 1 >= n_my, pv_done = false;
+            const unsigned long long t0 = now_ns();
+            for (unsigned it = 1; !(qk_done && pv_done); ++it) {
+                int flags = 0;  // bit 0: S can go, bit 1: P.V can go, bit 2: give up
+                if (lane == 0) {
+                    if (!qk_done && mbar_try(BAR(KF + s1), use1 & 1)) flags |= 1;
+                    if (!pv_done && mbar_try(BAR(PF + sb), (t >> 1) & 1) &&
+                        mbar_try(BAR(VF + s), use & 1))
+                        flags |= 2;
+                    if (flags == 0 && (it & 63u) == 0) {
+                        if (*abort_flag) {
+                            flags = 4;
+                        } else if (now_ns() - t0 > kWaitNs) {
+                            *abort_flag = 1;
+                            set_dev_err(p.dev_err, SD_DEVERR_TIMEOUT);
+                            flags = 4;
+                        }
+                    }
+                }
+                flags = __shfl_sync(0xffffffffu, flags, 0);
+                if (flags & 4) {
+                    alive = false;
+                    break;
+                }
+                if (flags & 1) {
+                    issue_qk(t + 1);
+                    qk_done = true;
+                }
+                if (flags & 2) {
+                    issue_pv(t);
+                    pv_done = true;
+                }
+            }
         }
         // Drain: every MMA this warp issued has completed once the drain barrier flips.
         const bool any_issued = __any_sync(0xffffffffu, issued);
@@ -469,14 +513,17 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         const int i = row_ok ? r / G : 0, h = g * G + (row_ok ? r % G : 0);
         const int row = q0 + i;
         float m_out = have ? m_used : -INFINITY, l_out = have ? l : 0.f;
-        float *s_o = nullptr;  // merged copies: [copy][RPC][D] scaled outputs (stage memory)
+        // merged copies: [copy][RPC][D/4] float4 of scaled outputs (stage memory); 16-byte
+        // chunk j of row r sits in slot j ^ (r & 7), so the eight rows of a quarter-warp
+        // access hit distinct banks
+        float4 *s_o = nullptr;
         if constexpr (NCP > 1) {
             // Merge the copies: M = max over copies, factors 2^(m_c - M), L = sum of scaled
             // sums; each copy's O, scaled, goes to shared memory (the K/V ring is idle now) and
             // copy 0 sums them in a fixed order.
             float *s_m = reinterpret_cast<float *>(sKV);
             float *s_l = s_m + kRows;
-            s_o = s_l + kRows;
+            s_o = reinterpret_cast<float4 *>(s_l + kRows);
             s_m[cp * RPC + r] = m_out;
             s_l[cp * RPC + r] = l_out;
             asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -494,25 +541,40 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             for (int c = 0; c < D / 32; ++c) {
                 float o[32];
                 if (read_o) tmem_ld32(lane_base + kColO + c * 32, o);
+                float4 *dst = s_o + (cp * RPC + r) * (D / 4);
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    s_o[(cp * RPC + r) * D + c * 32 + e] = have ? o[e] * f : 0.f;
+                for (int k = 0; k < 8; ++k)
+                    dst[(c * 8 + k) ^ (r & 7)] =
+                        have ? make_float4(o[4 * k] * f, o[4 * k + 1] * f, o[4 * k + 2] * f,
+                                           o[4 * k + 3] * f)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
             m_out = M;
             l_out = L;
         }
         const float inv = l_out > 0.f ? 1.f / l_out : 0.f;
+        const bool writer = row_ok && cp == 0;  // copy 0 holds the merged row
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
             float o[32];
             if constexpr (NCP > 1) {
+                if (!writer) continue;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float acc = 0.f;
+                for (int k = 0; k < 8; ++k) {
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                    for (int q = 0; q < NCP; ++q) acc += s_o[(q * RPC + r) * D + c * 32 + e];
-                    o[e] = acc;
+                    for (int q = 0; q < NCP; ++q) {
+                        const float4 x = s_o[(q * RPC + r) * (D / 4) + ((c * 8 + k) ^ (r & 7))];
+                        acc.x += x.x;
+                        acc.y += x.y;
+                        acc.z += x.z;
+                        acc.w += x.w;
+                    }
+                    o[4 * k] = acc.x;
+                    o[4 * k + 1] = acc.y;
+                    o[4 * k + 2] = acc.z;
+                    o[4 * k + 3] = acc.w;
                 }
             } else {
                 if (read_o) tmem_ld32(lane_base + kColO + c * 32, o);
@@ -520,7 +582,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 for (int e = 0; e < 32; ++e)
                     if (!have) o[e] = 0.f;
             }
-            if (!row_ok || cp != 0) continue;
+            if (!writer) continue;
             if (p.n_splits == 1) {
                 uint32_t pk[16];
 #pragma unroll
@@ -545,12 +607,13 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     }
 
     // ---- teardown: the producer drains its own copies if the CTA aborted ----
-    if (warp == kProducerWarp && lane == 0 && *abort_flag) {
+    if (warp == kProducerWarp && lane < 2 && *abort_flag) {
+        // only the last S copies this lane issued can still be in flight
         const unsigned long long t0 = now_ns();
-        for (int t = (n_my > S ? n_my - S : 0); t < n_my; ++t) {
+        const int full = lane == 0 ? KF : VF;
+        for (int t = (n_issued > S ? n_issued - S : 0); t < n_issued; ++t) {
             const int s = t % S, use = t / S;
-            while ((!mbar_try(BAR(KF + s), use & 1) || !mbar_try(BAR(VF + s), use & 1)) &&
-                   now_ns() - t0 < kWaitNs) {
+            while (!mbar_try(BAR(full + s), use & 1) && now_ns() - t0 < kWaitNs) {
             }
         }
     }
@@ -564,6 +627,8 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
 }
 
 // ---------------------------------------------------------------- host side ---------------
+
+constexpr int kNcp2Rows = 64;  // largest row count per KV head served with two copies
 
 template <int D, bool PAGED, int NCP>
 cudaError_t launch_t(const AttnParams &p, const TcMaps &maps, cudaStream_t s) {
@@ -674,12 +739,14 @@ cudaError_t launch_attention_tc(const AttnParams &p, const AttnPlan &plan, cudaS
     if (!encode_kv_maps(p, p.max_kv_len, &maps)) return cudaErrorNotSupported;
     (void)plan;
     const bool paged = p.kv.page_size != 0;
-    // row copies: four when the planned rows per KV head fit in 32 (the draft steps); with more
-    // rows, two copies measured no faster than one
+    // row copies: four when the planned rows per KV head fit in 32 (the draft steps), two when
+    // they fit in 64 (verification of up to 9 rows x 7 heads)
     const int rows = p.group * p.max_q_rows;
-    const int ncp = rows <= 32 ? 4 : 1;
-#define SD_TC_LAUNCH(DD, PG)                                                   \
-    (ncp == 4 ? launch_t<DD, PG, 4>(p, maps, s) : launch_t<DD, PG, 1>(p, maps, s))
+    const int ncp = rows <= 32 ? 4 : rows <= kNcp2Rows ? 2 : 1;
+#define SD_TC_LAUNCH(DD, PG)                                                                   \
+    (ncp == 4   ? launch_t<DD, PG, 4>(p, maps, s)                                              \
+     : ncp == 2 ? launch_t<DD, PG, 2>(p, maps, s)                                              \
+                : launch_t<DD, PG, 1>(p, maps, s))
     if (p.kv.head_dim == 128) return paged ? SD_TC_LAUNCH(128, true) : SD_TC_LAUNCH(128, false);
     return paged ? SD_TC_LAUNCH(64, true) : SD_TC_LAUNCH(64, false);
 #undef SD_TC_LAUNCH
