@@ -513,45 +513,46 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         const int i = row_ok ? r / G : 0, h = g * G + (row_ok ? r % G : 0);
         const int row = q0 + i;
         float m_out = have ? m_used : -INFINITY, l_out = have ? l : 0.f;
-        // merged copies: [copy][RPC][D/4] float4 of scaled outputs (stage memory); 16-byte
+        // merged copies: [copy][RPC][D/4] float4 of unscaled outputs (stage memory); 16-byte
         // chunk j of row r sits in slot j ^ (r & 7), so the eight rows of a quarter-warp
         // access hit distinct banks
         float4 *s_o = nullptr;
+        float fq[NCP];  // copy 0: the factor 2^(m_c - M) of every copy
         if constexpr (NCP > 1) {
-            // Merge the copies: M = max over copies, factors 2^(m_c - M), L = sum of scaled
-            // sums; each copy's O, scaled, goes to shared memory (the K/V ring is idle now) and
-            // copy 0 sums them in a fixed order.
+            // Merge the copies through shared memory (the K/V ring is idle now): every copy
+            // writes its (m, l) and its O, read from TMEM in one load; copy 0 then forms
+            // M = max over copies, the factors 2^(m_c - M), L = sum of scaled sums and the
+            // sum of scaled outputs, in a fixed order.
             float *s_m = reinterpret_cast<float *>(sKV);
             float *s_l = s_m + kRows;
             s_o = reinterpret_cast<float4 *>(s_l + kRows);
             s_m[cp * RPC + r] = m_out;
             s_l[cp * RPC + r] = l_out;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            float M = -INFINITY;
-#pragma unroll
-            for (int q = 0; q < NCP; ++q) M = fmaxf(M, s_m[q * RPC + r]);
-            float L = 0.f;
-#pragma unroll
-            for (int q = 0; q < NCP; ++q) {
-                const float mq = s_m[q * RPC + r];
-                L += mq == -INFINITY ? 0.f : ex2(mq - M) * s_l[q * RPC + r];
-            }
-            const float f = have ? ex2(m_used - M) : 0.f;
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                float o[32];
-                if (read_o) tmem_ld32(lane_base + kColO + c * 32, o);
+            {
+                float o[D];
+                if (read_o) tmem_ld_cols<D>(lane_base + kColO, o);
                 float4 *dst = s_o + (cp * RPC + r) * (D / 4);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    dst[(c * 8 + k) ^ (r & 7)] =
-                        have ? make_float4(o[4 * k] * f, o[4 * k + 1] * f, o[4 * k + 2] * f,
-                                           o[4 * k + 3] * f)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int k = 0; k < D / 4; ++k)
+                    dst[k ^ (r & 7)] = have ? make_float4(o[4 * k], o[4 * k + 1], o[4 * k + 2],
+                                                          o[4 * k + 3])
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            m_out = M;
-            l_out = L;
+            if (cp == 0) {
+                float M = -INFINITY;
+#pragma unroll
+                for (int q = 0; q < NCP; ++q) M = fmaxf(M, s_m[q * RPC + r]);
+                float L = 0.f;
+#pragma unroll
+                for (int q = 0; q < NCP; ++q) {
+                    const float mq = s_m[q * RPC + r];
+                    fq[q] = mq == -INFINITY ? 0.f : ex2(mq - M);
+                    L += fq[q] * s_l[q * RPC + r];
+                }
+                m_out = M;
+                l_out = L;
+            }
         }
         const float inv = l_out > 0.f ? 1.f / l_out : 0.f;
         const bool writer = row_ok && cp == 0;  // copy 0 holds the merged row
@@ -566,10 +567,10 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
 #pragma unroll
                     for (int q = 0; q < NCP; ++q) {
                         const float4 x = s_o[(q * RPC + r) * (D / 4) + ((c * 8 + k) ^ (r & 7))];
-                        acc.x += x.x;
-                        acc.y += x.y;
-                        acc.z += x.z;
-                        acc.w += x.w;
+                        acc.x = fmaf(fq[q], x.x, acc.x);
+                        acc.y = fmaf(fq[q], x.y, acc.y);
+                        acc.z = fmaf(fq[q], x.z, acc.z);
+                        acc.w = fmaf(fq[q], x.w, acc.w);
                     }
                     o[4 * k] = acc.x;
                     o[4 * k + 1] = acc.y;

@@ -2,12 +2,18 @@
 //
 // A weight-streaming GEMV with n_rows <= 16 right-hand sides, balanced so that every SM
 // streams the same number of weight bytes: one CTA per SM owns an even share of the output
-// features [r0, r1) and splits each weight row into four quarter-rows; its 16 warps take the
-// quarter-rows round-robin, two at a time (14 coalesced 16-byte loads per lane in flight), and
-// store one partial per (feature, quarter), which are summed in a fixed order (deterministic).
-// The input rows are copied once per CTA into shared memory as the concatenation
-// [emb ; hid] (the concatenation only ever exists there).  Weights are read once per group of
-// up to four input rows.
+// features [r0, r1) and splits each weight row into four quarter-rows (items); one partial per
+// (feature, quarter) is stored and the four are summed in a fixed order (deterministic).  The
+// input rows are copied once per CTA into shared memory as the concatenation [emb ; hid] (the
+// concatenation only ever exists there).  Weights are read once per group of up to four input
+// rows.
+//
+// Ring kernel (the weight share's items are contiguous in memory): stage u holds items
+// [16u, 16u + 16), copied by all threads with 16-byte cp.async chunks, S - 1 stages ahead
+// (112 KB in flight per SM for d_model = 3584), so the copies stream continuously; warp w
+// dots item 16u + w with the input rows.
+// Fallback kernel (rows too large for a ring of at least two stages): the 16 warps take the
+// items round-robin, two at a time (14 coalesced 16-byte loads per lane in flight).
 #include "sd_internal.h"
 
 namespace sd {
@@ -106,11 +112,128 @@ hsr_kernel(const uint16_t *emb, const uint16_t *hid, int n_rows, int d_model, co
     }
 }
 
+constexpr int kRingWarps = 16;
+constexpr int kRingThreads = kRingWarps * 32;
+constexpr size_t kRingSmemMax = 227 * 1024;
+
+template <int NR, int S>
+__global__ void __launch_bounds__(kRingThreads, 1)
+hsr_ring_kernel(const uint16_t *emb, const uint16_t *hid, int n_rows, int d_model,
+                const uint16_t *w, const uint16_t *bias, uint16_t *y) {
+    // [NR][cpr] input chunks, then the ring [S][16][cpp] chunks, then [items][NR] f32 partials
+    extern __shared__ __align__(16) uint4 s_x4[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g0 = blockIdx.y * NR;
+    const int nr = min(NR, n_rows - g0);
+    const int cpr = 2 * d_model / 8;  // 16-byte chunks per weight row
+    const int cpp = cpr / kParts;     // chunks per item (quarter-row)
+    const int r0 = (int)((int64_t)d_model * blockIdx.x / gridDim.x);
+    const int r1 = (int)((int64_t)d_model * (blockIdx.x + 1) / gridDim.x);
+    const int items = (r1 - r0) * kParts;
+    uint4 *ring = s_x4 + NR * cpr;
+    float *s_part = reinterpret_cast<float *>(ring + (size_t)S * kRingWarps * cpp);
+    const uint4 *wbase = reinterpret_cast<const uint4 *>(w) + (int64_t)r0 * cpr;
+    const int n_stages = (items + kRingWarps - 1) / kRingWarps;
+    auto issue = [&](int u) {
+        const uint32_t dst = static_cast<uint32_t>(
+            __cvta_generic_to_shared(ring + (size_t)(u % S) * kRingWarps * cpp));
+        const int i0 = u * kRingWarps;
+        const int nchunk = min(kRingWarps, items - i0) * cpp;
+        const uint4 *src = wbase + (int64_t)i0 * cpp;
+        for (int e = tid; e < nchunk; e += kRingThreads) cp_async16(dst + 16u * e, src + e);
+    };
+    for (int u = 0; u < S - 1; ++u) {
+        if (u < n_stages) issue(u);
+        cp_async_commit();
+    }
+    for (int e = tid; e < NR * cpr; e += kRingThreads) {
+        const int r = e / cpr, c = e % cpr;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < nr) {
+            const int col = c * 8;
+            const uint16_t *src = col < d_model ? emb + (int64_t)(g0 + r) * d_model + col
+                                                : hid + (int64_t)(g0 + r) * d_model + (col - d_model);
+            v = *reinterpret_cast<const uint4 *>(src);
+        }
+        s_x4[e] = v;
+    }
+    for (int u = 0; u < n_stages; ++u) {
+        cp_async_wait<S - 2>();
+        __syncthreads();  // stage u has landed for every thread; stage u - 1 is consumed
+        if (u + S - 1 < n_stages) issue(u + S - 1);
+        cp_async_commit();
+        const int it = u * kRingWarps + warp;
+        if (it < items) {
+            const uint4 *wr = ring + (size_t)(u % S) * kRingWarps * cpp + (size_t)warp * cpp;
+            const int col0 = (it % kParts) * cpp;
+            float part[NR];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) part[r] = 0.f;
+            for (int c = lane; c < cpp; c += 32) {
+                float wf[8];
+                Chunk<true>::to_float(wr[c], wf);
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    float xf[8];
+                    Chunk<true>::to_float(s_x4[r * cpr + col0 + c], xf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) part[r] = fmaf(wf[e], xf[e], part[r]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const float sum = warp_sum(part[r]);
+                if (lane == 0) s_part[it * NR + r] = sum;
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    for (int e = tid; e < nr * (r1 - r0); e += kRingThreads) {
+        const int r = e / (r1 - r0), i = e % (r1 - r0);
+        float val = 0.f;
+#pragma unroll
+        for (int q = 0; q < kParts; ++q) val += s_part[((i * kParts + q) * NR) + r];
+        if (bias) val += __uint_as_float((uint32_t)bias[r0 + i] << 16);
+        y[(int64_t)(g0 + r) * d_model + r0 + i] = (uint16_t)f32_to_bf16_bits(val);
+    }
+}
+
+template <int NR, int S>
+cudaError_t launch_ring_t(const void *emb, const void *hid, int n_rows, int d_model,
+                          const void *w, const void *bias, void *y, size_t smem, int ctas,
+                          cudaStream_t s) {
+    auto kern = hsr_ring_kernel<NR, S>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(ctas, (n_rows + NR - 1) / NR);
+    kern<<<grid, kRingThreads, smem, s>>>(
+        reinterpret_cast<const uint16_t *>(emb), reinterpret_cast<const uint16_t *>(hid), n_rows,
+        d_model, reinterpret_cast<const uint16_t *>(w), reinterpret_cast<const uint16_t *>(bias),
+        reinterpret_cast<uint16_t *>(y));
+    return cudaGetLastError();
+}
+
 template <int NR>
 cudaError_t launch_hsr_t(const void *emb, const void *hid, int n_rows, int d_model, const void *w,
                          const void *bias, void *y, cudaStream_t s) {
     const int ctas = min(device_sm_count(), d_model);
     const int max_rows = (d_model + ctas - 1) / ctas;
+    {
+        // ring: as many stages (2..4) as fit next to the input rows and the partials
+        const size_t fixed = (size_t)NR * 2 * d_model * sizeof(uint16_t) +
+                             (size_t)max_rows * kParts * NR * sizeof(float);
+        const size_t stage = (size_t)kRingWarps * (2 * d_model / 8 / kParts) * 16;
+        const int S = fixed < kRingSmemMax ? (int)min((size_t)4, (kRingSmemMax - fixed) / stage)
+                                           : 0;
+        if (S >= 2) {
+            const size_t smem = fixed + (size_t)S * stage;
+            if (S == 2) return launch_ring_t<NR, 2>(emb, hid, n_rows, d_model, w, bias, y, smem, ctas, s);
+            if (S == 3) return launch_ring_t<NR, 3>(emb, hid, n_rows, d_model, w, bias, y, smem, ctas, s);
+            return launch_ring_t<NR, 4>(emb, hid, n_rows, d_model, w, bias, y, smem, ctas, s);
+        }
+    }
     const size_t smem = (size_t)NR * 2 * d_model * sizeof(uint16_t) +
                         (size_t)max_rows * kParts * NR * sizeof(float);
     auto kern = hsr_kernel<NR>;

@@ -26,6 +26,20 @@ struct KVView {
     const int32_t *kv_len;
 };
 
+// 16-byte global -> shared copy through L2 only (cp.async), with its group commit and wait.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ void set_dev_err(int32_t *flag, unsigned bits) {
     if (flag) atomicOr(reinterpret_cast<unsigned *>(flag), bits);
 }

@@ -52,19 +52,6 @@ __device__ __forceinline__ void cand_range(const TopkParams &p, int b, int &cb, 
 // 3 for fp32 rows
 constexpr int score_stages(int row_bytes) { return row_bytes >= 512 ? 3 : 4; }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // Shared-memory chunk slot of chunk ch of tile row `row`.  A quarter-warp (the unit of a
 // 16-byte shared load) covers two rows x four threads; thread j of a row reads chunks
 // j, j + 4, ...; flipping bit 2 of the slot on odd rows puts the two rows on disjoint bank
