@@ -9,8 +9,9 @@
 // not ascending sets SD_DEVERR_INDEX (the result is then unspecified, as for every engine).
 //
 // Grid (parts, h_kv, batch): part r copies the kept entries among list entries
-// [k*r/parts, k*(r+1)/parts); each CTA first counts the kept entries before its range.  Warps
-// copy two rows (d = 128) or four (d = 64) per 16-byte-per-lane instruction.
+// [k*r/parts, k*(r+1)/parts); each CTA first counts the kept entries before its range (about
+// eight CTAs per SM, all resident at once).  Warps copy two rows (d = 128) or four (d = 64) per
+// 16-byte-per-lane instruction, four such row groups loaded before any is stored.
 #include "attn_stream.cuh"
 
 namespace sd {
@@ -82,21 +83,34 @@ __global__ void __launch_bounds__(kThreads) sparse_compact_kernel(const AttnPara
             p.cpos[row0 + slot] = x;
             off = kv_row_offset(p.kv, b, g, x, p.dev_err);  // element offset, or -1 (bad page)
         }
-        // copy the chunk's kept rows: each warp takes its own 32 entries
-        for (int r0 = 0; r0 < 32; r0 += RPI) {
-            const int r = r0 + lane / CPR, ch = lane % CPR;
-            const int64_t o = __shfl_sync(0xffffffffu, off, r);
-            const bool kr = (bal >> r) & 1u;
-            if (!kr) continue;
-            const int s = base + before + __popc(bal & ((1u << r) - 1u));
-            const int64_t dst = (row0 + s) * CPR + ch;
-            uint4 kx = make_uint4(0, 0, 0, 0), vx = make_uint4(0, 0, 0, 0);
-            if (o >= 0) {
-                kx = ldg_stream16(kb + o / 8 + ch);
-                vx = ldg_stream16(vb + o / 8 + ch);
+        // copy the chunk's kept rows: each warp takes its own 32 entries, loading kBatch
+        // row groups before storing them so that several loads per lane are in flight
+        constexpr int kBatch = 4;
+        for (int r0 = 0; r0 < 32; r0 += RPI * kBatch) {
+            uint4 kx[kBatch], vx[kBatch];
+            int64_t dst[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int r = r0 + u * RPI + lane / CPR, ch = lane % CPR;
+                const int64_t o = __shfl_sync(0xffffffffu, off, r);
+                const bool kr = r < 32 && ((bal >> r) & 1u);
+                dst[u] = -1;
+                kx[u] = make_uint4(0, 0, 0, 0);
+                vx[u] = make_uint4(0, 0, 0, 0);
+                if (kr) {
+                    dst[u] = (row0 + base + before + __popc(bal & ((1u << r) - 1u))) * CPR + ch;
+                    if (o >= 0) {
+                        kx[u] = ldg_stream16(kb + o / 8 + ch);
+                        vx[u] = ldg_stream16(vb + o / 8 + ch);
+                    }
+                }
             }
-            ck[dst] = kx;
-            cv[dst] = vx;
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                if (dst[u] >= 0) {
+                    ck[dst[u]] = kx[u];
+                    cv[dst[u]] = vx[u];
+                }
         }
         base += total;
         __syncthreads();  // s_warp is reused by the next chunk
@@ -108,7 +122,7 @@ __global__ void __launch_bounds__(kThreads) sparse_compact_kernel(const AttnPara
 
 cudaError_t launch_sparse_compact(const AttnParams &p, cudaStream_t s) {
     const int units = p.batch * p.kv.h_kv;
-    const int want = (2 * device_sm_count() + units - 1) / units;  // about two CTAs per SM
+    const int want = (8 * device_sm_count() + units - 1) / units;  // about eight CTAs per SM
     const int by_len = (p.k_sel + 127) / 128;
     const int parts = max(1, min(want, by_len));
     dim3 grid(parts, p.kv.h_kv, p.batch);
