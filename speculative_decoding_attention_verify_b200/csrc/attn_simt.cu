@@ -428,13 +428,8 @@ template <bool BF16, int D, int RB>
 cudaError_t launch_simt_t(const AttnParams &p, const AttnPlan &plan, cudaStream_t s) {
     const size_t dyn = SimtCfg<BF16, D>::DYN;
     auto kern = attn_simt_kernel<BF16, D, RB>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)dyn);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = set_max_dynamic_smem<attn_simt_kernel<BF16, D, RB>>((int)dyn);
+    if (e != cudaSuccess) return e;
     dim3 grid(p.n_splits * plan.n_rowblocks, p.kv.h_kv, p.batch);
     kern<<<grid, kThreads, dyn, s>>>(p);
     return cudaGetLastError();

@@ -634,13 +634,8 @@ constexpr int kNcp2Rows = 64;  // largest row count per KV head served with two 
 template <int D, bool PAGED, int NCP>
 cudaError_t launch_t(const AttnParams &p, const TcMaps &maps, cudaStream_t s) {
     auto kern = attn_tc_kernel<D, PAGED, NCP>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Cfg<D>::kSmem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = set_max_dynamic_smem<attn_tc_kernel<D, PAGED, NCP>>(Cfg<D>::kSmem);
+    if (e != cudaSuccess) return e;
     dim3 grid(p.n_splits, p.kv.h_kv, p.batch);
     kern<<<grid, kThreads, Cfg<D>::kSmem, s>>>(p, maps);
     return cudaGetLastError();

@@ -1,6 +1,8 @@
 // Device-side helpers shared by the kernels of libsdattn (sm_100a).
 #pragma once
 
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -25,6 +27,21 @@ struct KVView {
     int num_pages;
     const int32_t *kv_len;
 };
+
+// Opt kernel Kern in to `bytes` of dynamic shared memory, once per device (the attribute is
+// per device, and a process may drive several).  `bytes` must be the same on every call.
+template <auto Kern>
+cudaError_t set_max_dynamic_smem(int bytes) {
+    static std::atomic<unsigned long long> done{0};  // bit d: set on device d
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 // 16-byte global -> shared copy through L2 only (cp.async), with its group commit and wait.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {

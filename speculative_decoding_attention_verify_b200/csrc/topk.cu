@@ -380,12 +380,8 @@ template <bool BF16, int D>
 cudaError_t launch_score_t(const TopkParams &p, cudaStream_t s) {
     const int dyn = score_stages(D * (BF16 ? 2 : 4)) * kScoreTile * D * (BF16 ? 2 : 4);
     auto kern = topk_score_kernel<BF16, D>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = set_max_dynamic_smem<topk_score_kernel<BF16, D>>(dyn);
+    if (e != cudaSuccess) return e;
     dim3 grid(p.n_splits, p.kv.h_kv, p.batch);
     kern<<<grid, kScoreThreads, dyn, s>>>(p);
     return cudaGetLastError();
@@ -410,14 +406,9 @@ cudaError_t launch_topk(const TopkParams &p, cudaStream_t s) {
     dim3 grid(p.kv.h_kv, p.batch);
     if (p.max_cand <= kSmemKeys) {
         const size_t dyn = (size_t)p.max_cand * sizeof(unsigned long long);
-        static bool attr_set = false;
-        if (!attr_set) {
-            e = cudaFuncSetAttribute(topk_select_smem_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)(kSmemKeys * sizeof(unsigned long long)));
-            if (e != cudaSuccess) return e;
-            attr_set = true;
-        }
+        e = set_max_dynamic_smem<topk_select_smem_kernel>(
+            (int)(kSmemKeys * sizeof(unsigned long long)));
+        if (e != cudaSuccess) return e;
         topk_select_smem_kernel<<<grid, kSelectThreads, dyn, s>>>(p);
     } else {
         topk_select_kernel<<<grid, kSelectThreads, 0, s>>>(p);
