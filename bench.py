@@ -459,46 +459,46 @@ def run_ours(args):
 # ---------------------------------------------------------------- oracle on the host -------
 
 def cpu_baseline(w, layers=1):
-    """Time the fp64 oracle on a bounded sample of the same workload (one layer of every
-    attention call, plus HSR and acceptance); report GB/s of algorithmic bytes."""
+    """Time the fp64 oracle on a bounded sample of the same workload: one whole cycle (top-K,
+    every draft step's sparse attention, HSR projection and text-anchored attention, verify,
+    greedy and sampling acceptance) restricted to the first `layers` layers of the attention
+    calls; report GB/s of algorithmic bytes."""
     import oracle
     threads = oracle.set_threads(0)
-    t_total = 0.0
-    bytes_total = 0
     g = int(w.gamma[0])
     n_q = int(w.n_q_verify[0])
     sub = lambda lens: oracle.Cache(w.dtype, w.k[:layers], w.v[:layers], lens[:layers], w.h_kv, w.d)
     full = cycle_bytes(w, [w.kv_len_draft(t) for t in range(g)], w.topk)
     L = w.n_seq
-    t0 = time.perf_counter()
-    idx, _ = oracle.topk_select(w.h_q, w.q_verify[:layers * n_q], w.q_verify_start[:layers + 1],
-                                sub(w.kv_len_verify), np.zeros(layers, np.int32),
-                                w.l_vis[:layers], w.topk)
-    lens = w.kv_len_draft(0)
-    oracle.sparse_attention(w.h_q, w.q_draft[0][:layers], np.arange(layers + 1), sub(lens), idx,
-                            w.l_vis[:layers])
-    oracle.text_anchored_attention(w.h_q, w.q_draft[0][:layers], np.arange(layers + 1), sub(lens),
-                                   np.zeros(layers, np.int32), w.l_vis[:layers], w.window[:layers])
-    oracle.verify_attention(w.h_q, w.q_verify[:layers * n_q], w.q_verify_start[:layers + 1],
-                            sub(w.kv_len_verify))
-    t_total += time.perf_counter() - t0
-    bytes_total += (full["topk"] + full["verify"]) * layers // L
-    bytes_total += (full["sparse"] + full["text_anchored"]) * layers // (L * g)
     from speculative_decoding_attention_verify_b200 import inputs as gen
     hw = gen.make_hsr_workload(n=1)
     aw = gen.make_accept_workload(2, gammas=[g], batch=1)
     t0 = time.perf_counter()
-    oracle.hsr_project(hw.emb, hw.hid, hw.weight)
+    idx, _ = oracle.topk_select(w.h_q, w.q_verify[:layers * n_q], w.q_verify_start[:layers + 1],
+                                sub(w.kv_len_verify), np.zeros(layers, np.int32),
+                                w.l_vis[:layers], w.topk)
+    for t in range(g):
+        lens = w.kv_len_draft(t)
+        oracle.sparse_attention(w.h_q, w.q_draft[t][:layers], np.arange(layers + 1), sub(lens),
+                                idx, w.l_vis[:layers])
+        oracle.hsr_project(hw.emb, hw.hid, hw.weight)
+        oracle.text_anchored_attention(w.h_q, w.q_draft[t][:layers], np.arange(layers + 1),
+                                       sub(lens), np.zeros(layers, np.int32), w.l_vis[:layers],
+                                       w.window[:layers])
+    oracle.verify_attention(w.h_q, w.q_verify[:layers * n_q], w.q_verify_start[:layers + 1],
+                            sub(w.kv_len_verify))
     oracle.accept_greedy(aw.target_logits, aw.draft_tokens_greedy, aw.gamma, aw.vocab)
     oracle.accept_sample(aw.target_logits, aw.draft_logits, aw.draft_tokens_sampled, aw.u, aw.v,
                          aw.gamma, aw.vocab)
-    t_total += time.perf_counter() - t0
-    bytes_total += full["hsr"] // g + full["accept_greedy"] + full["accept_sample"]
+    t_total = time.perf_counter() - t0
+    per_layer = full["topk"] + full["verify"] + full["sparse"] + full["text_anchored"]
+    bytes_total = per_layer * layers // L + full["hsr"] + full["accept_greedy"] + \
+        full["accept_sample"]
     return {"value": round(bytes_total / t_total / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle", "seconds": round(t_total, 3),
-            "sample": f"{layers} of {L} layers of top-K, one sparse and one text-anchored draft "
-                      f"step, verify; one HSR projection; greedy + sampling acceptance "
-                      f"({t_total:.1f} s on {threads} threads)"}
+            "sample": f"one whole cycle on {layers} of {L} layers: top-K, {g} x (sparse draft "
+                      f"step, HSR projection, text-anchored draft step), verify, greedy + "
+                      f"sampling acceptance ({t_total:.1f} s on {threads} threads)"}
 
 
 def run_reference(args):
