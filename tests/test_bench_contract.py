@@ -1,0 +1,52 @@
+"""The benchmark's host-side contract on CPU: the algorithmic byte count of a cycle and the
+JSON line of the reference arm (the fp64 oracle timed on the host cores)."""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_cycle_bytes_counts_each_operand_once():
+    import bench
+    from speculative_decoding_attention_verify_b200 import inputs as gen
+    w = gen.make_attn_workload(1)  # one layer: 8,192 visual + 512 text positions, gamma 5
+    g = int(w.gamma[0])
+    lens = [w.kv_len_draft(t) for t in range(g)]
+    got = bench.cycle_bytes(w, lens, w.topk)
+    kv_row = w.h_kv * w.d * 2 * 2  # K and V of one position over all KV heads, bf16
+    n_q = int(w.n_q_verify[0])
+    q_and_o = 2 * n_q * w.h_q * w.d * 2
+    assert got["verify"] == int(w.kv_len_verify[0]) * kv_row + q_and_o
+    # top-K reads K of every visual candidate once, the last query row, writes K indices
+    assert got["topk"] == int(w.l_vis[0]) * w.h_kv * w.d * 2 + w.h_q * w.d * 2 + \
+        w.h_kv * w.topk * 4
+    # each draft step: the window (or all non-visual positions) for text-anchored attention,
+    # the selection plus the dense tail for sparse attention, one query row and one output row
+    ta = sum(min(int(w.window[0]), int(w.l_txt[0]) + t + 1) * kv_row + 2 * w.h_q * w.d * 2
+             for t in range(g))
+    sp = sum((w.topk + int(w.l_txt[0]) + t + 1) * kv_row + w.h_kv * w.topk * 4 +
+             2 * w.h_q * w.d * 2 for t in range(g))
+    assert got["text_anchored"] == ta
+    assert got["sparse"] == sp
+
+
+def test_reference_arm_prints_the_contract_line():
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                          "--warmup", "3"], cwd=ROOT, env=env, capture_output=True, text=True,
+                         timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["value"] > 0 and np.isfinite(line["value"])
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["config"]["workload"].startswith("spec-decode cycle")
