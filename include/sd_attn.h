@@ -148,7 +148,10 @@ SD_API sd_status sd_attention_workspace_size(sd_attn_kind kind, const sd_q_desc 
  *     O = softmax(scale * q . k_j  over j <= kv_len[b] - n_q + i) . V
  * computed as split-KV flash-decoding (each split keeps an online softmax; the splits are
  * merged by their log-sum-exp).  q: [rows][h_q][d], out: [rows][h_q][d] (kv dtype).
- * Tensor cores (tcgen05) serve bf16 when G*n_q >= 16 rows; CUDA cores otherwise.
+ * Tensor cores (tcgen05) serve bf16 caches with d = 64 or 128 and at most 128 planned rows
+ * per KV head (G * max_q_rows), when q_data and out are 16-byte aligned and the cache layout
+ * can be described to the copy engine (16-byte aligned base and strides); CUDA cores serve the
+ * rest (fp32 caches, more rows, other layouts).
  */
 SD_API sd_status sd_verify_attention(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
                               int32_t batch, void *out, void *workspace, size_t workspace_bytes,
