@@ -45,6 +45,8 @@ VERIFY_CASES = [
     (1, dict(l_vis=40, l_txt=9, gamma=3)),                     # a single tile
     (1, dict(l_vis=3000, l_txt=100, gamma=11)),                # R = 84 rows: one row copy
     (1, dict(l_vis=3000, l_txt=100, gamma=8)),                 # R = 63: two row copies
+    (0, dict(dtype="bf16", l_vis=1500, l_txt=90, gamma=10)),   # d=64: R = 44, two row copies
+    (0, dict(dtype="bf16", l_vis=1500, l_txt=90, gamma=20)),   # d=64: R = 84, one row copy
 ]
 
 
