@@ -58,12 +58,39 @@ def peak_hbm():
         return 6650.0, "fallback"
 
 
+def strip_comments(src):
+    """C/C++/CUDA source without its comments and with whitespace runs collapsed, so that a
+    change to comments or layout alone leaves the hash of the code unchanged."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":  # string or character literal, escapes included
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash():
+    """Hash of the attention kernels' code (comments and layout excluded)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "speculative_decoding_attention_verify_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.startswith("attn_") or name in ("sd_common.cuh", "sd_internal.h", "tc_ptx.cuh"):
-            h.update(open(os.path.join(csrc, name), "rb").read())
+            with open(os.path.join(csrc, name)) as f:
+                h.update(strip_comments(f.read()).encode())
     return h.hexdigest()[:12]
 
 

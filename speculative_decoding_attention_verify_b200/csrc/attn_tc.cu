@@ -1,27 +1,32 @@
-// Tensor-core (tcgen05 + TMA) split-KV verification attention for bf16 caches.
+// Tensor-core (tcgen05 + TMA) split-KV attention for bf16 caches: dense verification,
+// text-anchored draft attention and sparse draft attention (over a staged selection).
 //
-// Serves sd_verify_attention when the GQA group times the new rows, R = G * n_q, is between
-// 16 and 128 (7B-like layers verify gamma+1 = 6..9 rows with G = 7: R = 42..63).
+// Serves every bf16 attention call with d = 64 or 128 and R = G * max_q_rows <= 128 rows per
+// KV head (7B-like layers: R = 7 for a draft step, 42..63 for verification of 6..9 rows).
 //
 // One CTA per (split, KV head g, sequence b); 6 warps, one CTA per SM:
-//   warps 0-3  softmax: TMEM lane r holds query row r (rows ordered (i, h), h fastest; rows
-//              R..127 are padding and never read back)
-//   warp 4     TMA producer: K and V tiles of 128 positions (128-byte swizzle) into a
-//              3-4 stage shared-memory ring (a stage's K is released once S is computed, its V
-//              once P.V is) (contiguous caches: one 4-D box per half of
-//              head_dim; paged caches: one box per 16-position page)
+//   warps 0-3  softmax: TMEM lane r holds MMA row r; with NCP row copies the R rows are
+//              placed NCP times (copy c in lanes [c * 128/NCP, ...)) and each warp handles
+//              the 128/NCP tile columns of its copy (rows past R are padding, never read back)
+//   warp 4     TMA producer: lane 0 streams K tiles, lane 1 V tiles (128 positions,
+//              128-byte swizzle) into a 3-4 stage shared-memory ring, each through its own
+//              half of every stage (a stage's K is released once S is computed, its V once
+//              P.V is); contiguous caches: one 4-D box per half of head_dim; paged caches: one
+//              box per 16-position page
 //   warp 5     MMA issuer (one elected thread) and TMEM owner
 // Per tile t (double-buffered S in TMEM):
-//   S_t = Q K_t^T        tcgen05.mma kind::f16, M=128, N=128, A = Q (smem, K-major),
-//                        B = K tile (smem, K-major), fp32 accumulators in TMEM
-//   softmax              each thread reads its row of S_t from TMEM, applies the causal
-//                        mask j <= kv_len - n_q + i, updates its running max (base 2) and
-//                        writes P_t = 2^(s - m) as bf16 over S_t in TMEM.  The running max
-//                        used for the exponent only moves when the true max grows by more
-//                        than 2^8 ("lazy rescale"), so O is rarely touched.
+//   S_t = Q K_t^T        tcgen05.mma kind::f16, M=128, N=128, A = Q (TMEM, written once by
+//                        the softmax warps), B = K tile (smem, K-major), fp32 accumulators
+//   softmax              each thread reads its row's columns of S_t from TMEM, applies the
+//                        run bounds and the row's visible ranges, updates its running max
+//                        (base 2) and writes P_t = 2^(s - m) as bf16 over S_t in TMEM.  The
+//                        running max used for the exponent only moves when the true max grows
+//                        by more than 2^8 ("lazy rescale"), so O is rarely touched.
 //   O += P_t V_t         tcgen05.mma with A = P_t from TMEM, B = V tile (smem, MN-major)
-// Partial outputs (O, max, sum) go to the split workspace exactly like the CUDA-core engine,
-// or, with a single split, O / sum is written directly.
+// The issuer issues S of tile t+1 and P.V of tile t in whichever order their operands arrive.
+// The row copies' partial (m, l, O) are merged in shared memory at the end.  Partial outputs
+// (O, max, sum) go to the split workspace exactly like the CUDA-core engine, or, with a single
+// split, O / sum is written directly.
 // Every wait on an mbarrier is bounded (1 s); on expiry the CTA records SD_DEVERR_TIMEOUT,
 // drains its own copies and MMAs (again bounded), frees TMEM and exits.
 #include "attn_stream.cuh"
@@ -142,7 +147,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         }
         mbar_init(BAR(OD), 1);
         mbar_init(BAR(DR), 1);
-        mbar_init(BAR(QF), 128);  // Q in shared memory (warps 0-3)
+        mbar_init(BAR(QF), 128);  // Q in TMEM (warps 0-3)
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
