@@ -229,9 +229,10 @@ cudaError_t launch_hsr_t(const void *emb, const void *hid, int n_rows, int d_mod
                                            : 0;
         if (S >= 2) {
             const size_t smem = fixed + (size_t)S * stage;
-            if (S == 2) return launch_ring_t<NR, 2>(emb, hid, n_rows, d_model, w, bias, y, smem, ctas, s);
-            if (S == 3) return launch_ring_t<NR, 3>(emb, hid, n_rows, d_model, w, bias, y, smem, ctas, s);
-            return launch_ring_t<NR, 4>(emb, hid, n_rows, d_model, w, bias, y, smem, ctas, s);
+            auto ring = S == 2 ? launch_ring_t<NR, 2>
+                        : S == 3 ? launch_ring_t<NR, 3>
+                                 : launch_ring_t<NR, 4>;
+            return ring(emb, hid, n_rows, d_model, w, bias, y, smem, ctas, s);
         }
     }
     const size_t smem = (size_t)NR * 2 * d_model * sizeof(uint16_t) +
