@@ -50,3 +50,14 @@ def test_reference_arm_prints_the_contract_line():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"].startswith("spec-decode cycle")
+
+
+def test_code_hash_ignores_comments_but_not_code():
+    import bench
+    a = 'int f(int x) { // scale\n    return 2 * x; /* twice */ }\nconst char *s = "a // b";\n'
+    b = 'int f(int x) {\n  return 2 * x;\n}\n// a new comment line\nconst char *s = "a // b";'
+    c = 'int f(int x) { return 3 * x; }\nconst char *s = "a // b";'
+    d = 'int f(int x) { return 2 * x; }\nconst char *s = "a /* b";'
+    assert bench.strip_comments(a) == bench.strip_comments(b)
+    assert bench.strip_comments(a) != bench.strip_comments(c)
+    assert bench.strip_comments(a) != bench.strip_comments(d)  # string contents count
