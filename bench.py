@@ -1,28 +1,35 @@
 #!/usr/bin/env python
-"""Benchmark: one speculative-decoding cycle at 25k visual tokens through libsdattn.
+"""Benchmark: one speculative-decoding cycle through libsdattn, on synthetic seeded inputs.
 
-One *step* runs every call of the hot path once per its role in a cycle, over 28 independent
-layers (H_q=28, H_kv=4, d=128, bf16, 25,000 visual + 1,024 text positions, gamma = 8, vocab
-152,064), on synthetic seeded inputs:
-  top-K selection (K=1024 per KV head over the visual span)              1 launch group
-  8 draft steps x [sparse attention, HSR projection, text-anchored]       28 layers each
-  dense verification of the 9 new rows                                   28 layers
-  greedy acceptance and speculative-sampling acceptance                  batch 1
-The metric is algorithmic bytes moved by the step (KV, queries, outputs, weights, logits;
-implementation scratch not credited) divided by the step's device time: "spec-decode
-attention KV-read GB/s".  Inputs (1.49 GB of KV) exceed the L2 cache, so no flush is needed.
+Default workload (the long-video Sparse-to-Dense configuration, every call of the path): 28
+independent layers (H_q=28, H_kv=4, d=128, bf16, 25,000 visual + 1,024 text positions),
+gamma = 8, vocab 152,064.  One *step* is one cycle:
+  top-K selection (K=1024 per KV head over the visual span) and staging of the kept rows
+  8 draft steps x [sparse attention, HSR projection, text-anchored attention]   28 layers each
+  dense verification of the 9 new rows                                         28 layers
+  greedy acceptance and speculative-sampling acceptance                        batch 1
+The metric is the algorithmic bytes the step must move (KV rows, queries, outputs, weights,
+logits; implementation scratch not credited) over the step's device time: "spec-decode
+attention KV-read GB/s".  The step reads 4 GB (1.49 GB of KV for verification alone), far
+more than the 126 MB L2, so no flush is needed between steps; each of the 8 HSR projections
+reads its own copy of the 51.4 MB weight.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Besides the headline the JSON line carries, per call kind, a roofline measured with L2
+flushed before every call (`rooflines`), one-layer latencies, the cycle of each drafting
+method against plain decoding (gamma single-row dense decode steps), the end-to-end figure
+through the public API with host buffers, and the fp64 oracle timed on the host.
 
-With N > 1 (torchrun) every rank runs its own replica of the workload; the path has no
-exchange step, so there is no data-path collective (time is the max over ranks).
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
+
+``--config 0..4`` prints the line of another workload instead (its own set of calls).  With
+N > 1 (torchrun) every rank runs its own replica; the path has no exchange step, so there is
+no data-path collective (time is the max over ranks).
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -34,14 +41,33 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = dict(workload="spec-decode cycle, 28 layers, L_vis=25000, L_txt=1024, gamma=8, "
-                         "H_q=28, H_kv=4, d=128, bf16, top-K 1024, window 1024, vocab 152064",
-                layers=28, l_vis=25000, l_txt=1024, gamma=8, h_q=28, h_kv=4, head_dim=128,
-                topk=1024, window=1024, vocab=152064, hsr_d_model=3584,
-                l2="inputs larger than L2 (1.49 GB of KV per step)",
-                parallelism="replicas (no data-path collective)")
 METRIC = "spec-decode attention KV-read GB/s (% of B200 HBM peak) at 25k vis tokens"
-CFG_INDEX = 3  # the Sparse-to-Dense configuration carries every call of the path
+DEFAULT_CONFIG = 3
+NOMINAL_HBM_GBS = 8000.0
+FLUSH_BYTES = 1 << 30        # written before every separately timed call (L2 is 126 MB)
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+
+# Calls of each workload's cycle.  sparse: "staged" (selection staged once per cycle, bf16),
+# "direct" (gathered by every call) or None; draft_steps None means the workload's gamma.
+SPECS = {
+    0: dict(topk=True, sparse="direct", ta=True, hsr=False, accept=True, draft_steps=None),
+    1: dict(topk=False, sparse=None, ta=True, hsr=True, accept=False, draft_steps=None),
+    2: dict(topk=False, sparse=None, ta=True, hsr=True, accept=True, draft_steps=None),
+    3: dict(topk=True, sparse="staged", ta=True, hsr=True, accept=True, draft_steps=None),
+    4: dict(topk=True, sparse=None, ta=True, hsr=False, accept=True, draft_steps=1),
+}
+
+KERNELS = {  # call kind -> the library kernels one call launches
+    "topk": "topk_score_kernel + topk_select_smem_kernel",
+    "stage": "sparse_compact_kernel",
+    "sparse": "attn_tc_kernel (+ attn_merge_kernel when split)",
+    "sparse_direct": "attn_* engine (+ attn_merge_kernel when split)",
+    "hsr": "hsr_ring_kernel",
+    "text_anchored": "attn_tc_kernel (+ attn_merge_kernel when split)",
+    "verify": "attn_tc_kernel + attn_merge_kernel",
+    "accept_greedy": "accept_argmax_kernel + accept_greedy_kernel",
+    "accept_sample": "accept_stats/decide/wsum/draw kernels",
+}
 
 
 def env_rank():
@@ -84,219 +110,487 @@ def strip_comments(src):
 
 
 def kernel_source_hash():
-    """Hash of the attention kernels' code (comments and layout excluded)."""
+    """Hash of the library's code: every CUDA/C++ source and header of the package and the
+    public header (comments and layout excluded), so that a change to any kernel or to the
+    planner invalidates recorded counters."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "speculative_decoding_attention_verify_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.startswith("attn_") or name in ("sd_common.cuh", "sd_internal.h", "tc_ptx.cuh"):
-            with open(os.path.join(csrc, name)) as f:
-                h.update(strip_comments(f.read()).encode())
+    files = [os.path.join(csrc, n) for n in sorted(os.listdir(csrc))
+             if n.endswith((".cu", ".cuh", ".h", ".cpp"))]
+    files.append(os.path.join(ROOT, "include", "sd_attn.h"))
+    for path in files:
+        with open(path) as f:
+            h.update(strip_comments(f.read()).encode())
     return h.hexdigest()[:12]
 
 
 def recorded_traffic():
-    """DRAM bytes per verify launch from the committed ncu summary, if the kernel is unchanged."""
-    path = os.path.join(ROOT, "profiles", "verify_attention_c3_ncu.md")
+    """DRAM bytes (read + write) per launch of each call kind, from the committed ncu record,
+    for the entries taken on the current code; {} when none matches."""
     try:
-        text = open(path).read()
-    except OSError:
-        return None
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return {}
     want = kernel_source_hash()
-    for line in text.splitlines():
-        if line.startswith("traffic_bytes_per_full_launch:"):
-            parts = line.split()
-            if len(parts) >= 4 and parts[3] == want:
-                return float(parts[1])
-    return None
+    return {k: float(v["traffic_bytes_per_launch"]) for k, v in rec.get("calls", {}).items()
+            if v.get("source_hash") == want}
 
 
 # ---------------------------------------------------------------- algorithmic bytes --------
 
-def cycle_bytes(w, lens_draft, topk):
-    """Bytes the method must move in one step, per call kind (algorithmic bytes: every operand
-    the step reads or writes once; scratch is not credited)."""
-    d, hk, hq, s = w.d, w.h_kv, w.h_q, 2
+def call_bytes(w, kind, step=0, topk=None, hsr_d=None, aw=None):
+    """Bytes one call must move (every operand it reads or writes once; scratch and staging
+    not credited).  w: the attention workload; step: the draft step (0-based)."""
+    d, hk, hq = w.d, w.h_kv, w.h_q
+    s = 2 if w.dtype == "bf16" else 4
     row = hk * d * 2 * s  # K and V of one position, all KV heads
     L = w.n_seq
-    n_q = int(w.n_q_verify[0])
-    out = {}
-    out["verify"] = int(w.kv_len_verify.sum()) * row + 2 * L * n_q * hq * d * s
-    ctx_txt = int(w.l_txt[0])
-    ta = 0
-    sp = 0
-    for t in range(len(lens_draft)):
-        nonvis = ctx_txt + t + 1
-        ta += L * min(int(w.window[0]), nonvis) * row + 2 * L * hq * d * s
-        tail = nonvis
-        sp += L * (topk + tail) * row + L * hk * topk * 4 + 2 * L * hq * d * s
-    out["text_anchored"] = ta
-    out["sparse"] = sp
-    out["topk"] = L * int(w.l_vis[0]) * hk * d * s + L * hq * d * s + L * hk * topk * 4
-    D = WORKLOAD["hsr_d_model"]
-    out["hsr"] = len(lens_draft) * (D * 2 * D * 2 + (2 * D + D) * 2)
-    V, g = WORKLOAD["vocab"], WORKLOAD["gamma"]
-    out["accept_greedy"] = (g + 1) * V * 4 + g * 4
-    out["accept_sample"] = (2 * g + 1) * V * 4 + 2 * V * 4 + g * 4 + (2 * g + 1) * 4
-    return out
+    qo = 2 * hq * d * s   # one query row in, one output row out
+    nonvis = (w.l_txt + step + 1).astype(np.int64)  # text positions + the draft's own
+    if kind == "verify":
+        return int(w.kv_len_verify.astype(np.int64).sum()) * row + int(w.n_q_verify.sum()) * qo
+    if kind == "text_anchored":
+        return int(np.minimum(w.window, nonvis).sum()) * row + L * qo
+    if kind in ("sparse", "sparse_direct"):
+        kept = np.minimum(topk, w.l_vis).astype(np.int64)
+        return int((kept + nonvis).sum()) * row + L * hk * topk * 4 + L * qo
+    if kind == "topk":
+        return int(w.l_vis.astype(np.int64).sum()) * hk * d * s + L * hq * d * s + L * hk * topk * 4
+    if kind == "stage":  # staging copy of the kept rows (implementation traffic, not credited)
+        kept = int(np.minimum(topk, w.l_vis).sum())
+        return 2 * kept * row + L * hk * topk * 4
+    if kind == "hsr":
+        return hsr_d * 2 * hsr_d * 2 + 3 * hsr_d * 2
+    g = aw.gamma.astype(np.int64)
+    V = aw.vocab
+    if kind == "accept_greedy":
+        return int((g + 1).sum()) * V * 4 + int(g.sum()) * 4
+    if kind == "accept_sample":
+        return int((2 * g + 1).sum()) * V * 4 + 2 * V * 4 * aw.batch + int(g.sum()) * 8 + \
+            int((g + 1).sum()) * 4
+    raise ValueError(kind)
 
 
-# ---------------------------------------------------------------- the GPU step -------------
+# ---------------------------------------------------------------- the GPU cycle ------------
 
 class Cycle:
-    def __init__(self, device):
+    """Device tensors and the ordered calls of one cycle of workload `cfg`.
+
+    Per-step inputs that a caller would bring from the host (queries, embeddings, logits,
+    drafted tokens, uniforms) exist twice on the device, so that the end-to-end run can copy
+    the next step's inputs while the current step computes; `step(stream, buf)` uses set
+    `buf`.  Everything else (caches, selection, workspaces, outputs) exists once."""
+
+    def __init__(self, cfg, device):
         import torch
         from speculative_decoding_attention_verify_b200 import device as dev
         from speculative_decoding_attention_verify_b200 import inputs as gen
         from speculative_decoding_attention_verify_b200 import sdattn as sd
         self.torch, self.sd, self.dev, self.gen = torch, sd, dev, gen
-        w = gen.make_attn_workload(CFG_INDEX)
+        self.cfg, self.spec = cfg, SPECS[cfg]
+        w = gen.make_attn_workload(cfg)
         self.w = w
-        g = int(w.gamma[0])
-        self.gamma = g
         L = w.n_seq
+        self.g = int(self.spec["draft_steps"] or w.gamma_max)
+        i32 = lambda a: dev.int32(np.asarray(a), device)
         self.k = dev.tensor(w.k, w.dtype, device)
         self.v = dev.tensor(w.v, w.dtype, device)
-        self.kv_verify = dev.kv_cache(w, device=device, k=self.k, v=self.v)
-        self.lens_draft = [w.kv_len_draft(t) for t in range(g)]
-        self.kv_draft = [dev.kv_cache(w, kv_len=l, device=device, k=self.k, v=self.v)
-                         for l in self.lens_draft]
-        self.q_verify = dev.verify_queries(w, device)
-        self.q_draft = [dev.draft_queries(w, t, device) for t in range(g)]
-        self.cand_b = dev.int32(np.zeros(L, np.int32), device)
-        self.cand_e = dev.int32(w.l_vis, device)
-        self.tail = dev.int32(w.l_vis, device)
-        self.vis_b = dev.int32(np.zeros(L, np.int32), device)
-        self.vis_e = dev.int32(w.l_vis, device)
-        self.win = dev.int32(w.window, device)
+        kvc = lambda lens: dev.kv_cache(w, kv_len=lens, device=device, k=self.k, v=self.v)
+        self.kv_verify = kvc(w.kv_len_verify)
+        self.kv_draft = [kvc(w.kv_len_draft(t)) for t in range(self.g)]
         self.topk = w.topk
+        # per-step inputs, two sets
+        self.q_verify = [dev.verify_queries(w, device) for _ in range(2)]
+        self.q_draft = [[dev.draft_queries(w, t, device) for t in range(self.g)] for _ in range(2)]
+        self.cand_b, self.cand_e = i32(np.zeros(L)), i32(w.l_vis)
+        self.max_cand = int(w.l_vis.max())
+        self.tail = i32(w.l_vis)
+        self.vis_b, self.vis_e, self.win = i32(np.zeros(L)), i32(w.l_vis), i32(w.window)
+        self.max_win = int(w.window.max())
+        self.max_tail = int(max(int((w.kv_len_draft(t) - w.l_vis).max()) for t in range(self.g)))
         self.idx = torch.empty((L, w.h_kv, w.topk), dtype=torch.int32, device=device)
-        self.max_tail = int(max(int((l - w.l_vis).max()) for l in self.lens_draft))
-        hw = gen.make_hsr_workload(n=1)
-        self.hsr_np = hw
-        self.emb = [dev.tensor(hw.emb, gen.BF16, device) for _ in range(g)]
-        self.hid = dev.tensor(hw.hid, gen.BF16, device)
-        self.W = dev.tensor(hw.weight, gen.BF16, device)
-        self.y = torch.empty((1, hw.d_model), dtype=torch.bfloat16, device=device)
-        aw = gen.make_accept_workload(2, gammas=[g], batch=1)
-        self.aw = aw
-        t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
-        self.tgt, self.drf = t(aw.target_logits), t(aw.draft_logits)
-        self.tok_s, self.tok_g = t(aw.draft_tokens_sampled), t(aw.draft_tokens_greedy)
-        self.u, self.vv, self.gam = t(aw.u), t(aw.v), t(aw.gamma)
-        # outputs and workspaces allocated once
-        self.o_verify = torch.empty_like(self.q_verify.q)
-        self.o_draft = [torch.empty_like(q.q) for q in self.q_draft]
-        self.o_ta = [torch.empty_like(q.q) for q in self.q_draft]
         mk = lambda n: torch.empty(max(int(n), 16), dtype=torch.uint8, device=device)
-        self.ws_verify = mk(sd.sd_attention_workspace_size(sd.SD_ATTN_VERIFY, self.q_verify,
+        self.ws_verify = mk(sd.sd_attention_workspace_size(sd.SD_ATTN_VERIFY, self.q_verify[0],
                                                            self.kv_verify))
-        self.ws_sparse = mk(sd.sd_sparse_workspace_size(self.q_draft[-1], self.kv_draft[-1],
-                                                        w.topk, self.max_tail))
-        self.ws_ta = mk(sd.sd_attention_workspace_size(sd.SD_ATTN_TEXT_ANCHORED, self.q_draft[-1],
-                                                       self.kv_draft[-1]))
-        self.ws_topk = mk(sd.sd_topk_workspace_size(self.kv_verify, int(w.l_vis.max()), w.topk))
-        # the top-K rows are staged once per cycle and read by every draft step
-        self.sel = mk(sd.sd_sparse_selection_size(self.kv_draft[0], w.topk))
-        self.ws_acc = mk(sd.sd_accept_workspace_size(1, g, aw.vocab))
-        self.n_acc_g = torch.empty(1, dtype=torch.int32, device=device)
-        self.out_g = torch.empty((1, g + 1), dtype=torch.int32, device=device)
-        self.n_acc_s = torch.empty(1, dtype=torch.int32, device=device)
-        self.out_s = torch.empty((1, g + 1), dtype=torch.int32, device=device)
-        self.near = torch.empty(1, dtype=torch.int32, device=device)
-        self.bytes = cycle_bytes(w, self.lens_draft, w.topk)
-        self.verify_events = []
+        self.ws_ta = mk(sd.sd_attention_workspace_size(sd.SD_ATTN_TEXT_ANCHORED,
+                                                       self.q_draft[0][-1], self.kv_draft[-1]))
+        self.o_verify = torch.empty_like(self.q_verify[0].q)
+        self.o_draft = [torch.empty_like(q.q) for q in self.q_draft[0]]
+        self.o_ta = [torch.empty_like(q.q) for q in self.q_draft[0]]
+        if self.spec["topk"]:
+            self.ws_topk = mk(sd.sd_topk_workspace_size(self.kv_verify, self.max_cand, w.topk))
+        if self.spec["sparse"]:
+            self.ws_sparse = mk(sd.sd_sparse_workspace_size(self.q_draft[0][-1],
+                                                            self.kv_draft[-1], w.topk,
+                                                            self.max_tail))
+        if self.spec["sparse"] == "staged":
+            self.sel = mk(sd.sd_sparse_selection_size(self.kv_draft[0], w.topk))
+        self.hsr_d = None
+        if self.spec["hsr"]:
+            hw = gen.make_hsr_workload(n=1)
+            self.hsr_d = hw.d_model
+            base = dev.tensor(hw.weight, gen.BF16, device)
+            # one weight copy per draft step: 8 x 51.4 MB, so no projection finds its weight
+            # in L2
+            self.W = [base] + [base.clone() for _ in range(self.g - 1)]
+            self.emb = [[dev.tensor(hw.emb, gen.BF16, device) for _ in range(self.g)]
+                        for _ in range(2)]
+            self.hid = dev.tensor(hw.hid, gen.BF16, device)
+            self.y = [torch.empty((1, hw.d_model), dtype=torch.bfloat16, device=device)
+                      for _ in range(self.g)]
+        self.aw = None
+        if self.spec["accept"]:
+            if cfg in (2, 3):  # one sequence whose 28 layers were attended above
+                aw = gen.make_accept_workload(2, gammas=[self.g], batch=1)
+            else:
+                aw = gen.make_accept_workload(cfg, gammas=w.gamma)
+            self.aw = aw
+            t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+            self.acc_in = [dict(tgt=t(aw.target_logits), drf=t(aw.draft_logits),
+                                tok_s=t(aw.draft_tokens_sampled),
+                                tok_g=t(aw.draft_tokens_greedy), u=t(aw.u), v=t(aw.v))
+                           for _ in range(2)]
+            self.gam = t(aw.gamma)
+            self.gmax = int(aw.gamma.max())
+            B = aw.batch
+            self.ws_acc = mk(sd.sd_accept_workspace_size(B, self.gmax, aw.vocab))
+            self.n_acc_g = torch.empty(B, dtype=torch.int32, device=device)
+            self.out_g = torch.empty((B, self.gmax + 1), dtype=torch.int32, device=device)
+            self.n_acc_s = torch.empty(B, dtype=torch.int32, device=device)
+            self.out_s = torch.empty((B, self.gmax + 1), dtype=torch.int32, device=device)
+            self.near = torch.empty(B, dtype=torch.int32, device=device)
+        self.calls = self._calls()
+        self.bytes = {}
+        for kind, step, _ in self.calls:
+            if kind == "stage":
+                continue
+            self.bytes[kind] = self.bytes.get(kind, 0) + self.call_bytes(kind, step)
 
-    def launches_per_step(self, graph=None):
-        """Kernels one step launches: counted from the captured CUDA graph (kernel nodes; every
-        kernel of the step is libsdattn's), else an upper bound from the call structure."""
-        if graph is not None:
-            try:
-                from cuda.bindings import runtime as rt
-                h = rt.cudaGraph_t(init_value=int(graph.raw_cuda_graph()))
-                err, _, n = rt.cudaGraphGetNodes(h, 0)
-                err2, nodes, n = rt.cudaGraphGetNodes(h, n)
-                if err == rt.cudaError_t.cudaSuccess and err2 == rt.cudaError_t.cudaSuccess:
-                    kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
-                    return sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel)
-            except Exception:  # noqa: BLE001 - fall back to the structural count
-                pass
-        g = self.gamma
-        # top-K (score, select), staging; per draft step sparse (attention, merge), HSR,
-        # text-anchored (attention, merge); verify (attention, merge); greedy (2); sampling (4)
-        return 2 + 1 + g * 2 + g + g * 2 + 2 + 2 + 4
+    def call_bytes(self, kind, step=0):
+        return call_bytes(self.w, kind, step, topk=self.topk, hsr_d=self.hsr_d, aw=self.aw)
 
-    def step(self, stream=None, time_verify=False):
+    # ---- the calls, in cycle order: (kind, draft step, fn(stream, buf)) ----
+    def _calls(self):
+        sd, sp = self.sd, self.spec
+        calls = []
+        if sp["topk"]:
+            calls.append(("topk", 0, lambda s, b: sd.sd_topk_select(
+                self.q_verify[b], self.kv_verify, self.cand_b, self.cand_e, self.max_cand,
+                self.topk, idx_out=self.idx, workspace=self.ws_topk, stream=s)))
+        if sp["sparse"] == "staged":
+            calls.append(("stage", 0, lambda s, b: sd.sd_sparse_stage(
+                self.kv_draft[0], self.idx, self.tail, selection=self.sel, stream=s)))
+        for t in range(self.g):
+            if sp["sparse"] == "staged":
+                calls.append(("sparse", t, lambda s, b, t=t: sd.sd_sparse_attention_staged(
+                    self.q_draft[b][t], self.kv_draft[t], self.sel, self.topk, self.tail,
+                    self.max_tail, out=self.o_draft[t], workspace=self.ws_sparse, stream=s)))
+            elif sp["sparse"] == "direct":
+                calls.append(("sparse_direct", t, lambda s, b, t=t: sd.sd_sparse_attention(
+                    self.q_draft[b][t], self.kv_draft[t], self.idx, self.tail, self.max_tail,
+                    out=self.o_draft[t], workspace=self.ws_sparse, stream=s)))
+            if sp["hsr"]:
+                calls.append(("hsr", t, lambda s, b, t=t: sd.sd_hsr_project(
+                    self.emb[b][t], self.hid, self.W[t], out=self.y[t], stream=s)))
+            if sp["ta"]:
+                calls.append(("text_anchored", t, lambda s, b, t=t: sd.sd_text_anchored_attention(
+                    self.q_draft[b][t], self.kv_draft[t], self.vis_b, self.vis_e, self.win,
+                    self.max_win, out=self.o_ta[t], workspace=self.ws_ta, stream=s)))
+        calls.append(("verify", 0, lambda s, b: sd.sd_verify_attention(
+            self.q_verify[b], self.kv_verify, out=self.o_verify, workspace=self.ws_verify,
+            stream=s)))
+        if sp["accept"]:
+            calls.append(("accept_greedy", 0, lambda s, b: sd.sd_accept_greedy(
+                self.acc_in[b]["tgt"], self.acc_in[b]["tok_g"], self.gam, self.gmax,
+                n_acc=self.n_acc_g, out_tok=self.out_g, workspace=self.ws_acc, stream=s)))
+            calls.append(("accept_sample", 0, lambda s, b: sd.sd_accept_sample(
+                self.acc_in[b]["tgt"], self.acc_in[b]["drf"], self.acc_in[b]["tok_s"],
+                self.acc_in[b]["u"], self.acc_in[b]["v"], self.gam, self.gmax,
+                n_acc=self.n_acc_s, out_tok=self.out_s, near_boundary=self.near,
+                workspace=self.ws_acc, stream=s)))
+        return calls
+
+    def step(self, stream=None, buf=0, kinds=None):
+        for kind, _, fn in self.calls:
+            if kinds is None or kind in kinds:
+                fn(stream, buf)
+
+    def decode_step_calls(self):
+        """Plain decoding of the draft steps' tokens: each token is one dense single-row
+        attention over the whole cache (verification attention with n_q = 1)."""
         sd = self.sd
-        sd.sd_topk_select(self.q_verify, self.kv_verify, self.cand_b, self.cand_e,
-                          int(self.w.l_vis.max()), self.topk, idx_out=self.idx,
-                          workspace=self.ws_topk, stream=stream)
-        sd.sd_sparse_stage(self.kv_draft[0], self.idx, self.tail, selection=self.sel,
-                           stream=stream)
-        for t in range(self.gamma):
-            sd.sd_sparse_attention_staged(self.q_draft[t], self.kv_draft[t], self.sel, self.topk,
-                                          self.tail, self.max_tail, out=self.o_draft[t],
-                                          workspace=self.ws_sparse, stream=stream)
-            sd.sd_hsr_project(self.emb[t], self.hid, self.W, out=self.y, stream=stream)
-            sd.sd_text_anchored_attention(self.q_draft[t], self.kv_draft[t], self.vis_b,
-                                          self.vis_e, self.win, int(self.w.window.max()),
-                                          out=self.o_ta[t], workspace=self.ws_ta, stream=stream)
-        if time_verify:
-            e0 = self.torch.cuda.Event(enable_timing=True)
-            e1 = self.torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        sd.sd_verify_attention(self.q_verify, self.kv_verify, out=self.o_verify,
-                               workspace=self.ws_verify, stream=stream)
-        if time_verify:
-            e1.record(stream)
-            self.verify_events.append((e0, e1))
-        sd.sd_accept_greedy(self.tgt, self.tok_g, self.gam, self.gamma, n_acc=self.n_acc_g,
-                            out_tok=self.out_g, workspace=self.ws_acc, stream=stream)
-        sd.sd_accept_sample(self.tgt, self.drf, self.tok_s, self.u, self.vv, self.gam, self.gamma,
-                            n_acc=self.n_acc_s, out_tok=self.out_s, near_boundary=self.near,
-                            workspace=self.ws_acc, stream=stream)
+        return [lambda s, t=t: sd.sd_verify_attention(
+            self.q_draft[0][t], self.kv_draft[t], out=self.o_draft[t], workspace=self.ws_verify,
+            stream=s) for t in range(self.g)]
+
+    def one_layer(self, kind):
+        """A call of `kind` over the first layer (sequence) alone: the one-launch-per-layer
+        latency."""
+        sd, dev, w = self.sd, self.dev, self.w
+        if w.paged or w.n_seq == 1:
+            return None
+        k1, v1 = self.k[:1], self.v[:1]
+        torch = self.torch
+        dvc = self.k.device
+        lens = w.kv_len_verify if kind == "verify" else w.kv_len_draft(0)
+        kv = sd.KVCache(k1, v1, torch.tensor(lens[:1], dtype=torch.int32, device=dvc))
+        if kind == "verify":
+            nq = int(w.n_q_verify[0])
+            q = sd.Queries(self.q_verify[0].q[:nq], torch.tensor([0, nq], dtype=torch.int32,
+                                                                  device=dvc), nq, int(lens[0]))
+            out = torch.empty_like(q.q)
+            return lambda s: sd.sd_verify_attention(q, kv, out=out, workspace=self.ws_verify,
+                                                    stream=s)
+        q = sd.Queries(self.q_draft[0][0].q[:1], torch.tensor([0, 1], dtype=torch.int32,
+                                                               device=dvc), 1, int(lens[0]))
+        out = torch.empty_like(q.q)
+        if kind == "text_anchored":
+            return lambda s: sd.sd_text_anchored_attention(
+                q, kv, self.vis_b[:1], self.vis_e[:1], self.win[:1], self.max_win, out=out,
+                workspace=self.ws_ta, stream=s)
+        if kind == "sparse" and self.spec["sparse"] == "staged":
+            sel = self.torch.empty(max(sd.sd_sparse_selection_size(kv, self.topk), 16),
+                                   dtype=torch.uint8, device=dvc)
+            sd.sd_sparse_stage(kv, self.idx[:1].contiguous(), self.tail[:1], selection=sel)
+            ws = self.torch.empty(max(sd.sd_sparse_workspace_size(q, kv, self.topk,
+                                                                  self.max_tail), 16),
+                                  dtype=torch.uint8, device=dvc)
+            return lambda s: sd.sd_sparse_attention_staged(q, kv, sel, self.topk,
+                                                           self.tail[:1], self.max_tail,
+                                                           out=out, workspace=ws, stream=s)
+        return None
+
+    def count_graph_kernels(self, graph):
+        """Kernel nodes of a captured CUDA graph (every kernel of the cycle is libsdattn's)."""
+        try:
+            from cuda.bindings import runtime as rt
+            h = rt.cudaGraph_t(init_value=int(graph.raw_cuda_graph()))
+            err, _, n = rt.cudaGraphGetNodes(h, 0)
+            err2, nodes, n = rt.cudaGraphGetNodes(h, n)
+            if err == rt.cudaError_t.cudaSuccess and err2 == rt.cudaError_t.cudaSuccess:
+                kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+                return sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel)
+        except Exception:  # noqa: BLE001 - counted from the call structure below instead
+            pass
+        return None
 
 
-class HostInputs:
-    """Per-step inputs in pinned host memory for the end-to-end measurement."""
+def capture(torch, fn):
+    """Warm fn up eagerly, then capture one call of fn(stream) in a CUDA graph."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn(s)
+        fn(s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        fn(s)
+    torch.cuda.synchronize()
+    return graph
+
+
+def time_graph(torch, graph, reps, warmup=3):
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+class Flusher:
+    """Writes a buffer larger than L2 before a separately timed call, and times the call with
+    CUDA events on the launching stream.  The write (~0.15 ms) also gives the host time to
+    enqueue the call before the GPU reaches the first event."""
+
+    def __init__(self, torch, device):
+        self.torch = torch
+        self.buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def time_calls(self, fn, reps):
+        torch = self.torch
+        s = torch.cuda.current_stream()
+        evs = []
+        for _ in range(reps):
+            self.buf.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            fn(s)
+            e1.record(s)
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+
+def roofline_entries(cyc, flusher, peak, traffic, reps):
+    """One entry per call kind: median launch time with L2 flushed before every call, its
+    algorithmic bytes and the fraction of the HBM peak."""
+    per_kind = {}
+    for kind, step, fn in cyc.calls:
+        ms = flusher.time_calls(lambda s: fn(s, 0), reps)
+        per_kind.setdefault(kind, []).append((step, ms))
+    out = []
+    for kind, runs in per_kind.items():
+        times = [t for _, ms in runs for t in ms]
+        med = statistics.median(times)
+        byt = [cyc.call_bytes(kind, step) for step, _ in runs]
+        b = int(round(statistics.mean(byt)))
+        gbs = b / (med / 1e3) / 1e9
+        out.append({
+            "call": kind, "kernels": KERNELS[kind], "launches_per_step": len(runs),
+            "bytes_per_launch": b, "credited": kind != "stage",
+            "launch_us": round(med * 1e3, 2),
+            "launch_us_p10_p90": [round(float(np.percentile(times, 10)) * 1e3, 2),
+                                  round(float(np.percentile(times, 90)) * 1e3, 2)],
+            "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+            "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4),
+            "traffic": traffic.get(kind)})
+    return out
+
+
+def plain_decoding(cyc, torch, reps):
+    """Cycle of each drafting method against plain decoding, both replayed as CUDA graphs.
+
+    Plain decoding spends one dense single-row attention over the whole cache per token.  A
+    cycle yields n + 1 tokens (n accepted drafts plus the target's own next token); the
+    attention-path speed-up at acceptance n is (n + 1) * t_token / t_cycle.  Only the
+    attention and acceptance calls are timed: the models' other layers are outside this path."""
+    sp = cyc.spec
+    g = cyc.g
+    res = {"decode_steps": g}
+    dec = cyc.decode_step_calls()
+    gd = capture(torch, lambda s: [f(s) for f in dec])
+    t_dec = time_graph(torch, gd, reps) / g
+    w = cyc.w
+    row = w.h_kv * w.d * 2 * (2 if w.dtype == "bf16" else 4)
+    tok_bytes = statistics.mean(int(w.kv_len_draft(t).astype(np.int64).sum()) * row
+                                for t in range(g))
+    res["plain_ms_per_token"] = round(t_dec, 4)
+    res["plain_kv_bytes_per_token"] = int(tok_bytes)
+    res["plain_gbs"] = round(tok_bytes / (t_dec / 1e3) / 1e9, 1)
+    methods = {}
+    if sp["sparse"]:
+        methods["sparse_to_dense"] = ("topk", "stage", "sparse", "sparse_direct", "verify",
+                                      "accept_greedy")
+    if sp["ta"] and sp["hsr"]:
+        methods["sparrow"] = ("hsr", "text_anchored", "verify", "accept_greedy")
+    for name, kinds in methods.items():
+        gc = capture(torch, lambda s, kinds=kinds: cyc.step(s, 0, kinds))
+        t_cyc = time_graph(torch, gc, reps)
+        byt = sum(cyc.call_bytes(k, st) for k, st, _ in cyc.calls if k in kinds and k != "stage")
+        methods[name] = {
+            "calls": [k for k in kinds if any(c[0] == k for c in cyc.calls)],
+            "ms_per_cycle": round(t_cyc, 4), "bytes_per_cycle": int(byt),
+            "kv_bytes_per_token_at_n": {str(n): int(byt / (n + 1)) for n in range(g + 1)},
+            "speedup_at_n": {str(n): round((n + 1) * t_dec / t_cyc, 3) for n in range(g + 1)},
+            "break_even_n": next((n for n in range(g + 1) if (n + 1) * t_dec >= t_cyc), None)}
+        del gc
+    res["methods"] = methods
+    return res
+
+
+class HostIO:
+    """Per-step inputs in pinned host memory and the end-to-end loop: the next step's inputs
+    are copied on a second stream while the current step computes (two device input sets);
+    the new K/V rows go into the cache at the start of each step; the accepted counts and
+    tokens come back at its end."""
 
     def __init__(self, cyc):
         torch = cyc.torch
+        sets = []
+        for b in range(2):
+            d = [cyc.q_verify[b].q] + [q.q for q in cyc.q_draft[b]]
+            if cyc.spec["hsr"]:
+                d += list(cyc.emb[b])
+            if cyc.aw is not None:
+                d += [cyc.acc_in[b][k] for k in ("tgt", "drf", "tok_s", "tok_g", "u", "v")]
+            sets.append(d)
+        self.dev_sets = sets
+        # one pinned host copy serves both device sets (the inputs are the same every step)
+        self.host = [t.cpu().pin_memory() for t in sets[0]]
         w = cyc.w
-        pin = lambda t: t.cpu().pin_memory()
-        self.q_verify = pin(cyc.q_verify.q)
-        self.q_draft = [pin(q.q) for q in cyc.q_draft]
-        n_new = int(w.n_q_verify[0])
-        ctx = int(w.ctx_len[0])
-        self.ctx, self.n_new = ctx, n_new
-        self.k_new = pin(cyc.k[:, :, ctx:ctx + n_new].contiguous())
-        self.v_new = pin(cyc.v[:, :, ctx:ctx + n_new].contiguous())
-        self.emb = [pin(e) for e in cyc.emb]
-        self.tgt, self.drf = pin(cyc.tgt), pin(cyc.drf)
-        self.tok_s, self.tok_g = pin(cyc.tok_s), pin(cyc.tok_g)
-        self.u, self.v = pin(cyc.u), pin(cyc.vv)
-        self.res = [torch.empty(t.shape, dtype=t.dtype).pin_memory()
-                    for t in (cyc.n_acc_g, cyc.out_g, cyc.n_acc_s, cyc.out_s)]
-        tensors = [self.q_verify, *self.q_draft, self.k_new, self.v_new, *self.emb, self.tgt,
-                   self.drf, self.tok_s, self.tok_g, self.u, self.v]
-        self.h2d_bytes = sum(t.numel() * t.element_size() for t in tensors)
+        self.kv_rows = None
+        if not w.paged:
+            n_new = int(w.n_q_verify[0])
+            ctx = int(w.ctx_len[0])
+            assert (w.ctx_len == ctx).all() and (w.n_q_verify == n_new).all()
+            self.kv_rows = (ctx, n_new,
+                            cyc.k[:, :, ctx:ctx + n_new].contiguous().cpu().pin_memory(),
+                            cyc.v[:, :, ctx:ctx + n_new].contiguous().cpu().pin_memory())
+        if cyc.aw is not None:
+            self.outs = [cyc.n_acc_g, cyc.out_g, cyc.n_acc_s, cyc.out_s, cyc.near]
+        else:
+            self.outs = [cyc.o_verify]
+        self.res = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
+        kvb = 0 if self.kv_rows is None else sum(t.numel() * t.element_size()
+                                                 for t in self.kv_rows[2:])
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.host) + kvb
         self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.res)
 
-    def upload(self, cyc):
-        nb = True
-        cyc.q_verify.q.copy_(self.q_verify, non_blocking=nb)
-        for dq, hq in zip(cyc.q_draft, self.q_draft):
-            dq.q.copy_(hq, non_blocking=nb)
-        cyc.k[:, :, self.ctx:self.ctx + self.n_new].copy_(self.k_new, non_blocking=nb)
-        cyc.v[:, :, self.ctx:self.ctx + self.n_new].copy_(self.v_new, non_blocking=nb)
-        for de, he in zip(cyc.emb, self.emb):
-            de.copy_(he, non_blocking=nb)
-        for dst, src in ((cyc.tgt, self.tgt), (cyc.drf, self.drf), (cyc.tok_s, self.tok_s),
-                         (cyc.tok_g, self.tok_g), (cyc.u, self.u), (cyc.vv, self.v)):
-            dst.copy_(src, non_blocking=nb)
+    def upload(self, b):
+        """Copies on the current stream."""
+        for h, d in zip(self.host, self.dev_sets[b]):
+            d.copy_(h, non_blocking=True)
 
-    def download(self, cyc):
-        for dst, src in zip(self.res, (cyc.n_acc_g, cyc.out_g, cyc.n_acc_s, cyc.out_s)):
+    def kv_rows_in(self, cyc, stream):
+        """The new K/V rows of every (layer, KV head) into the cache: one strided copy each
+        for K and V from pinned memory (copy engine, no kernel)."""
+        if self.kv_rows is None:
+            return
+        from cuda.bindings import runtime as rt
+        ctx, n, hk, hv = self.kv_rows
+        d = cyc.w.d
+        esz = 2 if cyc.w.dtype == "bf16" else 4
+        cap = cyc.k.shape[2]
+        for dst, src in ((cyc.k, hk), (cyc.v, hv)):
+            err, = rt.cudaMemcpy2DAsync(dst.data_ptr() + ctx * d * esz, cap * d * esz,
+                                        src.data_ptr(), n * d * esz, n * d * esz,
+                                        dst.shape[0] * dst.shape[1],
+                                        rt.cudaMemcpyKind.cudaMemcpyHostToDevice,
+                                        stream.cuda_stream)
+            if err != rt.cudaError_t.cudaSuccess:
+                raise RuntimeError(f"cudaMemcpy2DAsync: {err}")
+
+    def download(self):
+        for dst, src in zip(self.res, self.outs):
             dst.copy_(src, non_blocking=True)
+
+    def run(self, cyc, steps):
+        """Returns the device time of `steps` end-to-end steps (ms)."""
+        torch = cyc.torch
+        comp = torch.cuda.current_stream()
+        copy = torch.cuda.Stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        done = [torch.cuda.Event() for _ in range(steps)]
+        up = [torch.cuda.Event() for _ in range(steps)]
+        e0.record(comp)
+        copy.wait_event(e0)
+        with torch.cuda.stream(copy):
+            self.upload(0)
+            up[0].record(copy)
+        for k in range(steps):
+            b = k % 2
+            if k + 1 < steps:  # next step's inputs, once the step that last used them is done
+                with torch.cuda.stream(copy):
+                    if k >= 1:
+                        copy.wait_event(done[k - 1])
+                    self.upload((k + 1) % 2)
+                    up[k + 1].record(copy)
+            comp.wait_event(up[k])
+            self.kv_rows_in(cyc, comp)
+            cyc.step(comp, b)
+            self.download()
+            done[k].record(comp)
+        e1.record(comp)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
 
 
 def reduce_max(x: float, world: int, device=None) -> float:
@@ -368,6 +662,32 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def workload_config(cyc):
+    w = cyc.w
+    sp = cyc.spec
+    calls = ["topk" if sp["topk"] else None, "stage" if sp["sparse"] == "staged" else None,
+             f"{cyc.g} x draft step [" + ", ".join(x for x in (
+                 "sparse" if sp["sparse"] else None, "hsr" if sp["hsr"] else None,
+                 "text_anchored" if sp["ta"] else None) if x) + "]",
+             "verify", "accept_greedy + accept_sample" if sp["accept"] else None]
+    lv = (int(w.l_vis.min()), int(w.l_vis.max()))
+    lt = (int(w.l_txt.min()), int(w.l_txt.max()))
+    desc = (f"{w.name}: {w.n_seq} {'layers' if w.n_seq > 1 and not w.paged else 'sequences'}"
+            f", H_q={w.h_q}, H_kv={w.h_kv}, d={w.d}, {w.dtype}, L_vis="
+            f"{lv[0] if lv[0] == lv[1] else lv}, L_txt={lt[0] if lt[0] == lt[1] else lt}, "
+            f"gamma={int(w.gamma_max)}" + (", paged (16)" if w.paged else "") +
+            (f", top-K {w.topk}" if sp["topk"] else "") +
+            (f", window {int(w.window.max())}" if sp["ta"] else "") +
+            (f", vocab {cyc.aw.vocab}" if cyc.aw is not None else ""))
+    return dict(workload=desc, config_index=cyc.cfg, calls=[c for c in calls if c],
+                layers_or_sequences=w.n_seq, l_vis=lv, l_txt=lt, gamma=int(w.gamma_max),
+                h_q=w.h_q, h_kv=w.h_kv, head_dim=w.d, kv_dtype=w.dtype,
+                topk=w.topk if sp["topk"] else None,
+                hsr_weight_copies=len(cyc.W) if sp["hsr"] else 0,
+                vocab=cyc.aw.vocab if cyc.aw is not None else None,
+                parallelism="replicas (no data-path collective)")
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -376,8 +696,7 @@ def run_ours(args):
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
     device = torch.device("cuda", torch.cuda.current_device())
-    cyc = Cycle(device)
-    stream = torch.cuda.current_stream()
+    cyc = Cycle(args.config, device)
 
     def barrier():
         if world > 1:
@@ -386,186 +705,235 @@ def run_ours(args):
 
     max_over_ranks = lambda x: reduce_max(x, world, device)
 
-    # ---- device-resident timing (optionally replayed from a CUDA graph) ----
-    graph = None
-    if args.graph:
-        for _ in range(2):
-            cyc.step()
-        torch.cuda.synchronize()
-        s = torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            cyc.step(stream=s)
-        torch.cuda.current_stream().wait_stream(s)
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=s):
-            cyc.step(stream=s)
-        torch.cuda.synchronize()
-    run = (lambda: graph.replay()) if graph is not None else (lambda: cyc.step())
+    # ---- device-resident timing of the whole step, replayed from a CUDA graph ----
+    graph = capture(torch, lambda s: cyc.step(s, 0))
     for _ in range(args.warmup):
-        run()
+        graph.replay()
     barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         ev0.record()
         for _ in range(args.steps):
-            run()
+            graph.replay()
         ev1.record()
         barrier()
-    ms = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms)
+    ms = max_over_ranks(ev0.elapsed_time(ev1))
     ms_per_step = ms / args.steps
     bytes_step = sum(cyc.bytes.values())
     value = whole_job_value(bytes_step, args.steps, ms, world)
+    n_kernels = cyc.count_graph_kernels(graph)
 
-    # ---- dominant kernel: verify, timed live with events on the launching stream ----
-    cyc.verify_events = []
-    for _ in range(args.steps):
-        cyc.step(time_verify=True)
-    barrier()
-    vt = [a.elapsed_time(b) for a, b in cyc.verify_events]
-    verify_ms = statistics.mean(vt)
-    verify_ms = max_over_ranks(verify_ms)
+    # ---- per call kind, L2 flushed before every call ----
     peak, peak_kind = peak_hbm()
-    achieved = cyc.bytes["verify"] / (verify_ms / 1e3) / 1e9
     traffic = recorded_traffic()
+    flusher = Flusher(torch, device)
+    rooflines = roofline_entries(cyc, flusher, peak, traffic, reps=args.call_reps)
+    for r in rooflines:
+        r["launch_us"] = round(max_over_ranks(r["launch_us"]), 2)
+    dom = max((r for r in rooflines if r["credited"]),
+              key=lambda r: r["launch_us"] * r["launches_per_step"])
+    roofline = {"bound": "hbm", "kernel": f"{dom['call']}: {dom['kernels']}",
+                "achieved": dom["achieved_gbs"], "peak": peak, "unit": "GB/s",
+                "frac": dom["frac"], "peak_source": f"{peak_kind} hbm_gbs",
+                "frac_of_8TBps": dom["frac_of_8TBps"], "bytes_per_launch": dom["bytes_per_launch"],
+                "launch_ms": round(dom["launch_us"] / 1e3, 4), "traffic": dom["traffic"],
+                "timing": "CUDA events on the launching stream, L2 flushed before each launch"}
+    layer_latency = []
+    for kind in ("verify", "sparse", "text_anchored"):
+        fn = cyc.one_layer(kind)
+        if fn is None:
+            continue
+        ms1 = statistics.median(flusher.time_calls(fn, args.call_reps))
+        b1 = cyc.call_bytes(kind, 0) // cyc.w.n_seq  # the layers are alike
+        layer_latency.append({"call": kind, "layers": 1, "launch_us": round(ms1 * 1e3, 2),
+                              "bytes": b1, "achieved_gbs": round(b1 / (ms1 / 1e3) / 1e9, 1),
+                              "frac": round(b1 / (ms1 / 1e3) / 1e9 / peak, 4)})
+    del flusher
+    torch.cuda.empty_cache()
+
+    # ---- each drafting method's cycle against plain decoding (CUDA graphs) ----
+    plain = plain_decoding(cyc, torch, reps=max(5, args.steps // 2)) if not args.no_plain \
+        else None
 
     # ---- end to end through the public API, host buffers, copies inside the timed region ----
-    host = HostInputs(cyc)
-    for _ in range(2):
-        host.upload(cyc)
-        cyc.step()
-        host.download(cyc)
+    host = HostIO(cyc)
+    host.run(cyc, 2)
     barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        host.upload(cyc)
-        cyc.step()
-        host.download(cyc)
-    e1.record()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_ms = max_over_ranks(host.run(cyc, args.steps))
     e2e_value = whole_job_value(bytes_step, args.steps, e2e_ms, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        probe = cpu_baseline(cyc.w, layers=1)
-        layers = int(max(1, min(cyc.w.n_seq, args.cpu_seconds / max(probe["seconds"], 1e-3))))
-        cpu = cpu_baseline(cyc.w, layers=layers)
+        cpu = cpu_baseline_report(cyc, args.cpu_seconds)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if cyc.w.dtype == "bf16" else "f32",
             "data": "synthetic (seeded; stands in for the pages' long-video benchmarks)",
-            "config": dict(WORKLOAD, graph=bool(graph is not None),
-                           bytes_per_step=bytes_step,
-                           bytes_per_call_kind=cyc.bytes),
-            "roofline": {"bound": "hbm", "kernel": "sd_verify_attention (28 layers, one call)",
-                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-                         "frac_of_8TBps": round(achieved / 8000.0, 4),
-                         "bytes_per_launch": cyc.bytes["verify"],
-                         "launch_ms": round(verify_ms, 4), "traffic": traffic},
+            "config": dict(workload_config(cyc), graph=True, bytes_per_step=bytes_step,
+                           bytes_per_call_kind=cyc.bytes,
+                           l2=("the step reads more than the 126 MB L2 (no flush between "
+                               "steps); per-call rooflines flush L2 before every call")),
+            "roofline": roofline,
+            "rooflines": rooflines,
+            "layer_latency": layer_latency,
+            "plain_decoding": plain,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": host.h2d_bytes, "d2h_bytes_per_step": host.d2h_bytes,
-                    "ms_per_step": round(e2e_ms / args.steps, 4)},
-            "gpu_launches": cyc.launches_per_step(graph) * args.steps,
+                    "ms_per_step": round(e2e_ms / args.steps, 4),
+                    "path": ("eager C-ABI calls through the Python binding; the next step's "
+                             "inputs copied on a second stream during the current step")},
+            "gpu_launches": (n_kernels if n_kernels is not None else -1) * args.steps,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+    del graph
     if world > 1:
-        del graph
         dist.destroy_process_group()
 
 
 # ---------------------------------------------------------------- oracle on the host -------
 
-def cpu_baseline(w, layers=1):
-    """Time the fp64 oracle on a bounded sample of the same workload: one whole cycle (top-K,
-    every draft step's sparse attention, HSR projection and text-anchored attention, verify,
-    greedy and sampling acceptance) restricted to the first `layers` layers of the attention
-    calls; report GB/s of algorithmic bytes."""
+def cpu_cycle(w, spec, g, layers, hsr_d, aw, topk):
+    """Run the fp64 oracle over one cycle of the workload restricted to its first `layers`
+    sequences (the acceptance and HSR calls in full); returns (seconds, algorithmic bytes)."""
     import oracle
-    threads = oracle.set_threads(0)
-    g = int(w.gamma[0])
-    n_q = int(w.n_q_verify[0])
-    sub = lambda lens: oracle.Cache(w.dtype, w.k[:layers], w.v[:layers], lens[:layers], w.h_kv, w.d)
-    full = cycle_bytes(w, [w.kv_len_draft(t) for t in range(g)], w.topk)
-    L = w.n_seq
     from speculative_decoding_attention_verify_b200 import inputs as gen
-    hw = gen.make_hsr_workload(n=1)
-    aw = gen.make_accept_workload(2, gammas=[g], batch=1)
+    sub = lambda lens: oracle.Cache(w.dtype, w.k[:layers], w.v[:layers], lens[:layers], w.h_kv,
+                                    w.d) if not w.paged else oracle.cache_from_workload(w, lens)
+    if w.paged:
+        layers = w.n_seq
+    nq = w.n_q_verify
+    qs = np.concatenate([[0], np.cumsum(nq[:layers])]).astype(np.int32)
+    hw = gen.make_hsr_workload(n=1) if spec["hsr"] else None
+    frac = layers / w.n_seq
+    byt = 0
     t0 = time.perf_counter()
-    idx, _ = oracle.topk_select(w.h_q, w.q_verify[:layers * n_q], w.q_verify_start[:layers + 1],
-                                sub(w.kv_len_verify), np.zeros(layers, np.int32),
-                                w.l_vis[:layers], w.topk)
+    idx = None
+    if spec["topk"]:
+        idx, _ = oracle.topk_select(w.h_q, w.q_verify[:qs[-1]], qs, sub(w.kv_len_verify),
+                                    np.zeros(layers, np.int32), w.l_vis[:layers], topk)
+        byt += call_bytes(w, "topk", topk=topk) * frac
     for t in range(g):
         lens = w.kv_len_draft(t)
-        oracle.sparse_attention(w.h_q, w.q_draft[t][:layers], np.arange(layers + 1), sub(lens),
-                                idx, w.l_vis[:layers])
-        oracle.hsr_project(hw.emb, hw.hid, hw.weight)
-        oracle.text_anchored_attention(w.h_q, w.q_draft[t][:layers], np.arange(layers + 1),
-                                       sub(lens), np.zeros(layers, np.int32), w.l_vis[:layers],
-                                       w.window[:layers])
-    oracle.verify_attention(w.h_q, w.q_verify[:layers * n_q], w.q_verify_start[:layers + 1],
-                            sub(w.kv_len_verify))
-    oracle.accept_greedy(aw.target_logits, aw.draft_tokens_greedy, aw.gamma, aw.vocab)
-    oracle.accept_sample(aw.target_logits, aw.draft_logits, aw.draft_tokens_sampled, aw.u, aw.v,
-                         aw.gamma, aw.vocab)
-    t_total = time.perf_counter() - t0
-    per_layer = full["topk"] + full["verify"] + full["sparse"] + full["text_anchored"]
-    bytes_total = per_layer * layers // L + full["hsr"] + full["accept_greedy"] + \
-        full["accept_sample"]
-    return {"value": round(bytes_total / t_total / 1e9, 4), "unit": "GB/s", "cores": threads,
-            "kind": "oracle", "seconds": round(t_total, 3),
-            "sample": f"one whole cycle on {layers} of {L} layers: top-K, {g} x (sparse draft "
-                      f"step, HSR projection, text-anchored draft step), verify, greedy + "
-                      f"sampling acceptance ({t_total:.1f} s on {threads} threads)"}
+        if spec["sparse"]:
+            oracle.sparse_attention(w.h_q, w.q_draft[t][:layers], np.arange(layers + 1),
+                                    sub(lens), idx, w.l_vis[:layers])
+            byt += call_bytes(w, "sparse", t, topk=topk) * frac
+        if spec["hsr"]:
+            oracle.hsr_project(hw.emb, hw.hid, hw.weight)
+            byt += call_bytes(w, "hsr", hsr_d=hsr_d)
+        if spec["ta"]:
+            oracle.text_anchored_attention(w.h_q, w.q_draft[t][:layers], np.arange(layers + 1),
+                                           sub(lens), np.zeros(layers, np.int32),
+                                           w.l_vis[:layers], w.window[:layers])
+            byt += call_bytes(w, "text_anchored", t) * frac
+    oracle.verify_attention(w.h_q, w.q_verify[:qs[-1]], qs, sub(w.kv_len_verify))
+    byt += call_bytes(w, "verify") * frac
+    if spec["accept"]:
+        oracle.accept_greedy(aw.target_logits, aw.draft_tokens_greedy, aw.gamma, aw.vocab)
+        oracle.accept_sample(aw.target_logits, aw.draft_logits, aw.draft_tokens_sampled, aw.u,
+                             aw.v, aw.gamma, aw.vocab)
+        byt += call_bytes(w, "accept_greedy", aw=aw) + call_bytes(w, "accept_sample", aw=aw)
+    return time.perf_counter() - t0, byt
+
+
+def cpu_baseline_at(w, spec, g, hsr_d, aw, topk, threads, seconds):
+    """The oracle on `threads` host threads (0: all), on as many layers of one cycle as fit in
+    about `seconds`."""
+    import oracle
+    used = oracle.set_threads(threads if threads > 0 else os.cpu_count() or 1)
+    t1, _ = cpu_cycle(w, spec, g, 1, hsr_d, aw, topk)
+    layers = int(max(1, min(w.n_seq, seconds / max(t1, 1e-3))))
+    t, byt = cpu_cycle(w, spec, g, layers, hsr_d, aw, topk)
+    return {"value": round(byt / t / 1e9, 4), "unit": "GB/s", "cores": used, "kind": "oracle",
+            "seconds": round(t, 3),
+            "sample": f"one whole cycle on {layers} of {w.n_seq} "
+                      f"{'layers' if w.n_seq > 1 and not w.paged else 'sequences'} "
+                      f"({t:.1f} s on {used} threads)"}
+
+
+def cpu_baseline_report(cyc, seconds):
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    args = (cyc.w, cyc.spec, cyc.g, cyc.hsr_d, cyc.aw, cyc.topk)
+    multi = cpu_baseline_at(*args, threads=cores, seconds=seconds)
+    single = cpu_baseline_at(*args, threads=1, seconds=seconds / 2)
+    oracle.set_threads(cores)
+    multi["single_thread"] = {k: single[k] for k in ("value", "unit", "cores", "seconds", "sample")}
+    multi["cpu_model"] = cpu_model()
+    return multi
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def run_reference(args):
+    """The reference arm: the fp64 oracle (the pages hold no code to install), timed on the
+    host's cores on bounded samples of the same workload."""
     rank, world, _ = env_rank()
     if rank != 0:
         return
     from speculative_decoding_attention_verify_b200 import inputs as gen
-    w = gen.make_attn_workload(CFG_INDEX)
-    for _ in range(args.warmup):
-        pass  # the oracle has no warm-up state; warm-up steps are skipped deliberately
+    import oracle
+    cfg = args.config
+    spec = SPECS[cfg]
+    w = gen.make_attn_workload(cfg)
+    g = int(spec["draft_steps"] or w.gamma_max)
+    aw = None
+    if spec["accept"]:
+        aw = gen.make_accept_workload(2, gammas=[g], batch=1) if cfg in (2, 3) else \
+            gen.make_accept_workload(cfg, gammas=w.gamma)
+    hsr_d = gen.HSR_D_MODEL if spec["hsr"] else None
+    cores = len(os.sched_getaffinity(0))
+    used = oracle.set_threads(cores)
     vals = []
     t0 = time.perf_counter()
     cpu = None
     for _ in range(args.steps):
-        cpu = cpu_baseline(w, layers=1)
-        vals.append(cpu["value"])
+        t, byt = cpu_cycle(w, spec, g, 1, hsr_d, aw, w.topk)
+        vals.append(byt / t / 1e9)
     elapsed = time.perf_counter() - t0
     value = statistics.mean(vals)
+    cpu = {"value": round(value, 4), "unit": "GB/s", "cores": used, "kind": "oracle",
+           "sample": f"one whole cycle on 1 of {w.n_seq} layers/sequences per step "
+                     f"({elapsed / max(args.steps, 1):.1f} s per step on {used} threads)"}
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * elapsed / max(args.steps, 1), 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded)", "config": WORKLOAD,
-            "cpu_baseline": dict(cpu, value=round(value, 4)),
+            "data": "synthetic (seeded)", "config": {"workload": w.name, "config_index": cfg},
+            "cpu_baseline": cpu,
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-CASES = ("verify", "sparse", "text_anchored", "topk", "hsr", "accept_greedy", "accept_sample")
+CASES = ("verify", "sparse", "sparse_staged", "stage", "text_anchored", "topk", "hsr",
+         "accept_greedy", "accept_sample", "decode")
 
 
 def run_case(args):
-    """One call kind of the cycle on a reduced workload (``--layers``), repeated ``--steps``
-    times after ``--warmup``; prints its device time.  Used for ncu captures of one kernel."""
+    """One call kind of the default workload on a reduced layer count (``--layers``), repeated
+    ``--steps`` times after ``--warmup``; prints its device time.  Used for ncu captures of one
+    kernel on a small case."""
     import torch
     from speculative_decoding_attention_verify_b200 import device as dev
     from speculative_decoding_attention_verify_b200 import inputs as gen
     from speculative_decoding_attention_verify_b200 import sdattn as sd
-    w = gen.make_attn_workload(CFG_INDEX, layers=args.layers)
+    w = gen.make_attn_workload(DEFAULT_CONFIG, layers=args.layers)
     L, g = w.n_seq, int(w.gamma[0])
     k = dev.tensor(w.k, w.dtype)
     v = dev.tensor(w.v, w.dtype)
@@ -574,16 +942,26 @@ def run_case(args):
     kv_draft = dev.kv_cache(w, kv_len=lens, k=k, v=v)
     qv, qd = dev.verify_queries(w), dev.draft_queries(w, 0)
     i32 = dev.int32
+    tail = i32(w.l_vis)
+    max_tail = int((lens - w.l_vis).max())
     if args.case == "verify":
         call = lambda: sd.sd_verify_attention(qv, kv_verify)
+    elif args.case == "decode":
+        call = lambda: sd.sd_verify_attention(qd, kv_draft)
     elif args.case == "topk":
         call = lambda: sd.sd_topk_select(qv, kv_verify, i32(np.zeros(L)), i32(w.l_vis),
                                          int(w.l_vis.max()), w.topk)
-    elif args.case == "sparse":
+    elif args.case in ("sparse", "sparse_staged", "stage"):
         idx = sd.sd_topk_select(qv, kv_verify, i32(np.zeros(L)), i32(w.l_vis),
                                 int(w.l_vis.max()), w.topk)
-        tail = i32(w.l_vis)
-        call = lambda: sd.sd_sparse_attention(qd, kv_draft, idx, tail, int((lens - w.l_vis).max()))
+        sel = sd.sd_sparse_stage(kv_draft, idx, tail)
+        if args.case == "sparse":
+            call = lambda: sd.sd_sparse_attention(qd, kv_draft, idx, tail, max_tail)
+        elif args.case == "stage":
+            call = lambda: sd.sd_sparse_stage(kv_draft, idx, tail, selection=sel)
+        else:
+            call = lambda: sd.sd_sparse_attention_staged(qd, kv_draft, sel, w.topk, tail,
+                                                         max_tail)
     elif args.case == "text_anchored":
         vb, ve, win = i32(np.zeros(L)), i32(w.l_vis), i32(w.window)
         call = lambda: sd.sd_text_anchored_attention(qd, kv_draft, vb, ve, win, int(w.window.max()))
@@ -619,9 +997,13 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--no-graph", dest="graph", action="store_false")
+    ap.add_argument("--config", type=int, choices=sorted(SPECS), default=DEFAULT_CONFIG,
+                    help="workload (default: the 28-layer 25k-visual-token Sparse-to-Dense case)")
+    ap.add_argument("--call-reps", type=int, default=10,
+                    help="separately timed repetitions of every call for the per-call rooflines")
+    ap.add_argument("--no-plain", action="store_true", help="skip the plain-decoding comparison")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--case", choices=CASES, default=None,
                     help="time one call kind on a reduced workload (for ncu captures)")
     ap.add_argument("--layers", type=int, default=4)

@@ -323,7 +323,7 @@ SD_API sd_status sd_accept_sample(const float *tgt_logits, const float *draft_lo
  * race; calls on one stream are safe.  Errors: as sd_verify_attention; SD_ERR_UNSUPPORTED if
  * the current device ordinal is 64 or more; SD_ERR_CUDA if the address lookup fails.
  */
-#define SD_VERIFY_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+#define SD_VERIFY_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 
 SD_API sd_status sd_verify_attention_noalloc(const sd_q_desc *q, const void *q_data,
                                       const sd_kv_desc *kv, int32_t batch, void *out,

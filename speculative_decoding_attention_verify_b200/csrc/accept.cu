@@ -247,12 +247,16 @@ __global__ void accept_decide_kernel(const AcceptParams p) {
     }
 }
 
-__device__ __forceinline__ double draw_weight(const float *zp, const float *zq, float lp, float lq,
-                                              bool residual, int x) {
-    const float pp = expf(__ldg(zp + x) - lp);
-    if (!residual) return (double)pp;
-    const float d = pp - expf(__ldg(zq + x) - lq);
-    return d > 0.f ? (double)d : 0.0;
+// Draw weight of token x: p_x, or max(0, p_x - q_x) in residual mode.  Evaluated in fp64 from
+// the fp64 log-sum-exps: in residual mode p and q nearly cancel, so rounding either exponent to
+// fp32 (about 1e-7 relative at |z - lse| ~ 16) could move a prefix sum across a token boundary
+// by more than the 1e-6 * Z window that is counted as near-boundary.
+__device__ __forceinline__ double draw_weight(const float *zp, const float *zq, double lp,
+                                              double lq, bool residual, int x) {
+    const double pp = exp((double)__ldg(zp + x) - lp);
+    if (!residual) return pp;
+    const double d = pp - exp((double)__ldg(zq + x) - lq);
+    return d > 0.0 ? d : 0.0;
 }
 
 __device__ double block_sum_d(double x, double *s_red) {
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(kThreads) accept_wsum_kernel(const AcceptParam
     chunk_range(p.vocab, p.n_chunks, c, lo, hi);
     double s = 0.0;
     for (int x = lo + threadIdx.x; x < hi; x += kThreads)
-        s += draw_weight(zp, zq, (float)dec.lse_p, (float)dec.lse_q, dec.residual != 0, x);
+        s += draw_weight(zp, zq, dec.lse_p, dec.lse_q, dec.residual != 0, x);
     s = block_sum_d(s, s_red);
     if (threadIdx.x == 0) chunk_sums(p)[(int64_t)b * p.n_chunks + c] = s;
 }
@@ -311,7 +315,7 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const AcceptParam
             chunk_range(p.vocab, p.n_chunks, c, lo, hi);
             double s = 0.0;
             for (int x = lo + tid; x < hi; x += kThreads)
-                s += draw_weight(zp, zq, (float)dec.lse_p, 0.f, false, x);
+                s += draw_weight(zp, zq, dec.lse_p, 0.0, false, x);
             Z += block_sum_d(s, s_red);
         }
     } else {
@@ -337,7 +341,7 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const AcceptParam
         chunk_range(p.vocab, p.n_chunks, c, lo, hi);
         for (int base = lo; base < hi; base += kThreads) {
             const int x = base + tid;
-            const double w = x < hi ? draw_weight(zp, zq, (float)dec.lse_p, (float)dec.lse_q,
+            const double w = x < hi ? draw_weight(zp, zq, dec.lse_p, dec.lse_q,
                                                   residual, x)
                                     : 0.0;
             // in-order inclusive prefix sum over the tile

@@ -29,9 +29,9 @@ AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, in
     plan.max_kv_len = (int)(max_stream < (1LL << 30) ? max_stream : (1LL << 30));
     plan.tensor_core = tc_supported(kind, dtype, head_dim, rows);
     // CUDA-core decomposition: 64-position tiles, a 3-stage K/V ring of 3*2*64 rows in
-    // shared memory; two CTAs fit per SM when the ring is at most 96 KB.  Choose the split
-    // count whose CTAs fill whole waves best, with at least two tiles per CTA and a penalty
-    // for the per-CTA set-up and the merge.
+    // shared memory; two CTAs fit per SM when the ring is at most 96 KB.  Modelled time of
+    // split count s: waves x (per-CTA set-up and merge share, about two tiles' worth, + tiles
+    // per CTA), with at least two tiles per CTA; the smallest wins.
     plan.rows_per_block = rows <= 8 ? 8 : 16;
     plan.n_rowblocks = (rows + plan.rows_per_block - 1) / plan.rows_per_block;
     {
@@ -40,15 +40,15 @@ AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, in
         const long long slots = (long long)sms * (ring <= 96 * 1024 ? 2 : 1);
         const long long units = (long long)batch * h_kv * plan.n_rowblocks;
         const long long tiles = (max_stream + 63) / 64;
-        double best = -1.0;
+        long long best = -1;
         plan.simt_splits = 1;
         for (long long s = 1; s <= 256; ++s) {
             if (s > 1 && tiles / s < 2) break;
             const long long ctas = units * s;
             const long long waves = (ctas + slots - 1) / slots;
-            const double score = (double)ctas / (double)(waves * slots) - 0.01 * (double)s;
-            if (score > best) {
-                best = score;
+            const long long t = waves * (2 + (tiles + s - 1) / s);
+            if (best < 0 || t < best) {
+                best = t;
                 plan.simt_splits = (int)s;
             }
         }

@@ -7,11 +7,12 @@
 // pointers given to it by another runtime and has no allocator of its own.  cudaMalloc may also
 // synchronise the device, which such callers cannot afford in a decode loop.
 //
-// The scratch is a file-scope device array of kScratchBytes (32 MiB: enough for a 28-layer
-// batch of 9 verify rows x 28 heads at d=128 and 26k cached positions).  A call whose plan
-// needs more is rejected with SD_ERR_WORKSPACE before anything is launched.  Nothing in the
-// scratch has to start at zero: every split writes the partial output and (max, sum) of every
-// row before the merge kernel reads them.
+// The scratch is a file-scope device array of kScratchBytes (64 MiB: enough for a 28-layer
+// batch of 9 verify rows x 28 heads at d=128 and 26k cached positions, whose plan needs 38.5 MiB
+// on 148 SMs, sized for either attention engine).  A call whose plan needs more is rejected
+// with SD_ERR_WORKSPACE before anything is launched.  Nothing in the scratch has to start at
+// zero: every split writes the partial output and (max, sum) of every row before the merge
+// kernel reads them.
 //
 // The scratch is shared by every call on a device: two calls that may overlap on the device
 // (different streams, or host threads, without ordering between them) race on it and give

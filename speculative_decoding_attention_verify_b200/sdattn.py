@@ -8,6 +8,7 @@ fallback: without the library, or without a GPU, calls raise.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -21,6 +22,7 @@ SD_OK, SD_ERR_INVALID_ARG, SD_ERR_UNSUPPORTED, SD_ERR_WORKSPACE, SD_ERR_CUDA = r
 SD_F32, SD_BF16 = 0, 1
 SD_ATTN_VERIFY, SD_ATTN_TEXT_ANCHORED, SD_ATTN_SPARSE = 0, 1, 2
 SD_DEVERR_PAGE, SD_DEVERR_INDEX, SD_DEVERR_TOKEN, SD_DEVERR_NUMERIC, SD_DEVERR_SHAPE = 1, 2, 4, 8, 16
+SD_DEVERR_TIMEOUT = 32
 PAGE_SIZE = 16
 
 _LIB = None
@@ -55,7 +57,7 @@ EXPORTS = ("sd_status_string", "sd_version", "sd_attention_workspace_size", "sd_
            "sd_sparse_selection_size", "sd_sparse_stage", "sd_sparse_attention_staged")
 
 # Size of the library's fixed scratch used by sd_verify_attention_noalloc.
-SD_VERIFY_NOALLOC_SCRATCH_BYTES = 32 << 20
+SD_VERIFY_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 def lib():
@@ -109,6 +111,15 @@ def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on(t: torch.Tensor):
+    """Make the tensor's device current for the call (the library launches on the current
+    device, and sd_verify_attention_noalloc picks its per-device scratch from it)."""
+    if t.device.type == "cuda" and t.device.index is not None and \
+            t.device.index != torch.cuda.current_device():
+        return torch.cuda.device(t.device)
+    return contextlib.nullcontext()
 
 
 def _check(status: int, where: str):
@@ -208,9 +219,10 @@ def sd_verify_attention(q: Queries, kv: KVCache, out=None, workspace=None, dev_e
                         stream=None) -> torch.Tensor:
     out = _attn_out(q, out)
     ws = _workspace(sd_attention_workspace_size(SD_ATTN_VERIFY, q, kv), q.q.device, workspace)
-    _check(lib().sd_verify_attention(ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc),
-                                     kv.batch, _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
-                                     _stream(stream)), "sd_verify_attention")
+    with _on(q.q):
+        _check(lib().sd_verify_attention(ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc),
+                                         kv.batch, _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
+                                         _stream(stream)), "sd_verify_attention")
     return out
 
 
@@ -219,9 +231,11 @@ def sd_verify_attention_noalloc(q: Queries, kv: KVCache, out: torch.Tensor, dev_
     """sd_verify_attention on the library's fixed scratch: the C call allocates nothing, so the
     caller passes ``out``.  Raises SdError (SD_ERR_WORKSPACE) when the call's workspace exceeds
     SD_VERIFY_NOALLOC_SCRATCH_BYTES."""
-    _check(lib().sd_verify_attention_noalloc(ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc),
-                                             kv.batch, _ptr(out), _ptr(dev_err), _stream(stream)),
-           "sd_verify_attention_noalloc")
+    with _on(q.q):
+        _check(lib().sd_verify_attention_noalloc(ctypes.byref(q.desc), _ptr(q.q),
+                                                 ctypes.byref(kv.desc), kv.batch, _ptr(out),
+                                                 _ptr(dev_err), _stream(stream)),
+               "sd_verify_attention_noalloc")
     return out
 
 
@@ -230,10 +244,11 @@ def sd_text_anchored_attention(q: Queries, kv: KVCache, vis_begin, vis_end, wind
                                stream=None) -> torch.Tensor:
     out = _attn_out(q, out)
     ws = _workspace(sd_attention_workspace_size(SD_ATTN_TEXT_ANCHORED, q, kv), q.q.device, workspace)
-    _check(lib().sd_text_anchored_attention(
-        ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(vis_begin),
-        _ptr(vis_end), _ptr(window), int(max_window), _ptr(out), _ptr(ws), ws.numel(),
-        _ptr(dev_err), _stream(stream)), "sd_text_anchored_attention")
+    with _on(q.q):
+        _check(lib().sd_text_anchored_attention(
+            ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(vis_begin),
+            _ptr(vis_end), _ptr(window), int(max_window), _ptr(out), _ptr(ws), ws.numel(),
+            _ptr(dev_err), _stream(stream)), "sd_text_anchored_attention")
     return out
 
 
@@ -242,10 +257,11 @@ def sd_sparse_attention(q: Queries, kv: KVCache, idx: torch.Tensor, tail_begin, 
     out = _attn_out(q, out)
     ws = _workspace(sd_sparse_workspace_size(q, kv, int(idx.shape[-1]), max_tail), q.q.device,
                     workspace)
-    _check(lib().sd_sparse_attention(
-        ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(idx),
-        int(idx.shape[-1]), _ptr(tail_begin), int(max_tail), _ptr(out), _ptr(ws), ws.numel(),
-        _ptr(dev_err), _stream(stream)), "sd_sparse_attention")
+    with _on(q.q):
+        _check(lib().sd_sparse_attention(
+            ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(idx),
+            int(idx.shape[-1]), _ptr(tail_begin), int(max_tail), _ptr(out), _ptr(ws), ws.numel(),
+            _ptr(dev_err), _stream(stream)), "sd_sparse_attention")
     return out
 
 
@@ -271,9 +287,10 @@ def sd_sparse_stage(kv: KVCache, idx: torch.Tensor, tail_begin, selection=None, 
     if selection is None:
         selection = torch.empty(max(sd_sparse_selection_size(kv, k), 16), dtype=torch.uint8,
                                 device=kv.k.device)
-    _check(lib().sd_sparse_stage(ctypes.byref(kv.desc), kv.batch, _ptr(idx), k, _ptr(tail_begin),
-                                 _ptr(selection), selection.numel(), _ptr(dev_err),
-                                 _stream(stream)), "sd_sparse_stage")
+    with _on(kv.k):
+        _check(lib().sd_sparse_stage(ctypes.byref(kv.desc), kv.batch, _ptr(idx), k,
+                                     _ptr(tail_begin), _ptr(selection), selection.numel(),
+                                     _ptr(dev_err), _stream(stream)), "sd_sparse_stage")
     return selection
 
 
@@ -282,10 +299,11 @@ def sd_sparse_attention_staged(q: Queries, kv: KVCache, selection: torch.Tensor,
                                stream=None) -> torch.Tensor:
     out = _attn_out(q, out)
     ws = _workspace(sd_sparse_workspace_size(q, kv, k, max_tail), q.q.device, workspace)
-    _check(lib().sd_sparse_attention_staged(
-        ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(selection),
-        int(k), _ptr(tail_begin), int(max_tail), _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
-        _stream(stream)), "sd_sparse_attention_staged")
+    with _on(q.q):
+        _check(lib().sd_sparse_attention_staged(
+            ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(selection),
+            int(k), _ptr(tail_begin), int(max_tail), _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
+            _stream(stream)), "sd_sparse_attention_staged")
     return out
 
 
@@ -301,10 +319,11 @@ def sd_topk_select(q: Queries, kv: KVCache, cand_begin, cand_end, max_cand: int,
     if idx_out is None:
         idx_out = torch.empty((kv.batch, kv.h_kv, int(k)), dtype=torch.int32, device=q.q.device)
     ws = _workspace(sd_topk_workspace_size(kv, max_cand, k), q.q.device, workspace)
-    _check(lib().sd_topk_select(
-        ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(cand_begin),
-        _ptr(cand_end), int(max_cand), int(k), _ptr(idx_out), _ptr(ws), ws.numel(), _ptr(dev_err),
-        _stream(stream)), "sd_topk_select")
+    with _on(q.q):
+        _check(lib().sd_topk_select(
+            ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(cand_begin),
+            _ptr(cand_end), int(max_cand), int(k), _ptr(idx_out), _ptr(ws), ws.numel(),
+            _ptr(dev_err), _stream(stream)), "sd_topk_select")
     return idx_out
 
 
@@ -313,8 +332,9 @@ def sd_hsr_project(emb: torch.Tensor, hid: torch.Tensor, weight: torch.Tensor, b
     n, dm = emb.shape
     if out is None:
         out = torch.empty((n, dm), dtype=torch.bfloat16, device=emb.device)
-    _check(lib().sd_hsr_project(_ptr(emb), _ptr(hid), n, dm, _ptr(weight), _ptr(bias), _ptr(out),
-                                _stream(stream)), "sd_hsr_project")
+    with _on(emb):
+        _check(lib().sd_hsr_project(_ptr(emb), _ptr(hid), n, dm, _ptr(weight), _ptr(bias),
+                                    _ptr(out), _stream(stream)), "sd_hsr_project")
     return out
 
 
@@ -333,10 +353,11 @@ def sd_accept_greedy(tgt_logits, draft_tok, gamma, max_gamma: int, n_acc=None, o
     if out_tok is None:
         out_tok = torch.full((batch, max_gamma + 1), -1, dtype=torch.int32, device=dev)
     ws = _workspace(sd_accept_workspace_size(batch, max_gamma, vocab), dev, workspace)
-    _check(lib().sd_accept_greedy(_ptr(tgt_logits), _ptr(draft_tok), _ptr(gamma), batch,
-                                  int(max_gamma), vocab, _ptr(n_acc), _ptr(out_tok),
-                                  out_tok.shape[1], _ptr(ws), ws.numel(), _ptr(dev_err),
-                                  _stream(stream)), "sd_accept_greedy")
+    with _on(tgt_logits):
+        _check(lib().sd_accept_greedy(_ptr(tgt_logits), _ptr(draft_tok), _ptr(gamma), batch,
+                                      int(max_gamma), vocab, _ptr(n_acc), _ptr(out_tok),
+                                      out_tok.shape[1], _ptr(ws), ws.numel(), _ptr(dev_err),
+                                      _stream(stream)), "sd_accept_greedy")
     return n_acc, out_tok
 
 
@@ -351,8 +372,10 @@ def sd_accept_sample(tgt_logits, draft_logits, draft_tok, u, v, gamma, max_gamma
     if near_boundary is None:
         near_boundary = torch.zeros(batch, dtype=torch.int32, device=dev)
     ws = _workspace(sd_accept_workspace_size(batch, max_gamma, vocab), dev, workspace)
-    _check(lib().sd_accept_sample(_ptr(tgt_logits), _ptr(draft_logits), _ptr(draft_tok), _ptr(u),
-                                  _ptr(v), _ptr(gamma), batch, int(max_gamma), vocab, _ptr(n_acc),
-                                  _ptr(out_tok), out_tok.shape[1], _ptr(near_boundary), _ptr(ws),
-                                  ws.numel(), _ptr(dev_err), _stream(stream)), "sd_accept_sample")
+    with _on(tgt_logits):
+        _check(lib().sd_accept_sample(_ptr(tgt_logits), _ptr(draft_logits), _ptr(draft_tok),
+                                      _ptr(u), _ptr(v), _ptr(gamma), batch, int(max_gamma), vocab,
+                                      _ptr(n_acc), _ptr(out_tok), out_tok.shape[1],
+                                      _ptr(near_boundary), _ptr(ws), ws.numel(), _ptr(dev_err),
+                                      _stream(stream)), "sd_accept_sample")
     return n_acc, out_tok, near_boundary

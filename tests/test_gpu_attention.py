@@ -297,3 +297,155 @@ def test_verify_short_chunks_repeated(l_vis, l_txt, batch):
             first = bits
         else:
             assert torch.equal(first, bits)
+
+
+# ---------------------------------------------------------------- CUDA-core engine ---------
+# The tensor-core kernel serves bf16 calls with at most 128 planned rows per KV head whose Q
+# and O are 16-byte aligned and whose cache the copy engine can describe; every other call runs
+# on the CUDA-core engine.  These cases reach that engine on purpose.
+
+
+def _unaligned_like(t):
+    """A contiguous copy of t whose data starts 2 bytes past a 16-byte boundary."""
+    flat = torch.empty(t.numel() + 8, dtype=t.dtype, device=t.device)
+    view = flat[1:1 + t.numel()].view(t.shape)
+    view.copy_(t)
+    assert view.data_ptr() % 16 != 0
+    return view
+
+
+@pytest.mark.parametrize("cfg,kw", [
+    (1, dict(l_vis=2000, l_txt=150, gamma=19)),               # 140 rows per KV head
+    (0, dict(dtype="bf16", l_vis=1500, l_txt=90, gamma=33)),  # d=64, 136 rows
+])
+def test_verify_cuda_core_engine_more_than_128_rows(cfg, kw):
+    w = gen.make_attn_workload(cfg, **kw)
+    assert w.group * int(w.n_q_verify.max()) > 128
+    out = sd.sd_verify_attention(dev.verify_queries(w), dev.kv_cache(w))
+    ref = oracle.verify_attention(w.h_q, w.q_verify, w.q_verify_start, oracle.cache_from_workload(w))
+    _assert_close(out, ref, w.dtype, f"verify >128 rows cfg{cfg}")
+
+
+@pytest.mark.parametrize("kind", ["verify", "text_anchored", "sparse"])
+def test_cuda_core_engine_unaligned_q_and_out_bf16(kind):
+    """Q and O that start off a 16-byte boundary cannot feed the tensor-core kernel."""
+    w = gen.make_attn_workload(1, l_vis=3000, l_txt=200, gamma=3)
+    q0 = dev.verify_queries(w)
+    q = sd.Queries(_unaligned_like(q0.q), q0.q_start, q0.desc.max_q_rows, q0.desc.max_kv_len)
+    out = _unaligned_like(torch.zeros_like(q0.q))
+    kv = dev.kv_cache(w)
+    cache = oracle.cache_from_workload(w)
+    if kind == "verify":
+        sd.sd_verify_attention(q, kv, out=out)
+        ref = oracle.verify_attention(w.h_q, w.q_verify, w.q_verify_start, cache)
+    elif kind == "text_anchored":
+        vb, ve, win = np.zeros(1, np.int32), w.l_vis.astype(np.int32), np.array([150], np.int32)
+        sd.sd_text_anchored_attention(q, kv, dev.int32(vb), dev.int32(ve), dev.int32(win), 150,
+                                      out=out)
+        ref = oracle.text_anchored_attention(w.h_q, w.q_verify, w.q_verify_start, cache, vb, ve,
+                                             win)
+    else:
+        idx, _ = oracle.topk_select(w.h_q, w.q_verify, w.q_verify_start, cache,
+                                    np.zeros(1, np.int32), w.l_vis, 300)
+        tail = w.l_vis.astype(np.int32)
+        sd.sd_sparse_attention(q, kv, dev.int32(idx), dev.int32(tail),
+                               int(w.kv_len_verify[0] - tail[0]), out=out)
+        ref = oracle.sparse_attention(w.h_q, w.q_verify, w.q_verify_start, cache, idx, tail)
+    _assert_close(out, ref, w.dtype, f"unaligned {kind}")
+
+
+@pytest.mark.parametrize("kw", [dict(gamma=5), dict(gamma=0, l_vis=3000, l_txt=100),
+                                dict(gamma=2, l_vis=700, l_txt=33, layers=3)])
+def test_verify_fp32_head_dim_128(kw):
+    """fp32 caches with the 7B-like head shapes (d=128, G=7): CUDA cores, 1e-4."""
+    w = gen.make_attn_workload(1, dtype="f32", **kw)
+    out = sd.sd_verify_attention(dev.verify_queries(w), dev.kv_cache(w))
+    ref = oracle.verify_attention(w.h_q, w.q_verify, w.q_verify_start, oracle.cache_from_workload(w))
+    _assert_close(out, ref, w.dtype, f"fp32 d=128 {kw}")
+
+
+def test_draft_calls_fp32_head_dim_128():
+    w = gen.make_attn_workload(1, dtype="f32", l_vis=2500, l_txt=300)
+    out, ref = _text_anchored_case(w, step=2, window=200)
+    _assert_close(out, ref, w.dtype, "fp32 text-anchored d=128")
+    lens = w.kv_len_draft(1)
+    idx = _oracle_topk(w, w.kv_len_verify, 256)
+    tail = w.l_vis.astype(np.int32)
+    out = sd.sd_sparse_attention(dev.draft_queries(w, 1), dev.kv_cache(w, kv_len=lens),
+                                 dev.int32(idx), dev.int32(tail), int((lens - tail).max()))
+    ref = oracle.sparse_attention(w.h_q, w.q_draft[1], np.arange(w.n_seq + 1),
+                                  oracle.cache_from_workload(w, kv_len=lens), idx, tail)
+    _assert_close(out, ref, w.dtype, "fp32 sparse d=128")
+
+
+# ---------------------------------------------------------------- full-size draft calls ----
+
+
+@pytest.fixture(scope="module")
+def c3_full():
+    """The 28-layer Sparse-to-Dense workload (25,000 visual + 1,024 text positions) on the GPU,
+    with the device's own top-K selection, as the benchmark cycle runs it."""
+    w = gen.make_attn_workload(3)
+    k, v = dev.tensor(w.k, w.dtype), dev.tensor(w.v, w.dtype)
+    kv_verify = dev.kv_cache(w, k=k, v=v)
+    L = w.n_seq
+    idx = sd.sd_topk_select(dev.verify_queries(w), kv_verify, dev.int32(np.zeros(L)),
+                            dev.int32(w.l_vis), int(w.l_vis.max()), w.topk).cpu().numpy()
+    return w, k, v, idx
+
+
+SAMPLED_LAYERS = (0, 13, 27)
+
+
+def _layer_cache(w, layer, lens):
+    return oracle.Cache(w.dtype, w.k[layer:layer + 1], w.v[layer:layer + 1],
+                        lens[layer:layer + 1], w.h_kv, w.d)
+
+
+@pytest.mark.parametrize("step", [0, 7])
+def test_staged_sparse_full_launch_sampled_layers(c3_full, step):
+    """The benchmark's exact staged sparse call: 28 layers x (1,024 selected + tail) in one
+    launch, three layers checked in full against the oracle (with the oracle's own top-K)."""
+    w, k, v, idx = c3_full
+    nq = int(w.n_q_verify[0])
+    tail = w.l_vis.astype(np.int32)
+    kv0 = dev.kv_cache(w, kv_len=w.kv_len_draft(0), k=k, v=v)
+    sel = sd.sd_sparse_stage(kv0, dev.int32(idx), dev.int32(tail))
+    lens = w.kv_len_draft(step)
+    max_tail = int(max(int((w.kv_len_draft(t) - w.l_vis).max()) for t in range(int(w.gamma[0]))))
+    out = sd.sd_sparse_attention_staged(dev.draft_queries(w, step),
+                                        dev.kv_cache(w, kv_len=lens, k=k, v=v), sel, w.topk,
+                                        dev.int32(tail), max_tail)
+    got = dev.to_numpy_f64(out)
+    assert np.isfinite(got).all()
+    for layer in SAMPLED_LAYERS:
+        ridx, gap = oracle.topk_select(w.h_q, w.q_verify[layer * nq:(layer + 1) * nq], [0, nq],
+                                       _layer_cache(w, layer, w.kv_len_verify), [0],
+                                       w.l_vis[layer:layer + 1], w.topk)
+        assert np.array_equal(idx[layer:layer + 1], ridx), (layer, gap)
+        ref = oracle.sparse_attention(w.h_q, w.q_draft[step][layer:layer + 1], [0, 1],
+                                      _layer_cache(w, layer, lens), ridx, tail[layer:layer + 1])
+        err = np.abs(got[layer:layer + 1] - ref).max()
+        assert err <= TOL[w.dtype], (layer, step, err)
+
+
+@pytest.mark.parametrize("step", [0, 7])
+def test_text_anchored_full_launch_sampled_layers(c3_full, step):
+    """The benchmark's exact text-anchored call: 28 layers, window 1,024 above a 25,000-position
+    visual span, one launch; three layers checked in full."""
+    w, k, v, _ = c3_full
+    L = w.n_seq
+    lens = w.kv_len_draft(step)
+    vb, ve = np.zeros(L, np.int32), w.l_vis.astype(np.int32)
+    out = sd.sd_text_anchored_attention(dev.draft_queries(w, step),
+                                        dev.kv_cache(w, kv_len=lens, k=k, v=v), dev.int32(vb),
+                                        dev.int32(ve), dev.int32(w.window), int(w.window.max()))
+    got = dev.to_numpy_f64(out)
+    assert np.isfinite(got).all()
+    for layer in SAMPLED_LAYERS:
+        sl = slice(layer, layer + 1)
+        ref = oracle.text_anchored_attention(w.h_q, w.q_draft[step][sl], [0, 1],
+                                             _layer_cache(w, layer, lens), vb[sl], ve[sl],
+                                             w.window[sl])
+        err = np.abs(got[sl] - ref).max()
+        assert err <= TOL[w.dtype], (layer, step, err)
