@@ -52,12 +52,15 @@ def configure(handle):
     handle.orc_sparse_attention.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp]
     handle.orc_topk_select.argtypes = [vp, vp, vp, i32, vp, vp, i32, vp, vp]
     handle.orc_topk_scores.argtypes = [vp, vp, vp, i32, vp, vp, i64, vp]
+    handle.orc_topk_attention_scores.argtypes = [vp, vp, vp, i32, vp, vp, i64, vp]
+    handle.orc_topk_select_attention.argtypes = [vp, vp, vp, i32, vp, vp, i32, vp, vp]
     handle.orc_hsr_project.argtypes = [vp, vp, i32, i32, vp, vp, vp]
     handle.orc_accept_greedy.argtypes = [vp, vp, vp, i32, i32, vp, vp, i32]
     handle.orc_accept_sample.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp]
     handle.orc_set_threads.argtypes = [i32]
     for name in ("orc_verify_attention", "orc_decode_attention", "orc_text_anchored_attention",
                  "orc_sparse_attention", "orc_topk_select", "orc_topk_scores",
+                 "orc_topk_attention_scores", "orc_topk_select_attention",
                  "orc_hsr_project", "orc_accept_greedy", "orc_accept_sample",
                  "orc_set_threads"):
         getattr(handle, name).restype = ctypes.c_int
@@ -203,6 +206,39 @@ def topk_scores(h_q, q, q_start, cache: Cache, cand_begin, cand_end):
                                _ptr(cb), _ptr(ce), width, _ptr(sc))
     _check(rc, "topk_scores")
     return sc
+
+
+def topk_attention_scores(h_q, q, q_start, cache: Cache, cand_begin, cand_end,
+                          scale: float = 0.0):
+    """Mean attention weight that the text query rows of every sequence (the last rows of its
+    cache, causal) give each candidate, averaged over rows and the KV head's query heads:
+    float64 [batch][h_kv][max candidates] (NaN where unused)."""
+    qs, keep = _query(h_q, q_start, scale)
+    qd = _c(q)
+    batch = len(keep) - 1
+    cb, ce = _c(cand_begin, np.int32), _c(cand_end, np.int32)
+    width = int(max(1, (ce - cb).max()))
+    sc = np.full((batch, cache.h_kv, width), np.nan, dtype=np.float64)
+    rc = lib().orc_topk_attention_scores(ctypes.byref(qs), _ptr(qd), ctypes.byref(cache.struct),
+                                         batch, _ptr(cb), _ptr(ce), width, _ptr(sc))
+    _check(rc, "topk_attention_scores")
+    return sc
+
+
+def topk_select_attention(h_q, q, q_start, cache: Cache, cand_begin, cand_end, k: int,
+                          scale: float = 0.0):
+    """Top-K by mean text attention.  Returns (idx [batch][h_kv][k] int32 ascending, -1 padded;
+    gap [batch][h_kv] float64: (score_k - score_k+1) / score_1)."""
+    qs, keep = _query(h_q, q_start, scale)
+    qd = _c(q)
+    batch = len(keep) - 1
+    cb, ce = _c(cand_begin, np.int32), _c(cand_end, np.int32)
+    idx = np.full((batch, cache.h_kv, k), -1, dtype=np.int32)
+    gap = np.zeros((batch, cache.h_kv), dtype=np.float64)
+    rc = lib().orc_topk_select_attention(ctypes.byref(qs), _ptr(qd), ctypes.byref(cache.struct),
+                                         batch, _ptr(cb), _ptr(ce), int(k), _ptr(idx), _ptr(gap))
+    _check(rc, "topk_select_attention")
+    return idx, gap
 
 
 def hsr_project(emb, hid, weight, bias=None):

@@ -425,6 +425,129 @@ int orc_topk_scores(const orc_query *q, const void *qdata, const orc_cache *c, i
     return err;
 }
 
+/* ---------------------------------------------------------------- mean text attention -- */
+
+/* Sparse-to-Dense's own selection score [StD "Selecao de Cache KV": the top-K visual KV
+ * entries are chosen at prefill from the mean attention scores that the text tokens direct to
+ * the visual tokens, separately for every layer and head].  The query rows of sequence b are
+ * its prefill text tokens: the last n_q positions of its cache, row i at position
+ * kv_len - n_q + i, attending causally (j <= limit_i = kv_len - n_q + i) with its own softmax
+ * over every position it sees.  For KV head g and candidate j, with the G query heads h of the
+ * group:
+ *     a_{h,i}(j) = exp(s_{h,i,j} - m_{h,i}) / sum_{j' <= limit_i} exp(s_{h,i,j'} - m_{h,i})
+ *                  (0 when j > limit_i),   s = scale * q_{h,i} . k_j,   m = max over j' <= limit_i
+ *     score_j    = 1 / (G * n_q) * sum_h sum_i a_{h,i}(j)
+ * (the mean over the group's heads as well as the text rows: one KV entry serves the whole
+ * group).  scores[(b*h_kv+g)*row_width + t] receives the score of candidate cand_begin[b] + t. */
+int orc_topk_attention_scores(const orc_query *q, const void *qdata, const orc_cache *c,
+                              int batch, const int32_t *cand_begin, const int32_t *cand_end,
+                              int64_t row_width, double *scores)
+{
+    if (q->h_q % c->h_kv != 0)
+        return ORC_ERR_ARG;
+    const int d = c->head_dim, hq = q->h_q, hk = c->h_kv, G = hq / hk;
+    const double scale = orc_scale(q, d);
+    int err = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int w = 0; w < batch * hk; ++w) {
+        int b = w / hk, g = w % hk;
+        int64_t kv_len = c->kv_len[b];
+        int64_t r0 = q->q_start[b], n_q = q->q_start[b + 1] - r0;
+        int64_t cb = cand_begin[b], ce = cand_end[b];
+        double *dst = scores + (int64_t)w * row_width;
+        for (int64_t t = 0; t < row_width; ++t)
+            dst[t] = (t < ce - cb) ? 0.0 : NAN;
+        if (n_q < 1 || kv_len < n_q)
+            continue;
+        double *s = (double *)malloc(sizeof(double) * (size_t)kv_len);
+        double *qv = (double *)malloc(sizeof(double) * (size_t)d);
+        for (int h = g * G; h < (g + 1) * G; ++h) {
+            for (int64_t i = 0; i < n_q; ++i) {
+                int64_t limit = kv_len - n_q + i;
+                for (int e = 0; e < d; ++e)
+                    qv[e] = orc_widen(qdata, c->dtype, ((r0 + i) * hq + h) * d + e);
+                /* every score the row sees, then its softmax denominator */
+                double m = -INFINITY;
+                for (int64_t j = 0; j <= limit; ++j) {
+                    int64_t kr = orc_kv_row(c, b, g, j);
+                    double dot = 0.0;
+                    if (kr < 0) {
+#pragma omp atomic write
+                        err = ORC_ERR_ARG;
+                    } else {
+                        for (int e = 0; e < d; ++e)
+                            dot += qv[e] * orc_widen(c->k, c->dtype, kr + e);
+                    }
+                    s[j] = scale * dot;
+                    if (s[j] > m)
+                        m = s[j];
+                }
+                double den = 0.0;
+                for (int64_t j = 0; j <= limit; ++j)
+                    den += exp(s[j] - m);
+                /* this row's weights of the candidates it sees */
+                for (int64_t j = cb; j < ce && j <= limit && j - cb < row_width; ++j)
+                    if (j >= 0)
+                        dst[j - cb] += exp(s[j] - m) / den;
+            }
+        }
+        for (int64_t t = 0; t < ce - cb && t < row_width; ++t)
+            dst[t] /= (double)G * (double)n_q;
+        free(qv);
+        free(s);
+    }
+    return err;
+}
+
+/* Top-K selection by the mean text attention above: the k highest scores of every
+ * (sequence, KV head), equal scores going to the lower position, written in ascending position
+ * order with -1 in unused slots (the same selection rule as orc_topk_select).  gap[b*h_kv+g]
+ * receives (score_(k) - score_(k+1)) / score_(1), or +inf when every candidate is selected. */
+int orc_topk_select_attention(const orc_query *q, const void *qdata, const orc_cache *c,
+                              int batch, const int32_t *cand_begin, const int32_t *cand_end,
+                              int k, int32_t *idx_out, double *gap)
+{
+    if (k < 1 || q->h_q % c->h_kv != 0)
+        return ORC_ERR_ARG;
+    const int hk = c->h_kv;
+    int64_t width = 1;
+    for (int b = 0; b < batch; ++b)
+        if ((int64_t)cand_end[b] - cand_begin[b] > width)
+            width = (int64_t)cand_end[b] - cand_begin[b];
+    double *all = (double *)malloc(sizeof(double) * (size_t)(batch * hk) * (size_t)width);
+    int err = orc_topk_attention_scores(q, qdata, c, batch, cand_begin, cand_end, width, all);
+    for (int w = 0; w < batch * hk; ++w) {
+        int b = w / hk;
+        int64_t cb = cand_begin[b], n = (int64_t)cand_end[b] - cb;
+        int32_t *dst = idx_out + (int64_t)w * k;
+        for (int e = 0; e < k; ++e)
+            dst[e] = -1;
+        if (n <= 0) {
+            if (gap) gap[w] = INFINITY;
+            continue;
+        }
+        orc_scored *sc = (orc_scored *)malloc(sizeof(orc_scored) * (size_t)n);
+        for (int64_t t = 0; t < n; ++t) {
+            sc[t].s = all[(int64_t)w * width + t];
+            sc[t].j = cb + t;
+        }
+        qsort(sc, (size_t)n, sizeof(orc_scored), orc_cmp_scored);
+        int64_t take = n < k ? n : k;
+        for (int64_t e = 0; e < take; ++e)
+            dst[e] = (int32_t)sc[e].j;
+        qsort(dst, (size_t)take, sizeof(int32_t), orc_cmp_i32);
+        if (gap) {
+            if (n <= k)
+                gap[w] = INFINITY;
+            else
+                gap[w] = sc[0].s > 0.0 ? (sc[k - 1].s - sc[k].s) / sc[0].s : 0.0;
+        }
+        free(sc);
+    }
+    free(all);
+    return err;
+}
+
 /* ---------------------------------------------------------------- HSR projection --------- */
 
 /* Hidden-state reuse [SPW 3.1]: the draft input is an FC over the concatenation

@@ -53,6 +53,12 @@ int orc_topk_select(const orc_query *q, const void *qdata, const orc_cache *c, i
 int orc_topk_scores(const orc_query *q, const void *qdata, const orc_cache *c, int batch,
                     const int32_t *cand_begin, const int32_t *cand_end, int64_t row_width,
                     double *scores);
+int orc_topk_attention_scores(const orc_query *q, const void *qdata, const orc_cache *c,
+                              int batch, const int32_t *cand_begin, const int32_t *cand_end,
+                              int64_t row_width, double *scores);
+int orc_topk_select_attention(const orc_query *q, const void *qdata, const orc_cache *c,
+                              int batch, const int32_t *cand_begin, const int32_t *cand_end,
+                              int k, int32_t *idx_out, double *gap);
 int orc_hsr_project(const uint16_t *emb, const uint16_t *hid, int n, int d_model,
                     const uint16_t *w, const uint16_t *bias, double *y);
 int orc_accept_greedy(const float *tgt, const int32_t *draft, const int32_t *gamma, int batch,

@@ -296,6 +296,25 @@ def make_attn_workload(cfg_index: int, layers: Optional[int] = None, l_vis: Opti
         window=window.astype(np.int32), topk=int(cfg["topk"]))
 
 
+def make_text_queries(w: AttnWorkload, seed: Optional[int] = None):
+    """Prefill query rows of every sequence's text tokens, for selecting the kept KV entries at
+    prefill: ``(q_text [sum(l_txt)][h_q][d] in the KV storage type, q_start [n_seq + 1])``.
+
+    The text tokens are the positions [l_vis, l_vis + l_txt) of each cache, i.e. the last
+    ``l_txt`` positions of a cache holding the ``ctx_len`` prefill positions.  Rows are N(0, 1)
+    drawn per sequence (seed ``SEED_BASE + cfg + 2000 * (sequence + 1)``)."""
+    q_start = np.zeros(w.n_seq + 1, dtype=np.int32)
+    q_start[1:] = np.cumsum(w.l_txt)
+    st = np.uint16 if w.dtype == BF16 else np.float32
+    q = np.empty((int(q_start[-1]), w.h_q, w.d), dtype=st)
+    base = SEED_BASE + w.cfg_index if seed is None else seed
+    for s in range(w.n_seq):
+        rng = np.random.Generator(np.random.PCG64(base + 2000 * (s + 1)))
+        rows = rng.standard_normal((int(w.l_txt[s]), w.h_q, w.d), dtype=np.float32)
+        q[q_start[s]:q_start[s + 1]] = to_kv_dtype(rows, w.dtype)
+    return q, q_start
+
+
 @dataclasses.dataclass
 class AcceptWorkload:
     """Logits, drafted tokens and uniforms for a batch of acceptance problems.

@@ -16,6 +16,7 @@ from oracle import build as obuild
 
 from . import test_oracle_accept as ta
 from . import test_oracle_attention as tt
+from . import test_oracle_text_attention as tx
 from . import test_oracle_topk_hsr as tk
 
 ATTN = [tt.test_golden_attention_tiny, lambda: tt.test_verify_matches_torch_sdpa("f32"),
@@ -27,6 +28,10 @@ SPARSE = [tt.test_sparse_matches_torch_with_explicit_set_mask,
 TOPK = [tk.test_golden_topk_tiny, lambda: tk.test_topk_brute_force_over_all_subsets(0, 3),
         tk.test_topk_duplicated_keys_tie_to_lower_positions]
 HSR = [tk.test_hsr_matches_torch_fp64_matmul, tk.test_hsr_concatenation_order]
+TEXT_ATTN = [tx.test_golden_text_attention_tiny, lambda: tx.test_scores_over_every_position_sum_to_one(0),
+             lambda: tx.test_scores_equal_mean_attention_output_with_one_hot_values(1, 3),
+             tx.test_zero_keys_give_uniform_weights_closed_form,
+             tx.test_candidates_beyond_a_rows_causal_limit_get_only_the_later_rows]
 GREEDY = [ta.test_golden_accept_greedy_tiny, ta.test_greedy_argmax_ties_nan_and_signed_zero,
           ta.test_greedy_own_argmax_accepts_everything]
 SAMPLE = [ta.test_golden_accept_sample_tiny,
@@ -49,6 +54,15 @@ MUTANTS = {
                             "return (x->j > y->j) ? -1 : (x->j < y->j);", TOPK),
     "topk_smallest_scores": ("if (x->s > y->s) return -1;\n    if (x->s < y->s) return 1;",
                              "if (x->s < y->s) return -1;\n    if (x->s > y->s) return 1;", TOPK),
+    "text_attention_not_causal": ("int64_t limit = kv_len - n_q + i;\n                for (int e = 0; e < d; ++e)",
+                                  "int64_t limit = kv_len - 1;\n                for (int e = 0; e < d; ++e)", TEXT_ATTN),
+    "text_attention_sum_not_mean_over_heads": ("dst[t] /= (double)G * (double)n_q;",
+                                               "dst[t] /= (double)n_q;", TEXT_ATTN),
+    "text_attention_first_head_of_group_only": ("for (int h = g * G; h < (g + 1) * G; ++h) {\n            for (int64_t i = 0; i < n_q; ++i) {",
+                                                "for (int h = g * G; h < g * G + 1; ++h) {\n            for (int64_t i = 0; i < n_q; ++i) {", TEXT_ATTN),
+    "text_attention_unscaled": ("s[j] = scale * dot;", "s[j] = dot;", TEXT_ATTN),
+    "text_attention_denominator_from_candidates": ("for (int64_t j = 0; j <= limit; ++j)\n                    den += exp(s[j] - m);",
+                                                   "for (int64_t j = cb; j <= limit && j < ce; ++j)\n                    den += exp(s[j] - m);", TEXT_ATTN),
     "hsr_hidden_reads_first_half": ("o * 2 * D + D + i", "o * 2 * D + i", HSR),
     "argmax_ties_to_higher": ("if (isnan(z[best]) || z[x] > z[best])", "if (isnan(z[best]) || z[x] >= z[best])", GREEDY),
     "greedy_bonus_from_draft": ("out_tok[(int64_t)b * out_stride + n] = (int32_t)t_n;",
