@@ -496,6 +496,62 @@ def plain_decoding(cyc, torch, reps):
     return res
 
 
+def peak_bf16():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def prefill_selection(cyc, torch, reps=3):
+    """Sparse-to-Dense's own selection (mean text attention at prefill) over the workload's
+    layers: the text rows of every layer score every visual key; timed with CUDA events.
+    FLOPs: both passes' Q.K products (pass 1 over every position a row sees, pass 2 over the
+    candidates), 2 * d per product."""
+    sd, dev, gen, w = cyc.sd, cyc.dev, cyc.gen, cyc.w
+    if w.dtype != "bf16":
+        return None
+    qt, qs = gen.make_text_queries(w)
+    device = cyc.k.device
+    q = dev.queries(qt, qs, w.dtype, int(w.ctx_len.max()), device)
+    kv = dev.kv_cache(w, kv_len=w.ctx_len, device=device, k=cyc.k, v=cyc.v)
+    cb = dev.int32(np.zeros(w.n_seq), device)
+    ce = dev.int32(w.l_vis, device)
+    max_cand = int(w.l_vis.max())
+    idx = torch.empty((w.n_seq, w.h_kv, w.topk), dtype=torch.int32, device=device)
+    ws = torch.empty(sd.sd_topk_scored_workspace_size(sd.SD_TOPK_MEAN_TEXT_ATTENTION, q, kv,
+                                                      max_cand, w.topk),
+                     dtype=torch.uint8, device=device)
+    call = lambda: sd.sd_topk_select_scored(sd.SD_TOPK_MEAN_TEXT_ATTENTION, q, kv, cb, ce,
+                                            max_cand, w.topk, idx_out=idx, workspace=ws)
+    call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    flop = 0
+    for s in range(w.n_seq):
+        n_q, ctx = int(w.l_txt[s]), int(w.ctx_len[s])
+        seen = sum(ctx - n_q + i + 1 for i in range(n_q))  # pass 1
+        flop += w.h_q * 2 * w.d * (seen + n_q * int(w.l_vis[s]))  # + pass 2
+    peak, kind = peak_bf16()
+    tf = flop / (ms / 1e3) / 1e12
+    return {"call": "sd_topk_select_scored (SD_TOPK_MEAN_TEXT_ATTENTION)",
+            "kernels": "text_lse_tc_kernel + text_colsum_tc_kernel + topk_select_smem_kernel",
+            "layers": w.n_seq, "text_rows": int(w.l_txt.max()), "visual_keys": max_cand,
+            "ms": round(ms, 3), "flop": int(flop), "achieved_tflops": round(tf, 1),
+            "bound": "tensor (and the exponentials)", "peak_tflops": peak,
+            "peak_source": f"{kind} bf16_tflops", "frac": round(tf / peak, 4),
+            "exp2_per_launch": int(flop // (2 * w.d))}
+
+
 class HostIO:
     """Per-step inputs in pinned host memory and the end-to-end loop: the next step's inputs
     are copied on a second stream while the current step computes (two device input sets);
@@ -755,6 +811,11 @@ def run_ours(args):
     plain = plain_decoding(cyc, torch, reps=max(5, args.steps // 2)) if not args.no_plain \
         else None
 
+    # ---- Sparse-to-Dense's prefill selection (once per video, outside the decode cycle) ----
+    prefill = prefill_selection(cyc, torch) if cyc.spec["topk"] and not args.no_prefill \
+        else None
+    torch.cuda.empty_cache()
+
     # ---- end to end through the public API, host buffers, copies inside the timed region ----
     host = HostIO(cyc)
     host.run(cyc, 2)
@@ -781,6 +842,7 @@ def run_ours(args):
             "rooflines": rooflines,
             "layer_latency": layer_latency,
             "plain_decoding": plain,
+            "prefill_selection": prefill,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": host.h2d_bytes, "d2h_bytes_per_step": host.d2h_bytes,
                     "ms_per_step": round(e2e_ms / args.steps, 4),
@@ -922,7 +984,7 @@ def run_reference(args):
 
 
 CASES = ("verify", "sparse", "sparse_staged", "stage", "text_anchored", "topk", "hsr",
-         "accept_greedy", "accept_sample", "decode")
+         "accept_greedy", "accept_sample", "decode", "prefill_select")
 
 
 def run_case(args):
@@ -951,6 +1013,13 @@ def run_case(args):
     elif args.case == "topk":
         call = lambda: sd.sd_topk_select(qv, kv_verify, i32(np.zeros(L)), i32(w.l_vis),
                                          int(w.l_vis.max()), w.topk)
+    elif args.case == "prefill_select":
+        qt, qs = gen.make_text_queries(w)
+        qp = dev.queries(qt, qs, w.dtype, int(w.ctx_len.max()))
+        kvp = dev.kv_cache(w, kv_len=w.ctx_len, k=k, v=v)
+        call = lambda: sd.sd_topk_select_scored(sd.SD_TOPK_MEAN_TEXT_ATTENTION, qp, kvp,
+                                                i32(np.zeros(L)), i32(w.l_vis),
+                                                int(w.l_vis.max()), w.topk)
     elif args.case in ("sparse", "sparse_staged", "stage"):
         idx = sd.sd_topk_select(qv, kv_verify, i32(np.zeros(L)), i32(w.l_vis),
                                 int(w.l_vis.max()), w.topk)
@@ -1002,6 +1071,8 @@ def main():
     ap.add_argument("--call-reps", type=int, default=10,
                     help="separately timed repetitions of every call for the per-call rooflines")
     ap.add_argument("--no-plain", action="store_true", help="skip the plain-decoding comparison")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill (mean text attention) selection")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--case", choices=CASES, default=None,

@@ -19,7 +19,9 @@
  * Conventions shared by every call
  *  - Every pointer argument is DEVICE memory owned by the caller unless stated otherwise;
  *    descriptor structs themselves are read on the host during the call and may be freed
- *    after it returns.  The library allocates no device memory and keeps no global state;
+ *    after it returns.  The library allocates no device memory and keeps no global state
+ *    (except the wait bound of sd_set_wait_timeout_ns and the fixed scratch of
+ *    sd_verify_attention_noalloc);
  *    scratch memory ("workspace") is passed in by the caller, sized by the *_workspace_size
  *    queries.  Calls on different streams with different workspaces may run concurrently.
  *  - Calls are asynchronous and stream-ordered on `stream` (a cudaStream_t; NULL means the
@@ -132,6 +134,17 @@ SD_API const char *sd_status_string(sd_status s);
 
 /* Library version, major*10000 + minor*100 + patch. */
 SD_API int32_t sd_version(void);
+
+/*
+ * Bound of every wait inside the library's tensor-core kernels (a pipeline stage waiting for a
+ * copy or an MMA that another warp of the same CTA issues).  A wait that runs out sets
+ * SD_DEVERR_TIMEOUT in the call's dev_err; the CTA then waits (at most 1 s more) for the copies
+ * and MMAs it has already issued, frees its tensor memory and exits, so the device stays usable
+ * and the call's outputs are undefined.  Process-wide, for the calls launched after it returns;
+ * ns = 0 restores the default of 1 s (1e9 ns).  Returns the previous bound.  Meant for failure
+ * detection and its tests: a bound of 1 ns makes a call's waits run out at once.
+ */
+SD_API uint64_t sd_set_wait_timeout_ns(uint64_t ns);
 
 /*
  * Workspace bytes a verify or text-anchored call needs for these descriptors (host hints only;
@@ -252,6 +265,51 @@ SD_API sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd
                          int32_t batch, const int32_t *cand_begin, const int32_t *cand_end,
                          int32_t max_cand, int32_t k, int32_t *idx_out, void *workspace,
                          size_t workspace_bytes, int32_t *dev_err, void *stream);
+
+/*
+ * Score modes of the top-K selection.
+ *  SD_TOPK_LAST_QUERY            the score of sd_topk_select: the sum over the KV head's query
+ *                                heads of the sequence's last query row dotted with k_j.
+ *  SD_TOPK_MEAN_TEXT_ATTENTION   Sparse-to-Dense's own rule [StD "Selecao de Cache KV": the
+ *                                top-K visual KV entries are chosen at prefill from the mean
+ *                                attention the text tokens direct to the visual tokens, per
+ *                                layer and head]: the query rows of sequence b are its n_q
+ *                                prefill text rows, the LAST n_q positions of its cache (row i
+ *                                at position kv_len[b] - n_q + i), each attending causally with
+ *                                its own softmax (scale softmax_scale, 0 = 1/sqrt(d)) over every
+ *                                position it sees; the score of candidate j is its attention
+ *                                weight averaged over the n_q rows and the G query heads:
+ *                                  score_j = 1/(G n_q) sum_h sum_i a_{h,i}(j)
+ */
+typedef enum { SD_TOPK_LAST_QUERY = 0, SD_TOPK_MEAN_TEXT_ATTENTION = 1 } sd_topk_score;
+
+/*
+ * Workspace of sd_topk_select_scored.  Mode SD_TOPK_MEAN_TEXT_ATTENTION also holds one float
+ * per (text row, query head): batch * q->max_q_rows * q->h_q * 4 bytes beyond the keys.
+ */
+SD_API sd_status sd_topk_scored_workspace_size(sd_topk_score mode, const sd_q_desc *q,
+                                               const sd_kv_desc *kv, int32_t batch,
+                                               int32_t max_cand, int32_t k, size_t *bytes);
+
+/*
+ * Top-K selection with a score mode (see sd_topk_score).  SD_TOPK_LAST_QUERY computes exactly
+ * what sd_topk_select computes.  The selection rule is the same for both modes: the k highest
+ * scores of every (sequence, KV head) among [cand_begin[b], cand_end[b]), equal scores to the
+ * lower position, written ascending to idx_out [batch][h_kv][k] (-1 padded).
+ * scores_out (device double [batch][h_kv][max_cand], may be NULL) receives every candidate's
+ * score (slot t: candidate cand_begin[b] + t); NaN-free inputs give finite scores.
+ * SD_TOPK_MEAN_TEXT_ATTENTION: q / q_data hold the prefill text rows (q->max_q_rows bounds the
+ * rows of every sequence; q->max_kv_len bounds kv_len); its scores are accumulated in fp32 per
+ * 128-row tile and in fp64 across tiles, with the scores themselves from fp32 tensor-core
+ * products of the bf16 inputs (CUDA cores for fp32 caches), so two scores closer than about
+ * 1e-5 relative may rank in either order.
+ */
+SD_API sd_status sd_topk_select_scored(sd_topk_score mode, const sd_q_desc *q, const void *q_data,
+                                       const sd_kv_desc *kv, int32_t batch,
+                                       const int32_t *cand_begin, const int32_t *cand_end,
+                                       int32_t max_cand, int32_t k, int32_t *idx_out,
+                                       double *scores_out, void *workspace,
+                                       size_t workspace_bytes, int32_t *dev_err, void *stream);
 
 /*
  * Hidden-state reuse projection [SPW 3.1]: the draft input is an FC over the concatenation

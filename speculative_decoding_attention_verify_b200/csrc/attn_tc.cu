@@ -225,7 +225,8 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 }
                 const CUtensorMap *map = cmp ? (half == 0 ? &maps.k2 : &maps.v2)
                                              : (half == 0 ? &maps.k : &maps.v);
-                if (t >= S && !mbar_wait(BAR(empty + s), (use - 1) & 1, abort_flag, p.dev_err))
+                if (t >= S && !mbar_wait(BAR(empty + s), (use - 1) & 1, abort_flag, p.dev_err,
+                                         p.wait_ns))
                     break;
                 mbar_arrive_tx(BAR(full + s), C::kTileBytes);
                 if (!PAGED || cmp) {
@@ -303,8 +304,8 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         if (n_my > 0) {
             bool qok = true;
             if (lane == 0)
-                qok = mbar_wait(BAR(QF), 0, abort_flag, p.dev_err) &&
-                      mbar_wait(BAR(KF), 0, abort_flag, p.dev_err);
+                qok = mbar_wait(BAR(QF), 0, abort_flag, p.dev_err, p.wait_ns) &&
+                      mbar_wait(BAR(KF), 0, abort_flag, p.dev_err, p.wait_ns);
             alive = __shfl_sync(0xffffffffu, qok ? 1 : 0, 0) != 0;
             if (alive) issue_qk(0);
         }
@@ -327,7 +328,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                     if (flags == 0 && (it & 63u) == 0) {
                         if (*abort_flag) {
                             flags = 4;
-                        } else if (now_ns() - t0 > kWaitNs) {
+                        } else if (now_ns() - t0 > p.wait_ns) {
                             *abort_flag = 1;
                             set_dev_err(p.dev_err, SD_DEVERR_TIMEOUT);
                             flags = 4;
@@ -354,7 +355,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         if (lane == 0 && any_issued) {
             mma_commit(BAR(DR));
             const unsigned long long t0 = now_ns();
-            while (!mbar_try(BAR(DR), 0) && now_ns() - t0 < kWaitNs) {
+            while (!mbar_try(BAR(DR), 0) && now_ns() - t0 < kDrainNs) {
             }
         }
         __syncwarp();
@@ -402,7 +403,8 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             // the run this tile belongs to: positions [seg_lo, seg_hi)
             const int seg_lo = tt < nt0 ? si.s0 : si.s1;
             const int seg_hi = tt < nt0 ? si.s0 + si.len0 : si.s1 + si.len1;
-            const bool got = mbar_wait(BAR(SF + sb), (t >> 1) & 1, abort_flag, p.dev_err);
+            const bool got =
+                mbar_wait(BAR(SF + sb), (t >> 1) & 1, abort_flag, p.dev_err, p.wait_ns);
             if (!__all_sync(FULL, got)) {
                 ok_run = false;
                 break;
@@ -459,7 +461,8 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 // O holds tiles < t: wait for the P.V of tile t-1, then rescale O in TMEM.
                 // S_t was committed after the P.V of tile t-2 and the P.V of tile t needs this
                 // warp's arrival, so o_done is in phase t-1 or t: its parity test is exact.
-                const bool done = mbar_wait(BAR(OD), (t - 1) & 1, abort_flag, p.dev_err);
+                const bool done =
+                    mbar_wait(BAR(OD), (t - 1) & 1, abort_flag, p.dev_err, p.wait_ns);
                 if (!__all_sync(FULL, done)) {
                     ok_run = false;
                     break;
@@ -511,7 +514,8 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         // per-tile o_done barrier: here only the P.V of tiles < n_my - 2 is known to be
         // complete, so o_done could be two phases behind and its parity test would pass early.
         bool done = ok_run;
-        if (ok_run && n_my > 0) done = mbar_wait(BAR(DR), 0, abort_flag, p.dev_err);
+        if (ok_run && n_my > 0)
+            done = mbar_wait(BAR(DR), 0, abort_flag, p.dev_err, p.wait_ns);
         const bool read_o = __all_sync(FULL, done) && n_my > 0;
         tc_after();
         const bool have = read_o && m_used != -INFINITY;
@@ -619,7 +623,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         const int full = lane == 0 ? KF : VF;
         for (int t = (n_issued > S ? n_issued - S : 0); t < n_issued; ++t) {
             const int s = t % S, use = t / S;
-            while (!mbar_try(BAR(full + s), use & 1) && now_ns() - t0 < kWaitNs) {
+            while (!mbar_try(BAR(full + s), use & 1) && now_ns() - t0 < kDrainNs) {
             }
         }
     }

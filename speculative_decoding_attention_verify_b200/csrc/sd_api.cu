@@ -1,12 +1,19 @@
 // C-ABI entry points of libsdattn: host-side validation, decomposition and dispatch.
 // Every check here runs before any launch; on failure nothing is launched.
 #include <math.h>
+#include <atomic>
 #include <stdint.h>
 #include <string.h>
 
 #include "sd_internal.h"
 
 namespace sd {
+
+namespace {
+std::atomic<unsigned long long> g_wait_ns{1000000000ull};
+}  // namespace
+
+unsigned long long wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
 int device_sm_count() {
     int dev = 0, n = 0;
@@ -158,6 +165,7 @@ AttnParams base_params(sd_attn_kind kind, const sd_q_desc *q, const void *q_data
     p.n_rowblocks = plan.n_rowblocks;
     p.ws_o = reinterpret_cast<float *>(ws);
     p.dev_err = dev_err;
+    p.wait_ns = wait_limit_ns();
     return p;
 }
 
@@ -220,6 +228,20 @@ size_t sparse_ws_bytes(const AttnPlan &plan, const sd_kv_desc *kv, int batch, in
     return plan.tensor_core ? sel_layout(plan.ws_bytes, kv, batch, k).end : plan.ws_bytes;
 }
 
+// Workspace of the mean text attention mode: the score keys, then one log-sum-exp per
+// (text row, query head), each region 256-byte aligned.
+struct TaLayout {
+    size_t keys, lse, end;
+};
+
+TaLayout text_attention_ws(int batch, int h_kv, int max_cand, int h_q, int max_q_rows) {
+    TaLayout l{};
+    l.keys = 0;
+    l.lse = up256(topk_workspace_bytes(batch, h_kv, max_cand));
+    l.end = l.lse + up256((size_t)batch * max_q_rows * h_q * sizeof(float));
+    return l;
+}
+
 long long stream_hint(sd_attn_kind kind, const sd_q_desc *q, long long extra) {
     if (kind == SD_ATTN_TEXT_ANCHORED) {
         const long long w = extra + q->max_q_rows - 1;
@@ -266,7 +288,11 @@ const char *sd_status_string(sd_status s) {
     return "unknown sd_status";
 }
 
-int32_t sd_version(void) { return 100; }
+int32_t sd_version(void) { return 200; }
+
+uint64_t sd_set_wait_timeout_ns(uint64_t ns) {
+    return g_wait_ns.exchange(ns == 0 ? 1000000000ull : ns, std::memory_order_relaxed);
+}
 
 sd_status sd_attention_workspace_size(sd_attn_kind kind, const sd_q_desc *q,
                                       const sd_kv_desc *kv, int32_t batch, size_t *bytes) {
@@ -437,14 +463,39 @@ sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd_kv_des
                          int32_t batch, const int32_t *cand_begin, const int32_t *cand_end,
                          int32_t max_cand, int32_t k, int32_t *idx_out, void *workspace,
                          size_t workspace_bytes, int32_t *dev_err, void *stream) {
+    return sd_topk_select_scored(SD_TOPK_LAST_QUERY, q, q_data, kv, batch, cand_begin, cand_end,
+                                 max_cand, k, idx_out, nullptr, workspace, workspace_bytes,
+                                 dev_err, stream);
+}
+
+sd_status sd_topk_scored_workspace_size(sd_topk_score mode, const sd_q_desc *q,
+                                        const sd_kv_desc *kv, int32_t batch, int32_t max_cand,
+                                        int32_t k, size_t *bytes) {
+    if (!kv || !bytes || batch < 1 || max_cand < 0 || k < 1 || kv->h_kv < 1)
+        return SD_ERR_INVALID_ARG;
+    if (mode == SD_TOPK_LAST_QUERY) {
+        *bytes = topk_workspace_bytes(batch, kv->h_kv, max_cand);
+        return SD_OK;
+    }
+    if (mode != SD_TOPK_MEAN_TEXT_ATTENTION || !q || q->h_q < 1 || q->max_q_rows < 1)
+        return SD_ERR_INVALID_ARG;
+    *bytes = text_attention_ws(batch, kv->h_kv, max_cand, q->h_q, q->max_q_rows).end;
+    return SD_OK;
+}
+
+sd_status sd_topk_select_scored(sd_topk_score mode, const sd_q_desc *q, const void *q_data,
+                                const sd_kv_desc *kv, int32_t batch, const int32_t *cand_begin,
+                                const int32_t *cand_end, int32_t max_cand, int32_t k,
+                                int32_t *idx_out, double *scores_out, void *workspace,
+                                size_t workspace_bytes, int32_t *dev_err, void *stream) {
+    if (mode != SD_TOPK_LAST_QUERY && mode != SD_TOPK_MEAN_TEXT_ATTENTION)
+        return SD_ERR_INVALID_ARG;
     if (!q || !q_data || !cand_begin || !cand_end || !idx_out || k < 1 || max_cand < 0 ||
         batch > 65535)
         return SD_ERR_INVALID_ARG;
     if (!kv_desc_ok(kv, batch)) return SD_ERR_INVALID_ARG;
     if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
     if (q->h_q < 1 || q->h_q % kv->h_kv != 0 || !q->q_start) return SD_ERR_INVALID_ARG;
-    const size_t need = topk_workspace_bytes(batch, kv->h_kv, max_cand);
-    if (need > workspace_bytes || (need && !workspace)) return SD_ERR_WORKSPACE;
     TopkParams p{};
     p.kv = make_view(kv);
     p.batch = batch;
@@ -458,7 +509,28 @@ sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd_kv_des
     p.k = k;
     p.idx_out = idx_out;
     p.keys = reinterpret_cast<unsigned long long *>(workspace);
+    p.scores = scores_out;
     p.dev_err = dev_err;
+    p.wait_ns = wait_limit_ns();
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (mode == SD_TOPK_MEAN_TEXT_ATTENTION) {
+        if (q->max_q_rows < 1 || q->max_kv_len < 1 || !(q->softmax_scale >= 0.f) ||
+            isinf(q->softmax_scale) || (long long)batch * q->max_q_rows > (1LL << 30))
+            return SD_ERR_INVALID_ARG;
+        const TaLayout l = text_attention_ws(batch, kv->h_kv, max_cand, q->h_q, q->max_q_rows);
+        if (l.end > workspace_bytes || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+            return SD_ERR_WORKSPACE;
+        p.max_q_rows = q->max_q_rows;
+        p.max_kv_len = q->max_kv_len;
+        p.rows_cap = batch * q->max_q_rows;
+        const float scale = q->softmax_scale > 0.f ? q->softmax_scale
+                                                   : (float)(1.0 / sqrt((double)kv->head_dim));
+        p.scale_log2 = scale * kLog2e;
+        p.lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + l.lse);
+        return cuda_status(launch_text_attention_scores(p, s));
+    }
+    const size_t need = topk_workspace_bytes(batch, kv->h_kv, max_cand);
+    if (need > workspace_bytes || (need && !workspace)) return SD_ERR_WORKSPACE;
     // Scoring CTAs stream 128-candidate spans through a shared-memory ring; choose the split
     // count whose CTAs fill whole waves best, with at least four spans per CTA.
     const int sms = device_sm_count();
@@ -467,17 +539,17 @@ sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd_kv_des
     const long long tiles = ((long long)max_cand + 127) / 128;
     double best = -1.0;
     p.n_splits = 1;
-    for (long long s = 1; s <= 1024; ++s) {
-        if (s > 1 && tiles / s < 4) break;
-        const long long ctas = units * s;
+    for (long long sp = 1; sp <= 1024; ++sp) {
+        if (sp > 1 && tiles / sp < 4) break;
+        const long long ctas = units * sp;
         const long long waves = (ctas + slots - 1) / slots;
-        const double score = (double)ctas / (double)(waves * slots) - 0.005 * (double)s;
+        const double score = (double)ctas / (double)(waves * slots) - 0.005 * (double)sp;
         if (score > best) {
             best = score;
-            p.n_splits = (int)s;
+            p.n_splits = (int)sp;
         }
     }
-    return cuda_status(launch_topk(p, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_topk(p, s));
 }
 
 sd_status sd_hsr_project(const void *emb, const void *hid, int32_t n_rows, int32_t d_model,

@@ -43,6 +43,7 @@ struct AttnParams {
     float *ws_o;   // [n_splits][rows_cap][h_q][head_dim] unnormalised partial outputs
     float *ws_ml;  // [n_splits][rows_cap][h_q][2] (running max in log2 units, sum)
     int32_t *dev_err;
+    unsigned long long wait_ns;  // bound of every pipeline wait inside the kernel
 };
 
 // Decomposition of an attention call (host side; depends on host hints only).  Both the
@@ -59,6 +60,7 @@ struct AttnPlan {
 };
 
 int device_sm_count();
+unsigned long long wait_limit_ns();  // the process-wide bound set by sd_set_wait_timeout_ns
 AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, int batch,
                         int max_q_rows, long long max_stream);
 
@@ -84,10 +86,23 @@ struct TopkParams {
     int n_splits;
     unsigned long long *keys;  // [batch][h_kv][max_cand] order-preserving score keys
     int32_t *dev_err;
+    // mean text attention mode: the query rows are the prefill text rows (the last rows of
+    // each cache); their log-sum-exps (log2 units of the scaled scores) go to lse
+    int max_q_rows;     // host hint of the text rows per sequence
+    int max_kv_len;     // host hint: an upper bound of every kv_len
+    int rows_cap;       // batch * max_q_rows: rows addressable in lse
+    float scale_log2;   // softmax scale * log2(e)
+    float *lse;         // [rows_cap][h_q]
+    double *scores;     // nullable: [batch][h_kv][max_cand] every candidate's score
+    unsigned long long wait_ns;  // bound of every pipeline wait inside the kernels
 };
 size_t topk_workspace_bytes(int batch, int h_kv, int max_cand);
 int topk_score_ctas_per_sm();  // resident scoring CTAs per SM
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t s);
+// The selection half of top-K (radix select of p.keys, ascending output).
+cudaError_t launch_topk_select(const TopkParams &p, cudaStream_t s);
+// Mean text attention scores into p.keys (two passes: row log-sum-exps, then column sums).
+cudaError_t launch_text_attention_scores(const TopkParams &p, cudaStream_t s);
 
 // HSR projection.
 cudaError_t launch_hsr(const void *emb, const void *hid, int n_rows, int d_model, const void *w,

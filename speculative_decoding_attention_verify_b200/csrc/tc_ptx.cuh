@@ -26,7 +26,10 @@ bool encode_kv_maps(const AttnParams &p, int max_kv_len, TcMaps *maps);
 
 namespace tc {
 
-constexpr unsigned long long kWaitNs = 1000000000ull;  // bound of every mbarrier wait (1 s)
+// Bound of the drains after an abort (a CTA waiting for its own copies and MMAs to finish):
+// fixed at 1 s.  The bound of the waits of the pipeline itself is a launch parameter (default
+// 1 s, see sd_set_wait_timeout_ns).
+constexpr unsigned long long kDrainNs = 1000000000ull;
 
 
 __device__ __forceinline__ uint32_t saddr(const void *p) {
@@ -64,10 +67,10 @@ __device__ __forceinline__ unsigned long long now_ns() {
     return t;
 }
 
-// Bounded wait for the phase of `bar` with the given parity.  Returns false when the CTA is
-// aborting (this wait timed out, or another one did).
+// Bounded wait (limit_ns) for the phase of `bar` with the given parity.  Returns false when
+// the CTA is aborting (this wait timed out, or another one did).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          int32_t *dev_err) {
+                                          int32_t *dev_err, unsigned long long limit_ns) {
     if (mbar_try(bar, parity)) return true;
     const unsigned long long t0 = now_ns();
     for (unsigned it = 1;; ++it) {
@@ -76,7 +79,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         // take thousands of cycles while the tensor core and the copy engine stream
         if ((it & 63u) == 0) {
             if (*abort_flag) return false;
-            if (now_ns() - t0 > kWaitNs) {
+            if (now_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
                 set_dev_err(dev_err, SD_DEVERR_TIMEOUT);
                 return false;
@@ -133,6 +136,16 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, 
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
         "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// D (TMEM) += A (shared memory descriptor) * B (shared memory descriptor); acc = 0 overwrites D.
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
 

@@ -15,7 +15,7 @@
 //    equal scores go to the lower position, and block-wide prefix sums write the kept
 //    positions in ascending order.  When the keys fit in shared memory (up to 26,624) they are
 //    loaded once and the select touches shared memory only.
-#include "sd_internal.h"
+#include "topk_common.cuh"
 
 namespace sd {
 namespace {
@@ -25,28 +25,6 @@ constexpr int kScoreTile = 64;    // candidates per staged tile
 constexpr int kScoreThreads = kRowThreads * kScoreTile;
 constexpr int kScoreCtasPerSm = 2;
 constexpr int kSelectThreads = 1024;
-
-__device__ __forceinline__ unsigned long long score_key(double x) {
-    if (x != x) return 0ull;  // NaN ranks lowest
-    x += 0.0;                 // -0 -> +0
-    unsigned long long u = (unsigned long long)__double_as_longlong(x);
-    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
-}
-
-// Clamp the candidate range of sequence b to [0, kv_len) and to max_cand entries.
-__device__ __forceinline__ void cand_range(const TopkParams &p, int b, int &cb, int &n) {
-    const int kv_len = __ldg(p.kv.kv_len + b);
-    int lo = __ldg(p.cand_begin + b), hi = __ldg(p.cand_end + b);
-    const bool bad = lo < 0 || hi > kv_len || hi - lo > p.max_cand ||
-                     (p.kv.page_size != 0 && kv_len > p.kv.max_pages * kPageSize);
-    lo = max(lo, 0);
-    hi = min(hi, kv_len);
-    if (p.kv.page_size != 0) hi = min(hi, p.kv.max_pages * kPageSize);
-    hi = min(hi, lo + p.max_cand);
-    cb = lo;
-    n = max(0, hi - lo);
-    if (bad && threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
-}
 
 // cp.async ring depth: 4 stages of 64 rows (bf16, d = 128: two CTAs x 48 KB ahead per SM),
 // 3 for fp32 rows
@@ -202,7 +180,11 @@ __global__ void __launch_bounds__(kScoreThreads, kScoreCtasPerSm) topk_score_ker
             r += __shfl_xor_sync(0xffffffffu, r, 2);
             if (redo) part = r;
         }
-        if (quarter == 0 && cand < t_end) keys[cand] = live ? score_key(part) : 0ull;
+        if (quarter == 0 && cand < t_end) {
+            keys[cand] = live ? score_key(part) : 0ull;
+            if (p.scores)
+                p.scores[((int64_t)b * p.kv.h_kv + g) * p.max_cand + cand] = live ? part : NAN;
+        }
         __syncthreads();
     }
     cp_async_wait<0>();
@@ -403,6 +385,11 @@ cudaError_t launch_topk(const TopkParams &p, cudaStream_t s) {
     else
         e = bf ? launch_score_t<true, 64>(p, s) : launch_score_t<false, 64>(p, s);
     if (e != cudaSuccess) return e;
+    return launch_topk_select(p, s);
+}
+
+cudaError_t launch_topk_select(const TopkParams &p, cudaStream_t s) {
+    cudaError_t e;
     dim3 grid(p.kv.h_kv, p.batch);
     if (p.max_cand <= kSmemKeys) {
         const size_t dyn = (size_t)p.max_cand * sizeof(unsigned long long);

@@ -21,6 +21,7 @@ from . import build as _build
 SD_OK, SD_ERR_INVALID_ARG, SD_ERR_UNSUPPORTED, SD_ERR_WORKSPACE, SD_ERR_CUDA = range(5)
 SD_F32, SD_BF16 = 0, 1
 SD_ATTN_VERIFY, SD_ATTN_TEXT_ANCHORED, SD_ATTN_SPARSE = 0, 1, 2
+SD_TOPK_LAST_QUERY, SD_TOPK_MEAN_TEXT_ATTENTION = 0, 1
 SD_DEVERR_PAGE, SD_DEVERR_INDEX, SD_DEVERR_TOKEN, SD_DEVERR_NUMERIC, SD_DEVERR_SHAPE = 1, 2, 4, 8, 16
 SD_DEVERR_TIMEOUT = 32
 PAGE_SIZE = 16
@@ -54,7 +55,8 @@ EXPORTS = ("sd_status_string", "sd_version", "sd_attention_workspace_size", "sd_
            "sd_text_anchored_attention", "sd_sparse_attention", "sd_topk_workspace_size",
            "sd_topk_select", "sd_hsr_project", "sd_accept_workspace_size", "sd_accept_greedy",
            "sd_accept_sample", "sd_verify_attention_noalloc", "sd_sparse_workspace_size",
-           "sd_sparse_selection_size", "sd_sparse_stage", "sd_sparse_attention_staged")
+           "sd_sparse_selection_size", "sd_sparse_stage", "sd_sparse_attention_staged",
+           "sd_topk_scored_workspace_size", "sd_topk_select_scored", "sd_set_wait_timeout_ns")
 
 # Size of the library's fixed scratch used by sd_verify_attention_noalloc.
 SD_VERIFY_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -74,6 +76,8 @@ def lib():
                 h.sd_status_string.restype = ctypes.c_char_p
                 h.sd_status_string.argtypes = [ctypes.c_int]
                 h.sd_version.restype = I32
+                h.sd_set_wait_timeout_ns.restype = ctypes.c_uint64
+                h.sd_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
                 h.sd_attention_workspace_size.argtypes = [ctypes.c_int, P, P, I32, ctypes.POINTER(SZ)]
                 h.sd_verify_attention.argtypes = [P, P, P, I32, P, P, SZ, P, P]
                 h.sd_text_anchored_attention.argtypes = [P, P, P, I32, P, P, P, I32, P, P, SZ, P, P]
@@ -91,8 +95,13 @@ def lib():
                 h.sd_sparse_stage.argtypes = [P, I32, P, I32, P, P, SZ, P, P]
                 h.sd_sparse_attention_staged.argtypes = [P, P, P, I32, P, I32, P, I32, P, P, SZ,
                                                          P, P]
+                h.sd_topk_scored_workspace_size.argtypes = [ctypes.c_int, P, P, I32, I32, I32,
+                                                            ctypes.POINTER(SZ)]
+                h.sd_topk_select_scored.argtypes = [ctypes.c_int, P, P, P, I32, P, P, I32, I32, P,
+                                                    P, P, SZ, P, P]
                 for name in EXPORTS[2:]:
-                    getattr(h, name).restype = ctypes.c_int
+                    if name != "sd_set_wait_timeout_ns":
+                        getattr(h, name).restype = ctypes.c_int
                 _LIB = h
     return _LIB
 
@@ -202,6 +211,12 @@ def _workspace(nbytes: int, device, given: Optional[torch.Tensor]):
     if given is not None:
         return given
     return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def sd_set_wait_timeout_ns(ns: int) -> int:
+    """Bound of the waits inside the tensor-core kernels (0 restores 1 s); returns the previous
+    bound."""
+    return int(lib().sd_set_wait_timeout_ns(int(ns)))
 
 
 def sd_attention_workspace_size(kind: int, q: Queries, kv: KVCache) -> int:
@@ -324,6 +339,35 @@ def sd_topk_select(q: Queries, kv: KVCache, cand_begin, cand_end, max_cand: int,
             ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(cand_begin),
             _ptr(cand_end), int(max_cand), int(k), _ptr(idx_out), _ptr(ws), ws.numel(),
             _ptr(dev_err), _stream(stream)), "sd_topk_select")
+    return idx_out
+
+
+def sd_topk_scored_workspace_size(mode: int, q: Queries, kv: KVCache, max_cand: int,
+                                  k: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().sd_topk_scored_workspace_size(int(mode), ctypes.byref(q.desc),
+                                               ctypes.byref(kv.desc), kv.batch, int(max_cand),
+                                               int(k), ctypes.byref(n)),
+           "sd_topk_scored_workspace_size")
+    return n.value
+
+
+def sd_topk_select_scored(mode: int, q: Queries, kv: KVCache, cand_begin, cand_end,
+                          max_cand: int, k: int, idx_out=None, scores_out=None, workspace=None,
+                          dev_err=None, stream=None) -> torch.Tensor:
+    """Top-K with a score mode: SD_TOPK_LAST_QUERY (as sd_topk_select) or
+    SD_TOPK_MEAN_TEXT_ATTENTION (q holds the prefill text rows).  scores_out: optional float64
+    [batch][h_kv][max_cand] tensor that receives every candidate's score."""
+    if idx_out is None:
+        idx_out = torch.empty((kv.batch, kv.h_kv, int(k)), dtype=torch.int32, device=q.q.device)
+    ws = _workspace(sd_topk_scored_workspace_size(mode, q, kv, max_cand, k), q.q.device,
+                    workspace)
+    with _on(q.q):
+        _check(lib().sd_topk_select_scored(
+            int(mode), ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch,
+            _ptr(cand_begin), _ptr(cand_end), int(max_cand), int(k), _ptr(idx_out),
+            _ptr(scores_out), _ptr(ws), ws.numel(), _ptr(dev_err), _stream(stream)),
+            "sd_topk_select_scored")
     return idx_out
 
 

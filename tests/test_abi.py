@@ -140,3 +140,33 @@ def test_workspace_sizes_scale_with_the_problem():
     _, kv = _descs()
     assert lib.sd_topk_workspace_size(ctypes.byref(kv), 28, 25000, 1024, ctypes.byref(n1)) == 0
     assert n1.value == 28 * 4 * 25000 * 8
+
+
+def test_topk_scored_validation():
+    q, kv = _descs(max_q=64, max_kv=4096)
+    lib = sd.lib()
+    n = ctypes.c_size_t(0)
+    assert lib.sd_topk_scored_workspace_size(7, ctypes.byref(q), ctypes.byref(kv), 2, 4000, 64,
+                                             ctypes.byref(n)) == sd.SD_ERR_INVALID_ARG
+    assert lib.sd_topk_scored_workspace_size(sd.SD_TOPK_MEAN_TEXT_ATTENTION, ctypes.byref(q),
+                                             ctypes.byref(kv), 2, 4000, 64,
+                                             ctypes.byref(n)) == sd.SD_OK
+    keys = 2 * 4 * 4000 * 8
+    assert n.value >= keys + 2 * 64 * 28 * 4
+    call = lambda mode, ws, nbytes: lib.sd_topk_select_scored(
+        mode, ctypes.byref(q), FAKE, ctypes.byref(kv), 2, FAKE, FAKE, 4000, 64, FAKE, None, ws,
+        nbytes, None, None)
+    assert call(5, FAKE, n.value) == sd.SD_ERR_INVALID_ARG
+    assert call(sd.SD_TOPK_MEAN_TEXT_ATTENTION, FAKE, n.value - 1) == sd.SD_ERR_WORKSPACE
+    assert call(sd.SD_TOPK_MEAN_TEXT_ATTENTION, ctypes.c_void_p(0x7f0000001010),
+                n.value) == sd.SD_ERR_WORKSPACE  # not 256-byte aligned
+    assert call(sd.SD_TOPK_MEAN_TEXT_ATTENTION, None, n.value) == sd.SD_ERR_WORKSPACE
+
+
+def test_wait_timeout_setting_round_trips():
+    lib = sd.lib()
+    prev = sd.sd_set_wait_timeout_ns(5000)
+    assert prev == 10**9  # the default bound of 1 s
+    assert sd.sd_set_wait_timeout_ns(0) == 5000   # 0 restores the default ...
+    assert sd.sd_set_wait_timeout_ns(0) == 10**9  # ... which is what is now set
+    assert lib.sd_version() >= 200
