@@ -496,6 +496,53 @@ def plain_decoding(cyc, torch, reps):
     return res
 
 
+def long_context(torch, sd, flusher, peak, l_vis=140_000, layers=28, topk=1024, reps=3):
+    """The path at an hour of video: 28 layers x 140,000 visual + 1,024 text positions (8.1 GB
+    of KV, drawn on the device), each call timed with L2 flushed before it."""
+    from speculative_decoding_attention_verify_b200 import inputs as gen
+    L, g = layers, 8
+    t = gen.make_device_workload(layers, l_vis, 1024, g)
+    dvc = t["k"].device
+    i32 = lambda a: torch.tensor(a, dtype=torch.int32, device=dvc)
+    ctx = l_vis + 1024
+    kv = lambda n: sd.KVCache(t["k"], t["v"], i32([n] * L))
+    kv_verify, kv_draft = kv(ctx + g + 1), kv(ctx + 1)
+    qv = sd.Queries(t["q_verify"], i32(list(range(0, L * (g + 1) + 1, g + 1))), g + 1, ctx + g + 1)
+    qd = sd.Queries(t["q_draft"], i32(list(range(L + 1))), 1, ctx + 1)
+    row = 4 * 128 * 2 * 2
+    cb, ce, tail = i32([0] * L), i32([l_vis] * L), i32([l_vis] * L)
+    idx = sd.sd_topk_select(qv, kv_verify, cb, ce, l_vis, topk)
+    sel = sd.sd_sparse_stage(kv_draft, idx, tail)
+    vb, ve, win = i32([0] * L), i32([l_vis] * L), i32([1024] * L)
+    outs = {}
+    calls = {
+        "verify": (lambda s: sd.sd_verify_attention(qv, kv_verify, stream=s),
+                   L * (ctx + g + 1) * row + 2 * L * (g + 1) * 28 * 128 * 2),
+        "decode": (lambda s: sd.sd_verify_attention(qd, kv_draft, stream=s),
+                   L * (ctx + 1) * row + 2 * L * 28 * 128 * 2),
+        "topk": (lambda s: sd.sd_topk_select(qv, kv_verify, cb, ce, l_vis, topk, idx_out=idx,
+                                             stream=s),
+                 L * l_vis * 4 * 128 * 2 + L * 28 * 128 * 2 + L * 4 * topk * 4),
+        "sparse": (lambda s: sd.sd_sparse_attention_staged(qd, kv_draft, sel, topk, tail, 1025,
+                                                           stream=s),
+                   L * (topk + 1025) * row + L * 4 * topk * 4 + 2 * L * 28 * 128 * 2),
+        "text_anchored": (lambda s: sd.sd_text_anchored_attention(qd, kv_draft, vb, ve, win,
+                                                                  1024, stream=s),
+                          L * 1024 * row + 2 * L * 28 * 128 * 2),
+    }
+    for name, (fn, byt) in calls.items():
+        fn(None)
+        ms = statistics.median(flusher.time_calls(fn, reps))
+        gbs = byt / (ms / 1e3) / 1e9
+        outs[name] = {"launch_us": round(ms * 1e3, 1), "bytes": int(byt),
+                      "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+    del t, sel, idx
+    torch.cuda.empty_cache()
+    return {"workload": f"{L} layers x ({l_vis} visual + 1024 text) positions, H_q=28, H_kv=4, "
+                        "d=128, bf16, gamma 8, top-K 1024, window 1024 (device-drawn N(0,1))",
+            "kv_bytes": int(L * (ctx + g + 1) * row), "calls": outs}
+
+
 def peak_bf16():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -804,6 +851,8 @@ def run_ours(args):
         layer_latency.append({"call": kind, "layers": 1, "launch_us": round(ms1 * 1e3, 2),
                               "bytes": b1, "achieved_gbs": round(b1 / (ms1 / 1e3) / 1e9, 1),
                               "frac": round(b1 / (ms1 / 1e3) / 1e9 / peak, 4)})
+    longctx = long_context(torch, cyc.sd, flusher, peak) \
+        if args.long_context and args.config == DEFAULT_CONFIG else None
     del flusher
     torch.cuda.empty_cache()
 
@@ -843,6 +892,7 @@ def run_ours(args):
             "layer_latency": layer_latency,
             "plain_decoding": plain,
             "prefill_selection": prefill,
+            "long_context": longctx,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": host.h2d_bytes, "d2h_bytes_per_step": host.d2h_bytes,
                     "ms_per_step": round(e2e_ms / args.steps, 4),
@@ -1071,6 +1121,8 @@ def main():
     ap.add_argument("--call-reps", type=int, default=10,
                     help="separately timed repetitions of every call for the per-call rooflines")
     ap.add_argument("--no-plain", action="store_true", help="skip the plain-decoding comparison")
+    ap.add_argument("--no-long-context", dest="long_context", action="store_false",
+                    help="skip the 140,000-position measurement")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the prefill (mean text attention) selection")
     ap.add_argument("--no-cpu-baseline", action="store_true")

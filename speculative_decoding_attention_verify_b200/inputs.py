@@ -315,6 +315,26 @@ def make_text_queries(w: AttnWorkload, seed: Optional[int] = None):
     return q, q_start
 
 
+def make_device_workload(layers: int, l_vis: int, l_txt: int, gamma: int, h_q: int = 28,
+                         h_kv: int = 4, d: int = 128, seed: int = SEED_BASE + 5, device="cuda"):
+    """bf16 caches and queries drawn directly on the device with a seeded torch generator, for
+    benchmark workloads too large to draw on the host (e.g. 28 layers x 140,000 positions):
+    K, V [layers][h_kv][l_vis + l_txt + gamma + 1][d] and verify / draft query rows, all
+    N(0, 1).  No salient keys: timing only, no oracle comparison."""
+    import torch
+    gen_ = torch.Generator(device=device)
+    gen_.manual_seed(int(seed))
+    cap = l_vis + l_txt + gamma + 1
+    draw = lambda *shape: torch.randn(*shape, generator=gen_, device=device,
+                                      dtype=torch.float32).to(torch.bfloat16)
+    k = draw(layers, h_kv, cap, d)
+    v = draw(layers, h_kv, cap, d)
+    q_verify = draw(layers * (gamma + 1), h_q, d)
+    q_draft = draw(layers, h_q, d)
+    return dict(k=k, v=v, q_verify=q_verify, q_draft=q_draft, layers=layers, l_vis=l_vis,
+                l_txt=l_txt, gamma=gamma, h_q=h_q, h_kv=h_kv, d=d, cap=cap)
+
+
 @dataclasses.dataclass
 class AcceptWorkload:
     """Logits, drafted tokens and uniforms for a batch of acceptance problems.
