@@ -318,19 +318,20 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             const int s1 = (t + 1) % S, use1 = (t + 1) / S;
             bool qk_done = t + 1 >= n_my, pv_done = false;
             const unsigned long long t0 = now_ns();
+            const uint32_t hint = poll_hint(p.wait_ns);
             for (unsigned it = 1; !(qk_done && pv_done); ++it) {
                 int flags = 0;  // bit 0: S can go, bit 1: P.V can go, bit 2: give up
                 if (lane == 0) {
-                    if (!qk_done && mbar_try(BAR(KF + s1), use1 & 1)) flags |= 1;
-                    if (!pv_done && mbar_try(BAR(PF + sb), (t >> 1) & 1) &&
-                        mbar_try(BAR(VF + s), use & 1))
+                    if (!qk_done && mbar_try_for(BAR(KF + s1), use1 & 1, hint)) flags |= 1;
+                    if (!pv_done && mbar_try_for(BAR(PF + sb), (t >> 1) & 1, hint) &&
+                        mbar_try_for(BAR(VF + s), use & 1, hint))
                         flags |= 2;
-                    if (flags == 0 && (it & 63u) == 0) {
-                        if (*abort_flag) {
-                            flags = 4;
-                        } else if (now_ns() - t0 > p.wait_ns) {
+                    if (flags == 0) {
+                        if (now_ns() - t0 > p.wait_ns) {
                             *abort_flag = 1;
                             set_dev_err(p.dev_err, SD_DEVERR_TIMEOUT);
+                            flags = 4;
+                        } else if ((it & 7u) == 0 && *abort_flag) {
                             flags = 4;
                         }
                     }
@@ -743,6 +744,8 @@ cudaError_t launch_attention_tc(const AttnParams &p, const AttnPlan &plan, cudaS
     TcMaps maps;
     if (!encode_kv_maps(p, p.max_kv_len, &maps)) return cudaErrorNotSupported;
     (void)plan;
+    if (narrow_supported(p.kv.head_dim, p.group, p.max_q_rows))
+        return launch_attention_narrow(p, maps, s);
     const bool paged = p.kv.page_size != 0;
     // row copies: four when the planned rows per KV head fit in 32 (the draft steps), two when
     // they fit in 64 (verification of up to 9 rows x 7 heads)

@@ -24,6 +24,11 @@ struct TcMaps {
 // engine).
 bool encode_kv_maps(const AttnParams &p, int max_kv_len, TcMaps *maps);
 
+// The narrow-row tensor-core engine (one query row, at most 16 query heads per KV head,
+// head_dim 128): the products taken transposed so that positions fill the MMA's M dimension.
+bool narrow_supported(int head_dim, int group, int max_q_rows);
+cudaError_t launch_attention_narrow(const AttnParams &p, const TcMaps &maps, cudaStream_t s);
+
 namespace tc {
 
 // Bound of the drains after an abort (a CTA waiting for its own copies and MMAs to finish):
@@ -67,24 +72,46 @@ __device__ __forceinline__ unsigned long long now_ns() {
     return t;
 }
 
+// Longest suspension of one poll of an mbarrier (ns): a thread waiting on a phase sleeps at
+// most this long before it looks at the clock and the abort flag again.
+constexpr uint32_t kPollNs = 20000;
+
+// One poll that may suspend the thread up to hint_ns (or until the phase completes).
+__device__ __forceinline__ bool mbar_try_for(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// The suspension hint of the polls of a wait bounded by limit_ns.
+__device__ __forceinline__ uint32_t poll_hint(unsigned long long limit_ns) {
+    return limit_ns < kPollNs ? (uint32_t)limit_ns : kPollNs;
+}
+
 // Bounded wait (limit_ns) for the phase of `bar` with the given parity.  Returns false when
-// the CTA is aborting (this wait timed out, or another one did).
+// the CTA is aborting (this wait timed out, or another one did).  Each poll suspends at most
+// min(limit_ns, kPollNs), so a short bound is honoured however slow the awaited copy is.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                           int32_t *dev_err, unsigned long long limit_ns) {
-    if (mbar_try(bar, parity)) return true;
+    const uint32_t hint = poll_hint(limit_ns);
+    if (mbar_try_for(bar, parity, hint)) return true;
     const unsigned long long t0 = now_ns();
     for (unsigned it = 1;; ++it) {
-        if (mbar_try(bar, parity)) return true;
-        // the abort flag and the clock are checked every 64 polls: a shared-memory load can
-        // take thousands of cycles while the tensor core and the copy engine stream
-        if ((it & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (now_ns() - t0 > limit_ns) {
-                *abort_flag = 1;
-                set_dev_err(dev_err, SD_DEVERR_TIMEOUT);
-                return false;
-            }
+        if (mbar_try_for(bar, parity, hint)) return true;
+        if (now_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            set_dev_err(dev_err, SD_DEVERR_TIMEOUT);
+            return false;
         }
+        // the abort flag every 8 polls: a shared-memory load can take thousands of cycles while
+        // the tensor core and the copy engine stream
+        if ((it & 7u) == 0 && *abort_flag) return false;
     }
 }
 
@@ -126,6 +153,14 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t addr, uint32_t lbo) {
 __host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
            ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// kind::f16 instruction descriptor with both operand majors given: fp32 accumulate, bf16 A and
+// B, M = 128, N = n (a multiple of 16); a_mn / b_mn select MN-major (transposed) operands.
+__host__ __device__ constexpr uint32_t idesc_bf16_ab(int n, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(128 >> 4) << 24);
 }
 
 // D (TMEM) += A (TMEM, M x 16, packed bf16 pairs along K) * B (shared memory descriptor);
@@ -193,6 +228,37 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
         "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
         "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane, load and wait in one statement.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 fp32 columns to this thread's TMEM lane, store and wait in one statement.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15]))
         : "memory");
 }
 

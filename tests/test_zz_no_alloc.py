@@ -68,8 +68,9 @@ def test_noalloc_matches_oracle():
 def test_noalloc_rejects_a_plan_beyond_its_scratch():
     w = gen.make_attn_workload(3, l_vis=3000, l_txt=100)
     kv, q = dev.kv_cache(w), dev.verify_queries(w)
-    # Same tensors; a looser row hint (18 rows per sequence) plans a workspace of about 66 MB.
-    big = sd.Queries(q.q, q.q_start, max_q_rows=18, max_kv_len=int(w.kv_len_verify.max()))
+    # Same tensors; a much looser length hint (up to 2,000,000 positions) plans more splits
+    # and a workspace of about 129 MiB.
+    big = sd.Queries(q.q, q.q_start, max_q_rows=q.desc.max_q_rows, max_kv_len=2_000_000)
     assert sd.sd_attention_workspace_size(sd.SD_ATTN_VERIFY, big, kv) > \
         sd.SD_VERIFY_NOALLOC_SCRATCH_BYTES
     out = torch.zeros_like(q.q)
