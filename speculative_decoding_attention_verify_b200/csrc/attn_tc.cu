@@ -744,8 +744,6 @@ cudaError_t launch_attention_tc(const AttnParams &p, const AttnPlan &plan, cudaS
     TcMaps maps;
     if (!encode_kv_maps(p, p.max_kv_len, &maps)) return cudaErrorNotSupported;
     (void)plan;
-    if (narrow_supported(p.kv.head_dim, p.group, p.max_q_rows))
-        return launch_attention_narrow(p, maps, s);
     const bool paged = p.kv.page_size != 0;
     // row copies: four when the planned rows per KV head fit in 32 (the draft steps), two when
     // they fit in 64 (verification of up to 9 rows x 7 heads)
