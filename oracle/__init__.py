@@ -57,12 +57,15 @@ def configure(handle):
     handle.orc_hsr_project.argtypes = [vp, vp, i32, i32, vp, vp, vp]
     handle.orc_accept_greedy.argtypes = [vp, vp, vp, i32, i32, vp, vp, i32]
     handle.orc_accept_sample.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp]
+    handle.orc_rmsnorm_rows.argtypes = [vp, i32, i32, vp, ctypes.c_double, vp]
+    handle.orc_rope_rows.argtypes = [vp, i32, i32, vp, ctypes.c_double]
+    handle.orc_draft_layer.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp]
     handle.orc_set_threads.argtypes = [i32]
     for name in ("orc_verify_attention", "orc_decode_attention", "orc_text_anchored_attention",
                  "orc_sparse_attention", "orc_topk_select", "orc_topk_scores",
                  "orc_topk_attention_scores", "orc_topk_select_attention",
                  "orc_hsr_project", "orc_accept_greedy", "orc_accept_sample",
-                 "orc_set_threads"):
+                 "orc_rmsnorm_rows", "orc_rope_rows", "orc_draft_layer", "orc_set_threads"):
         getattr(handle, name).restype = ctypes.c_int
     return handle
 
@@ -250,6 +253,63 @@ def hsr_project(emb, hid, weight, bias=None):
     rc = lib().orc_hsr_project(_ptr(e), _ptr(h), n, D, _ptr(w), _ptr(b), _ptr(y))
     _check(rc, "hsr_project")
     return y
+
+
+def rmsnorm(x, gamma, eps: float):
+    """Row-wise RMSNorm of float64 x [rows][n] with bf16 gamma [n]; returns float64."""
+    xx = _c(np.atleast_2d(x), np.float64)
+    gm = _c(gamma, np.uint16)
+    y = np.zeros_like(xx)
+    _check(lib().orc_rmsnorm_rows(_ptr(xx), xx.shape[0], xx.shape[1], _ptr(gm), float(eps),
+                                  _ptr(y)), "rmsnorm")
+    return y
+
+
+def rope(v, pos, theta: float):
+    """Rotary embedding (rotate-half pairs) of float64 rows v [rows][d] at positions pos [rows];
+    returns a new float64 array."""
+    vv = np.array(np.atleast_2d(v), dtype=np.float64, order="C")
+    pp = _c(pos, np.float64)
+    _check(lib().orc_rope_rows(_ptr(vv), vv.shape[0], vv.shape[1], _ptr(pp), float(theta)),
+           "rope")
+    return vv
+
+
+class _DraftWeights(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int32), ("h_q", ctypes.c_int32), ("h_kv", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("d_ff", ctypes.c_int32),
+                ("rms_eps", ctypes.c_double), ("rope_theta", ctypes.c_double),
+                ("w_hsr", ctypes.c_void_p), ("ln1", ctypes.c_void_p), ("w_qkv", ctypes.c_void_p),
+                ("b_qkv", ctypes.c_void_p), ("w_o", ctypes.c_void_p), ("ln2", ctypes.c_void_p),
+                ("w_gate_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p)]
+
+
+def draft_layer(wt, emb, hid, k_cache, v_cache, kv_len: int, window: int):
+    """One draft layer for the rows of emb / hid [n][D] (bf16 bits), the last n positions of a
+    one-sequence cache k_cache / v_cache [1][h_kv][cap][d] (bf16 bits, copied: the rows' k and v
+    are written into the copies).  wt: an object with the fields of the weights (bf16 bits) and
+    shapes.  Returns (y [n][D] float64, k copy, v copy, inter dict of x, q, o, x2)."""
+    n, D = emb.shape
+    k = np.array(k_cache, dtype=np.uint16, order="C")
+    v = np.array(v_cache, dtype=np.uint16, order="C")
+    cache = Cache(BF16, k, v, [kv_len], wt.h_kv, wt.head_dim)
+    keep = {name: _c(getattr(wt, name), np.uint16) if getattr(wt, name) is not None else None
+            for name in ("w_hsr", "ln1", "w_qkv", "b_qkv", "w_o", "ln2", "w_gate_up", "w_down")}
+    s = _DraftWeights()
+    s.d_model, s.h_q, s.h_kv, s.head_dim, s.d_ff = D, wt.h_q, wt.h_kv, wt.head_dim, wt.d_ff
+    s.rms_eps, s.rope_theta = float(wt.rms_eps), float(wt.rope_theta)
+    for name, arr in keep.items():
+        setattr(s, name, None if arr is None else arr.ctypes.data)
+    e, h = _c(emb, np.uint16), _c(hid, np.uint16)
+    y = np.zeros((n, D), dtype=np.float64)
+    hd = wt.h_q * wt.head_dim
+    inter = np.zeros((n, 2 * D + 2 * hd), dtype=np.float64)
+    rc = lib().orc_draft_layer(ctypes.byref(s), _ptr(e), _ptr(h), n, ctypes.byref(cache.struct),
+                               int(window), _ptr(y), _ptr(inter))
+    _check(rc, "draft_layer")
+    parts = {"x": inter[:, :D], "q": inter[:, D:D + hd], "o": inter[:, D + hd:D + 2 * hd],
+             "x2": inter[:, D + 2 * hd:]}
+    return y, cache.k, cache.v, parts
 
 
 def accept_greedy(tgt, draft_tokens, gamma, vocab: int, out_stride: Optional[int] = None):

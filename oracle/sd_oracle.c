@@ -577,6 +577,165 @@ int orc_hsr_project(const uint16_t *emb, const uint16_t *hid, int n, int d_model
     return ORC_OK;
 }
 
+/* ---------------------------------------------------------------- draft layer ----------- */
+
+/* Sparrow's draft layer [SPW 3.1 HSR-VATA: the draft takes an FC over [text embedding ; reused
+ * target hidden state] and attends only to text-anchored positions].  The pages name no layer
+ * internals; the reading taken is one pre-norm decoder layer of the target's shapes:
+ *   x  = W_hsr [e ; h]
+ *   a  = RMSNorm(x) * ln1,       [q ; k ; v] = W_qkv a + b_qkv
+ *   q, k rotated by RoPE at the row's position (rotate-half pairs (i, i + d/2),
+ *        angle = pos * theta^(-2i/d))
+ *   k, v stored in the draft's own cache at the row's position (the cache's bf16 type), q
+ *        rounded to bf16 (the attention call's query type)
+ *   o  = text-anchored attention of the rows over the cache (window W, no visual span)
+ *   x2 = x + W_o o
+ *   m  = RMSNorm(x2) * ln2,      y = x2 + W_down (silu(W_gate m) * (W_up m))
+ * with RMSNorm(x)_i = x_i / sqrt(mean_j x_j^2 + eps) and silu(t) = t / (1 + exp(-t)).  All
+ * arithmetic in double; weights and caches are bf16 bits. */
+
+static void orc_rmsnorm(const double *x, int n, const uint16_t *gamma, double eps, double *y)
+{
+    double ss = 0.0;
+    for (int i = 0; i < n; ++i)
+        ss += x[i] * x[i];
+    double r = 1.0 / sqrt(ss / (double)n + eps);
+    for (int i = 0; i < n; ++i)
+        y[i] = x[i] * r * orc_widen(gamma, ORC_BF16, i);
+}
+
+static void orc_rope(double *v, int d, double pos, double theta)
+{
+    int half = d / 2;
+    for (int i = 0; i < half; ++i) {
+        double ang = pos * pow(theta, -2.0 * (double)i / (double)d);
+        double c = cos(ang), s = sin(ang);
+        double a = v[i], b = v[i + half];
+        v[i] = a * c - b * s;
+        v[i + half] = b * c + a * s;
+    }
+}
+
+/* y[o] = sum_i W[o][i] x[i] (+ bias[o]); W bf16 [m][k] row-major. */
+static void orc_linear(const uint16_t *W, const uint16_t *bias, const double *x, int64_t m,
+                       int64_t k, double *y)
+{
+    for (int64_t o = 0; o < m; ++o) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < k; ++i)
+            acc += orc_widen(W, ORC_BF16, o * k + i) * x[i];
+        if (bias)
+            acc += orc_widen(bias, ORC_BF16, o);
+        y[o] = acc;
+    }
+}
+
+/* Nearest bf16 (ties to even) of a double, through float. */
+static uint16_t orc_to_bf16(double x)
+{
+    float f = (float)x;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+int orc_rmsnorm_rows(const double *x, int rows, int n, const uint16_t *gamma, double eps,
+                     double *y)
+{
+    for (int r = 0; r < rows; ++r)
+        orc_rmsnorm(x + (int64_t)r * n, n, gamma, eps, y + (int64_t)r * n);
+    return ORC_OK;
+}
+
+int orc_rope_rows(double *v, int rows, int d, const double *pos, double theta)
+{
+    for (int r = 0; r < rows; ++r)
+        orc_rope(v + (int64_t)r * d, d, pos[r], theta);
+    return ORC_OK;
+}
+
+/* The n rows are the last n positions of the cache (row r at position kv_len - n + r); the
+ * caller's cache arrays receive the rows' k and v.  inter (may be NULL) receives, per row,
+ * x [D], q [h_q d] (after RoPE, before rounding), o [h_q d], x2 [D] (in that order). */
+int orc_draft_layer(const orc_draft_weights *w, const uint16_t *emb, const uint16_t *hid, int n,
+                    const orc_cache *c, int window, double *y, double *inter)
+{
+    const int D = w->d_model, d = w->head_dim, hq = w->h_q, hk = w->h_kv, F = w->d_ff;
+    const int nqkv = (hq + 2 * hk) * d;
+    if (n < 1 || c->h_kv != hk || c->head_dim != d || c->dtype != ORC_BF16 || hq % hk)
+        return ORC_ERR_ARG;
+    const int64_t kv_len = c->kv_len[0];
+    if (kv_len < n || window < 1)
+        return ORC_ERR_ARG;
+    double *x = malloc(sizeof(double) * (size_t)n * D);
+    double *a = malloc(sizeof(double) * (size_t)D);
+    double *qkv = malloc(sizeof(double) * (size_t)nqkv);
+    double *q = malloc(sizeof(double) * (size_t)n * hq * d);
+    uint16_t *qb = malloc(sizeof(uint16_t) * (size_t)n * hq * d);
+    double *o = malloc(sizeof(double) * (size_t)n * hq * d);
+    double *x2 = malloc(sizeof(double) * (size_t)D);
+    double *gu = malloc(sizeof(double) * (size_t)2 * F);
+    double *sv = malloc(sizeof(double) * (size_t)F);
+    double *cat = malloc(sizeof(double) * (size_t)2 * D);
+    uint16_t *kc = (uint16_t *)c->k, *vc = (uint16_t *)c->v;
+    int err = ORC_OK;
+    for (int r = 0; r < n; ++r) {
+        for (int i = 0; i < D; ++i) {
+            cat[i] = orc_widen(emb, ORC_BF16, (int64_t)r * D + i);
+            cat[D + i] = orc_widen(hid, ORC_BF16, (int64_t)r * D + i);
+        }
+        orc_linear(w->w_hsr, NULL, cat, D, 2 * D, x + (int64_t)r * D);
+        orc_rmsnorm(x + (int64_t)r * D, D, w->ln1, w->rms_eps, a);
+        orc_linear(w->w_qkv, w->b_qkv, a, nqkv, D, qkv);
+        const int64_t pos = kv_len - n + r;
+        for (int h = 0; h < hq + hk; ++h)
+            orc_rope(qkv + (int64_t)h * d, d, (double)pos, w->rope_theta);
+        for (int i = 0; i < hq * d; ++i) {
+            q[(int64_t)r * hq * d + i] = qkv[i];
+            qb[(int64_t)r * hq * d + i] = orc_to_bf16(qkv[i]);
+        }
+        for (int g = 0; g < hk; ++g) {
+            int64_t row = orc_kv_row(c, 0, g, pos);
+            if (row < 0) {
+                err = ORC_ERR_ARG;
+                continue;
+            }
+            for (int e = 0; e < d; ++e) {
+                kc[row + e] = orc_to_bf16(qkv[(int64_t)(hq + g) * d + e]);
+                vc[row + e] = orc_to_bf16(qkv[(int64_t)(hq + hk + g) * d + e]);
+            }
+        }
+    }
+    if (err == ORC_OK) {
+        int32_t qs[2] = {0, n}, vb = 0, ve = 0, win = window;
+        orc_query qd = {hq, 0.0, qs};
+        err = orc_text_anchored_attention(&qd, qb, c, 1, &vb, &ve, &win, o);
+    }
+    for (int r = 0; err == ORC_OK && r < n; ++r) {
+        orc_linear(w->w_o, NULL, o + (int64_t)r * hq * d, D, (int64_t)hq * d, x2);
+        for (int i = 0; i < D; ++i)
+            x2[i] += x[(int64_t)r * D + i];
+        orc_rmsnorm(x2, D, w->ln2, w->rms_eps, a);
+        orc_linear(w->w_gate_up, NULL, a, 2 * (int64_t)F, D, gu);
+        for (int i = 0; i < F; ++i)
+            sv[i] = gu[i] / (1.0 + exp(-gu[i])) * gu[F + i];
+        orc_linear(w->w_down, NULL, sv, D, F, y + (int64_t)r * D);
+        for (int i = 0; i < D; ++i)
+            y[(int64_t)r * D + i] += x2[i];
+        if (inter) {
+            double *dst = inter + (int64_t)r * (2 * D + 2 * hq * d);
+            memcpy(dst, x + (int64_t)r * D, sizeof(double) * (size_t)D);
+            memcpy(dst + D, q + (int64_t)r * hq * d, sizeof(double) * (size_t)hq * d);
+            memcpy(dst + D + hq * d, o + (int64_t)r * hq * d, sizeof(double) * (size_t)hq * d);
+            memcpy(dst + D + 2 * hq * d, x2, sizeof(double) * (size_t)D);
+        }
+    }
+    free(x); free(a); free(qkv); free(q); free(qb); free(o); free(x2); free(gu); free(sv);
+    free(cat);
+    return err;
+}
+
 /* ---------------------------------------------------------------- acceptance ------------- */
 
 /* Index of the largest entry; equal values go to the lower index; NaN ranks below -inf. */

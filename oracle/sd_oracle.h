@@ -67,6 +67,25 @@ int orc_accept_sample(const float *tgt, const float *drf, const int32_t *draft, 
                       const float *v, const int32_t *gamma, int batch, int vocab, int32_t *n_acc,
                       int32_t *out_tok, int out_stride, double *accept_margin,
                       double *draw_margin);
+/* Weights of one draft layer (all bf16 bits; b_qkv may be NULL). */
+typedef struct {
+    int32_t d_model, h_q, h_kv, head_dim, d_ff;
+    double rms_eps, rope_theta;
+    const uint16_t *w_hsr;     /* [d_model][2 d_model] */
+    const uint16_t *ln1;       /* [d_model] */
+    const uint16_t *w_qkv;     /* [(h_q + 2 h_kv) head_dim][d_model] */
+    const uint16_t *b_qkv;     /* [(h_q + 2 h_kv) head_dim] */
+    const uint16_t *w_o;       /* [d_model][h_q head_dim] */
+    const uint16_t *ln2;       /* [d_model] */
+    const uint16_t *w_gate_up; /* [2 d_ff][d_model]: the gate rows, then the up rows */
+    const uint16_t *w_down;    /* [d_model][d_ff] */
+} orc_draft_weights;
+
+int orc_rmsnorm_rows(const double *x, int rows, int n, const uint16_t *gamma, double eps,
+                     double *y);
+int orc_rope_rows(double *v, int rows, int d, const double *pos, double theta);
+int orc_draft_layer(const orc_draft_weights *w, const uint16_t *emb, const uint16_t *hid, int n,
+                    const orc_cache *c, int window, double *y, double *inter);
 int orc_set_threads(int n);
 
 #ifdef __cplusplus

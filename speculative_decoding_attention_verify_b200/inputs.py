@@ -336,6 +336,76 @@ def make_device_workload(layers: int, l_vis: int, l_txt: int, gamma: int, h_q: i
 
 
 @dataclasses.dataclass
+class DraftLayerWorkload:
+    """Weights and inputs of one draft layer (all bf16 bits): the HSR FC, two RMSNorm weights,
+    the QKV projection with bias, the output projection, the gate/up and down projections;
+    the rows' embeddings and reused hidden states; the draft's own text-only KV cache
+    [1][h_kv][cap][d] whose last n positions are the rows' (their k, v are written there)."""
+
+    n: int
+    d_model: int
+    h_q: int
+    h_kv: int
+    head_dim: int
+    d_ff: int
+    rms_eps: float
+    rope_theta: float
+    l_txt: int
+    window: int
+    w_hsr: np.ndarray
+    ln1: np.ndarray
+    w_qkv: np.ndarray
+    b_qkv: np.ndarray
+    w_o: np.ndarray
+    ln2: np.ndarray
+    w_gate_up: np.ndarray
+    w_down: np.ndarray
+    emb: np.ndarray
+    hid: np.ndarray
+    k_cache: np.ndarray
+    v_cache: np.ndarray
+
+    @property
+    def kv_len(self) -> int:
+        return self.l_txt + self.n
+
+
+def make_draft_layer_workload(n: int = 1, d_model: int = HSR_D_MODEL, h_q: int = 28,
+                              h_kv: int = 4, head_dim: int = 128, d_ff: int = 18944,
+                              l_txt: int = 1024, window: Optional[int] = None,
+                              seed: Optional[int] = None) -> DraftLayerWorkload:
+    """Random weights of the 7B-like shapes by default (N(0, 1/fan_in) matrices, RMSNorm weights
+    1 + N(0, 0.1^2), QKV bias N(0, 0.1^2)), N(0, 1) embeddings, hidden states and cache rows;
+    the cache holds l_txt earlier text positions and room for the n new rows."""
+    rng = np.random.Generator(np.random.PCG64(SEED_BASE + 9 + 800_000 if seed is None else seed))
+    D, F, d = d_model, d_ff, head_dim
+    nqkv = (h_q + 2 * h_kv) * d
+    mat = lambda m, k: bf16_bits_from_f32(rng.standard_normal((m, k), dtype=np.float32) *
+                                          np.float32(1.0 / np.sqrt(k)))
+    vec = lambda m, mu, sd: bf16_bits_from_f32(
+        (mu + sd * rng.standard_normal(m)).astype(np.float32))
+    w_hsr = mat(D, 2 * D)
+    ln1 = vec(D, 1.0, 0.1)
+    w_qkv = mat(nqkv, D)
+    b_qkv = vec(nqkv, 0.0, 0.1)
+    w_o = mat(D, h_q * d)
+    ln2 = vec(D, 1.0, 0.1)
+    w_gate_up = mat(2 * F, D)
+    w_down = mat(D, F)
+    emb = bf16_bits_from_f32(rng.standard_normal((n, D), dtype=np.float32))
+    hid = bf16_bits_from_f32(rng.standard_normal((n, D), dtype=np.float32))
+    cap = l_txt + n
+    k_cache = bf16_bits_from_f32(rng.standard_normal((1, h_kv, cap, d), dtype=np.float32))
+    v_cache = bf16_bits_from_f32(rng.standard_normal((1, h_kv, cap, d), dtype=np.float32))
+    return DraftLayerWorkload(n=n, d_model=D, h_q=h_q, h_kv=h_kv, head_dim=d, d_ff=F,
+                              rms_eps=1e-6, rope_theta=1e6, l_txt=l_txt,
+                              window=l_txt if window is None else window, w_hsr=w_hsr, ln1=ln1,
+                              w_qkv=w_qkv, b_qkv=b_qkv, w_o=w_o, ln2=ln2, w_gate_up=w_gate_up,
+                              w_down=w_down, emb=emb, hid=hid, k_cache=k_cache,
+                              v_cache=v_cache)
+
+
+@dataclasses.dataclass
 class AcceptWorkload:
     """Logits, drafted tokens and uniforms for a batch of acceptance problems.
 

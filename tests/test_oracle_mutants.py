@@ -15,6 +15,7 @@ import oracle
 from oracle import build as obuild
 
 from . import test_oracle_accept as ta
+from . import test_oracle_draft_layer as tdl
 from . import test_oracle_attention as tt
 from . import test_oracle_text_attention as tx
 from . import test_oracle_topk_hsr as tk
@@ -32,6 +33,12 @@ TEXT_ATTN = [tx.test_golden_text_attention_tiny, lambda: tx.test_scores_over_eve
              lambda: tx.test_scores_equal_mean_attention_output_with_one_hot_values(1, 3),
              tx.test_zero_keys_give_uniform_weights_closed_form,
              tx.test_candidates_beyond_a_rows_causal_limit_get_only_the_later_rows]
+DRAFT = [tdl.test_rmsnorm_matches_torch_fp64, tdl.test_rope_equals_complex_rotation,
+         tdl.test_layer_input_is_the_hsr_projection_and_zero_projections_pass_it_through,
+         tdl.test_layer_attention_is_the_text_anchored_attention_over_the_appended_cache,
+         tdl.test_layer_with_zero_norm_weights_has_closed_forms,
+         tdl.test_layer_with_zero_input_norm_projects_the_bias_rotated_at_the_row_positions,
+         tdl.test_layer_mlp_half_matches_torch_fp64]
 GREEDY = [ta.test_golden_accept_greedy_tiny, ta.test_greedy_argmax_ties_nan_and_signed_zero,
           ta.test_greedy_own_argmax_accepts_everything]
 SAMPLE = [ta.test_golden_accept_sample_tiny,
@@ -63,6 +70,22 @@ MUTANTS = {
     "text_attention_unscaled": ("s[j] = scale * dot;", "s[j] = dot;", TEXT_ATTN),
     "text_attention_denominator_from_candidates": ("for (int64_t j = 0; j <= limit; ++j)\n                    den += exp(s[j] - m);",
                                                    "for (int64_t j = cb; j <= limit && j < ce; ++j)\n                    den += exp(s[j] - m);", TEXT_ATTN),
+    "rope_rotation_sign": ("v[i] = a * c - b * s;", "v[i] = a * c + b * s;", DRAFT),
+    "rope_frequency_exponent": ("pow(theta, -2.0 * (double)i / (double)d)",
+                                "pow(theta, -1.0 * (double)i / (double)d)", DRAFT),
+    "rmsnorm_sum_not_mean": ("1.0 / sqrt(ss / (double)n + eps)", "1.0 / sqrt(ss + eps)", DRAFT),
+    "draft_attention_residual_missing": ("            x2[i] += x[(int64_t)r * D + i];\n",
+                                         "            x2[i] += 0.0;\n", DRAFT),
+    "draft_silu_as_sigmoid": ("sv[i] = gu[i] / (1.0 + exp(-gu[i])) * gu[F + i];",
+                              "sv[i] = 1.0 / (1.0 + exp(-gu[i])) * gu[F + i];", DRAFT),
+    "draft_gate_up_swapped": ("sv[i] = gu[i] / (1.0 + exp(-gu[i])) * gu[F + i];",
+                              "sv[i] = gu[F + i] / (1.0 + exp(-gu[F + i])) * gu[i];", DRAFT),
+    "draft_rope_position_one_late": ("orc_rope(qkv + (int64_t)h * d, d, (double)pos, w->rope_theta);",
+                                     "orc_rope(qkv + (int64_t)h * d, d, (double)(pos + 1), w->rope_theta);", DRAFT),
+    "draft_keys_not_rotated": ("for (int h = 0; h < hq + hk; ++h)\n            orc_rope(",
+                               "for (int h = 0; h < hq; ++h)\n            orc_rope(", DRAFT),
+    "draft_mlp_residual_from_x": ("            y[(int64_t)r * D + i] += x2[i];",
+                                  "            y[(int64_t)r * D + i] += x[(int64_t)r * D + i];", DRAFT),
     "hsr_hidden_reads_first_half": ("o * 2 * D + D + i", "o * 2 * D + i", HSR),
     "argmax_ties_to_higher": ("if (isnan(z[best]) || z[x] > z[best])", "if (isnan(z[best]) || z[x] >= z[best])", GREEDY),
     "greedy_bonus_from_draft": ("out_tok[(int64_t)b * out_stride + n] = (int32_t)t_n;",
