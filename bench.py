@@ -604,8 +604,64 @@ def plain_decoding(cyc, torch, reps):
             "speedup_at_n": {str(n): round((n + 1) * t_dec / t_cyc, 3) for n in range(g + 1)},
             "break_even_n": next((n for n in range(g + 1) if (n + 1) * t_dec >= t_cyc), None)}
         del gc
+    if sp["ta"] and sp["hsr"] and cyc.w.dtype == "bf16" and cyc.w.d == 128:
+        dl = DraftLayerSteps(cyc)
+        kinds = ("verify", "accept_greedy")
+        gc = capture(torch, lambda s: ([f(s) for f in dl.calls] + [cyc.step(s, 0, kinds)]))
+        t_cyc = time_graph(torch, gc, reps)
+        gl = capture(torch, lambda s: [f(s) for f in dl.calls])
+        t_layer = time_graph(torch, gl, reps) / g
+        byt = dl.bytes_per_call * g + sum(cyc.call_bytes(k, st) for k, st, _ in cyc.calls
+                                          if k in kinds)
+        methods["sparrow_draft_layer"] = {
+            "calls": [f"{g} x sd_draft_layer (HSR, RMSNorm, QKV + RoPE, text-anchored "
+                      "attention, O projection, RMSNorm, gated MLP)", *kinds],
+            "ms_per_cycle": round(t_cyc, 4), "bytes_per_cycle": int(byt),
+            "draft_layer_us": round(t_layer * 1e3, 2),
+            "draft_layer_bytes": int(dl.bytes_per_call),
+            "draft_layer_gbs": round(dl.bytes_per_call / (t_layer / 1e3) / 1e9, 1),
+            "kv_bytes_per_token_at_n": {str(n): int(byt / (n + 1)) for n in range(g + 1)},
+            "speedup_at_n": {str(n): round((n + 1) * t_dec / t_cyc, 3) for n in range(g + 1)},
+            "break_even_n": next((n for n in range(g + 1) if (n + 1) * t_dec >= t_cyc), None)}
+        del gc, gl, dl
     res["methods"] = methods
     return res
+
+
+class DraftLayerSteps:
+    """One Sparrow draft layer of the 7B-like shapes (random bf16 weights, 517 MB) run for each
+    of the cycle's draft steps on its own text-only cache (1,024 earlier text positions, one row
+    appended per step)."""
+
+    def __init__(self, cyc):
+        from speculative_decoding_attention_verify_b200 import sdattn as sd
+        torch, dev, gen = cyc.torch, cyc.dev, cyc.gen
+        g = cyc.g
+        w = gen.make_draft_layer_workload(n=1, l_txt=int(cyc.w.l_txt[0]))
+        dvc = cyc.k.device
+        t = lambda a: dev.tensor(a, gen.BF16, dvc)
+        self.layer = sd.DraftLayer(w.d_model, w.h_q, w.h_kv, w.head_dim, w.d_ff, w.rms_eps,
+                                   w.rope_theta, **{n: t(getattr(w, n)) for n in sd.DraftLayer.NAMES})
+        cap = w.l_txt + g
+        k = torch.zeros((1, w.h_kv, cap, w.head_dim), dtype=torch.bfloat16, device=dvc)
+        v = torch.zeros_like(k)
+        k[:, :, :w.l_txt] = t(w.k_cache[:, :, :w.l_txt])
+        v[:, :, :w.l_txt] = t(w.v_cache[:, :, :w.l_txt])
+        self.caches = [sd.KVCache(k, v, dev.int32([w.l_txt + i + 1], dvc)) for i in range(g)]
+        self.emb = [t(w.emb) for _ in range(g)]
+        self.hid = t(w.hid)
+        self.y = [torch.empty((1, w.d_model), dtype=torch.bfloat16, device=dvc) for _ in range(g)]
+        nb = sd.sd_draft_layer_workspace_size(self.layer, 1, self.caches[-1], cap, w.window)
+        self.ws = torch.empty(nb, dtype=torch.uint8, device=dvc)
+        self.calls = [lambda s, i=i: sd.sd_draft_layer(self.layer, self.emb[i], self.hid,
+                                                       self.caches[i], cap, w.window,
+                                                       out=self.y[i], workspace=self.ws, stream=s)
+                      for i in range(g)]
+        D, F, HD = w.d_model, w.d_ff, w.h_q * w.head_dim
+        nqkv = (w.h_q + 2 * w.h_kv) * w.head_dim
+        weights = 2 * (D * 2 * D + nqkv * D + D * HD + 2 * F * D + D * F + 2 * D + nqkv)
+        window = min(w.window, w.l_txt + 1) * w.h_kv * w.head_dim * 2 * 2
+        self.bytes_per_call = weights + window + 3 * D * 2 + 2 * w.h_kv * w.head_dim * 2
 
 
 def long_context(torch, sd, flusher, peak, l_vis=140_000, layers=28, topk=1024, reps=3):

@@ -323,6 +323,50 @@ SD_API sd_status sd_hsr_project(const void *emb, const void *hid, int32_t n_rows
                          const void *weight, const void *bias, void *y, void *stream);
 
 /*
+ * Sparrow's draft layer [SPW 3.1 HSR-VATA: the draft model takes an FC over [text embedding ;
+ * reused target hidden state] and attends only to text-anchored positions].  The pages name no
+ * other layer internals; this is one pre-norm decoder layer of the target's shapes:
+ *     x  = W_hsr [e ; h]                                   (as sd_hsr_project, kept in fp32)
+ *     a  = RMSNorm(x) * ln1,  [q ; k ; v] = W_qkv a + b_qkv
+ *     q, k rotated by RoPE at the row's position (rotate-half pairs (i, i + d/2),
+ *          angle = pos * rope_theta^(-2i/d))
+ *     k, v written into the draft's cache at the row's position; q rounded to bf16
+ *     o  = text-anchored attention of the rows over that cache (window, no visual span)
+ *     x2 = x + W_o o,  m = RMSNorm(x2) * ln2,  y = x2 + W_down (silu(W_gate m) * (W_up m))
+ * with RMSNorm(x)_i = x_i / sqrt(mean_j x_j^2 + rms_eps).  All weights bf16, row-major
+ * [out][in]: w_hsr [d_model][2 d_model], ln1 / ln2 [d_model], w_qkv [(h_q + 2 h_kv) head_dim]
+ * [d_model] (query heads, then key heads, then value heads), b_qkv [(h_q + 2 h_kv) head_dim] or
+ * NULL, w_o [d_model][h_q head_dim], w_gate_up [2 d_ff][d_model] (the gate rows, then the up
+ * rows), w_down [d_model][d_ff]; the big matrices 16-byte aligned.
+ */
+typedef struct {
+    int32_t d_model, h_q, h_kv, head_dim, d_ff;
+    float rms_eps, rope_theta;
+    const void *w_hsr, *ln1, *w_qkv, *b_qkv, *w_o, *ln2, *w_gate_up, *w_down;
+} sd_draft_layer_desc;
+
+/*
+ * Workspace of sd_draft_layer (fp32 activations of the rows and the attention's workspace).
+ */
+SD_API sd_status sd_draft_layer_workspace_size(const sd_draft_layer_desc *w, int32_t n_rows,
+                                               const sd_kv_desc *cache, int32_t max_kv_len,
+                                               int32_t window, size_t *bytes);
+
+/*
+ * One draft layer for n_rows (1..4) rows of one sequence: emb, hid [n_rows][d_model] bf16 in,
+ * y [n_rows][d_model] bf16 out.  cache: the draft's own bf16 KV cache of that sequence (batch 1,
+ * contiguous or paged, head_dim 64 or 128), whose device kv_len[0] already counts the rows: row r
+ * is position kv_len[0] - n_rows + r, and the call WRITES its k and v there.  max_kv_len: host
+ * hint >= kv_len[0]; window >= 1.  The fp32 accumulation of every projection is exact to about
+ * 1e-6 relative; the rows' q, k and v pass through bf16 (the cache's type), the MLP input too.
+ * workspace: sd_draft_layer_workspace_size bytes, 256-byte aligned.
+ */
+SD_API sd_status sd_draft_layer(const sd_draft_layer_desc *w, const void *emb, const void *hid,
+                                int32_t n_rows, const sd_kv_desc *cache, int32_t max_kv_len,
+                                int32_t window, void *y, void *workspace, size_t workspace_bytes,
+                                int32_t *dev_err, void *stream);
+
+/*
  * Workspace for sd_accept_greedy / sd_accept_sample.  max_gamma: host hint >= gamma[b].
  */
 SD_API sd_status sd_accept_workspace_size(int32_t batch, int32_t max_gamma, int32_t vocab,

@@ -56,7 +56,8 @@ EXPORTS = ("sd_status_string", "sd_version", "sd_attention_workspace_size", "sd_
            "sd_topk_select", "sd_hsr_project", "sd_accept_workspace_size", "sd_accept_greedy",
            "sd_accept_sample", "sd_verify_attention_noalloc", "sd_sparse_workspace_size",
            "sd_sparse_selection_size", "sd_sparse_stage", "sd_sparse_attention_staged",
-           "sd_topk_scored_workspace_size", "sd_topk_select_scored", "sd_set_wait_timeout_ns")
+           "sd_topk_scored_workspace_size", "sd_topk_select_scored", "sd_set_wait_timeout_ns",
+           "sd_draft_layer_workspace_size", "sd_draft_layer")
 
 # Size of the library's fixed scratch used by sd_verify_attention_noalloc.
 SD_VERIFY_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -76,6 +77,8 @@ def lib():
                 h.sd_status_string.restype = ctypes.c_char_p
                 h.sd_status_string.argtypes = [ctypes.c_int]
                 h.sd_version.restype = I32
+                h.sd_draft_layer_workspace_size.argtypes = [P, I32, P, I32, I32, ctypes.POINTER(SZ)]
+                h.sd_draft_layer.argtypes = [P, P, P, I32, P, I32, I32, P, P, SZ, P, P]
                 h.sd_set_wait_timeout_ns.restype = ctypes.c_uint64
                 h.sd_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
                 h.sd_attention_workspace_size.argtypes = [ctypes.c_int, P, P, I32, ctypes.POINTER(SZ)]
@@ -100,7 +103,7 @@ def lib():
                 h.sd_topk_select_scored.argtypes = [ctypes.c_int, P, P, P, I32, P, P, I32, I32, P,
                                                     P, P, SZ, P, P]
                 for name in EXPORTS[2:]:
-                    if name != "sd_set_wait_timeout_ns":
+                    if name not in ("sd_set_wait_timeout_ns",):
                         getattr(h, name).restype = ctypes.c_int
                 _LIB = h
     return _LIB
@@ -369,6 +372,60 @@ def sd_topk_select_scored(mode: int, q: Queries, kv: KVCache, cand_begin, cand_e
             _ptr(scores_out), _ptr(ws), ws.numel(), _ptr(dev_err), _stream(stream)),
             "sd_topk_select_scored")
     return idx_out
+
+
+class sd_draft_layer_desc(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int32), ("h_q", ctypes.c_int32), ("h_kv", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("d_ff", ctypes.c_int32),
+                ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
+                ("w_hsr", ctypes.c_void_p), ("ln1", ctypes.c_void_p), ("w_qkv", ctypes.c_void_p),
+                ("b_qkv", ctypes.c_void_p), ("w_o", ctypes.c_void_p), ("ln2", ctypes.c_void_p),
+                ("w_gate_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p)]
+
+
+class DraftLayer:
+    """The weights of one draft layer (bf16 tensors on the GPU) and their C descriptor."""
+
+    NAMES = ("w_hsr", "ln1", "w_qkv", "b_qkv", "w_o", "ln2", "w_gate_up", "w_down")
+
+    def __init__(self, d_model, h_q, h_kv, head_dim, d_ff, rms_eps, rope_theta, **weights):
+        self.weights = weights
+        d = sd_draft_layer_desc()
+        d.d_model, d.h_q, d.h_kv, d.head_dim, d.d_ff = d_model, h_q, h_kv, head_dim, d_ff
+        d.rms_eps, d.rope_theta = float(rms_eps), float(rope_theta)
+        for name in self.NAMES:
+            t = weights.get(name)
+            setattr(d, name, _ptr(t))
+        self.desc = d
+        self.d_model = d_model
+
+
+def sd_draft_layer_workspace_size(layer: DraftLayer, n_rows: int, cache: KVCache,
+                                  max_kv_len: int, window: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().sd_draft_layer_workspace_size(ctypes.byref(layer.desc), int(n_rows),
+                                               ctypes.byref(cache.desc), int(max_kv_len),
+                                               int(window), ctypes.byref(n)),
+           "sd_draft_layer_workspace_size")
+    return n.value
+
+
+def sd_draft_layer(layer: DraftLayer, emb: torch.Tensor, hid: torch.Tensor, cache: KVCache,
+                   max_kv_len: int, window: int, out=None, workspace=None, dev_err=None,
+                   stream=None) -> torch.Tensor:
+    """One draft layer for the rows of emb / hid [n][d_model]; writes the rows' k and v into
+    `cache` (whose kv_len already counts them)."""
+    n = emb.shape[0]
+    if out is None:
+        out = torch.empty((n, layer.d_model), dtype=torch.bfloat16, device=emb.device)
+    nbytes = sd_draft_layer_workspace_size(layer, n, cache, max_kv_len, window)
+    ws = _workspace(nbytes, emb.device, workspace)
+    with _on(emb):
+        _check(lib().sd_draft_layer(ctypes.byref(layer.desc), _ptr(emb), _ptr(hid), int(n),
+                                    ctypes.byref(cache.desc), int(max_kv_len), int(window),
+                                    _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
+                                    _stream(stream)), "sd_draft_layer")
+    return out
 
 
 def sd_hsr_project(emb: torch.Tensor, hid: torch.Tensor, weight: torch.Tensor, bias=None,
