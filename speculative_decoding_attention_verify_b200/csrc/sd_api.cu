@@ -26,7 +26,7 @@ int device_sm_count() {
 }
 
 AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, int batch,
-                        int max_q_rows, long long max_stream) {
+                        int max_q_rows, long long max_stream, long long ws_stream) {
     AttnPlan plan{};
     const int G = h_q / h_kv;
     const int rows = G * max_q_rows;
@@ -77,6 +77,13 @@ AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, in
                 plan.tc_splits = (int)s;
             }
         }
+    }
+    if (ws_stream > max_stream) {
+        const AttnPlan w = plan_attention(kind, dtype, head_dim, h_q, h_kv, batch, max_q_rows,
+                                          ws_stream);
+        const int cap = w.simt_splits > w.tc_splits ? w.simt_splits : w.tc_splits;
+        if (plan.simt_splits > cap) plan.simt_splits = cap;
+        if (plan.tc_splits > cap) plan.tc_splits = cap;
     }
     const int splits = plan.simt_splits > plan.tc_splits ? plan.simt_splits : plan.tc_splits;
     plan.ws_bytes = splits > 1 ? (size_t)splits * rows_cap * h_q * (head_dim + 2) * sizeof(float)
@@ -131,7 +138,7 @@ sd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SD_OK : SD_ERR_
 
 // Common validation of the attention calls; fills the plan for the kind.
 sd_status check_attention(sd_attn_kind kind, const sd_q_desc *q, const sd_kv_desc *kv, int batch,
-                          long long max_stream, AttnPlan *plan) {
+                          long long max_stream, AttnPlan *plan, long long ws_stream = 0) {
     if (!q || !kv || batch < 1 || batch > 65535) return SD_ERR_INVALID_ARG;
     if (!kv_desc_ok(kv, batch)) return SD_ERR_INVALID_ARG;
     if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
@@ -140,7 +147,7 @@ sd_status check_attention(sd_attn_kind kind, const sd_q_desc *q, const sd_kv_des
         return SD_ERR_INVALID_ARG;
     if ((long long)batch * q->max_q_rows > (1LL << 30)) return SD_ERR_INVALID_ARG;
     *plan = plan_attention(kind, kv->dtype, kv->head_dim, q->h_q, kv->h_kv, batch, q->max_q_rows,
-                           max_stream);
+                           max_stream, ws_stream);
     return SD_OK;
 }
 
@@ -331,8 +338,10 @@ sd_status sd_text_anchored_attention(const sd_q_desc *q, const void *q_data,
         return SD_ERR_INVALID_ARG;
     AttnPlan plan;
     if (!q) return SD_ERR_INVALID_ARG;
+    // (the workspace query sized the plan of a max_kv_len stream)
     sd_status st = check_attention(SD_ATTN_TEXT_ANCHORED, q, kv, batch,
-                                   stream_hint(SD_ATTN_TEXT_ANCHORED, q, max_window), &plan);
+                                   stream_hint(SD_ATTN_TEXT_ANCHORED, q, max_window), &plan,
+                                   q->max_kv_len);
     if (st != SD_OK) return st;
     if (plan.ws_bytes > workspace_bytes || (plan.ws_bytes && !workspace)) return SD_ERR_WORKSPACE;
     AttnParams p = base_params(SD_ATTN_TEXT_ANCHORED, q, q_data, kv, batch, out, plan, workspace,

@@ -61,8 +61,13 @@ struct AttnPlan {
 
 int device_sm_count();
 unsigned long long wait_limit_ns();  // the process-wide bound set by sd_set_wait_timeout_ns
+// Plan of an attention call whose streams hold at most max_stream positions.  When the caller's
+// workspace was sized for a longer stream (ws_stream > max_stream: a text-anchored call whose
+// workspace query knew only max_kv_len), the split counts are capped at those of the ws_stream
+// plan, so that the workspace it reported always suffices (the split model is not monotone in
+// the stream length).
 AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, int batch,
-                        int max_q_rows, long long max_stream);
+                        int max_q_rows, long long max_stream, long long ws_stream = 0);
 
 cudaError_t launch_attention_simt(const AttnParams &p, const AttnPlan &plan, cudaStream_t s);
 cudaError_t launch_attention_tc(const AttnParams &p, const AttnPlan &plan, cudaStream_t s);

@@ -24,6 +24,10 @@ struct TcMaps {
 // engine).
 bool encode_kv_maps(const AttnParams &p, int max_kv_len, TcMaps *maps);
 
+// The small-row engine (S on the tensor core, P.V on CUDA cores) for G * max_q_rows <= 8.
+bool tc_small_supported(int head_dim, int rows);
+cudaError_t launch_attention_tc_small(const AttnParams &p, const TcMaps &maps, cudaStream_t s);
+
 namespace tc {
 
 // Bound of the drains after an abort (a CTA waiting for its own copies and MMAs to finish):

@@ -164,6 +164,17 @@ def test_text_anchored_matches_oracle(cfg, kw, case):
     _assert_close(out, ref, w.dtype, f"text-anchored cfg{cfg} {kw} {case}")
 
 
+@pytest.mark.parametrize("window", [900, 960, 1000, 1023])
+def test_text_anchored_window_shorter_than_cache_fits_reported_workspace(window):
+    """The workspace query knows only max_kv_len; a call whose window makes the streams shorter
+    plans from the window, and its split count (the split model is not monotone in the stream
+    length) must not outgrow the workspace the query reported.  No visual span, 7 rows per KV
+    head, about 1,025 positions: the draft layer's own attention."""
+    w = gen.make_attn_workload(1, l_vis=64, l_txt=960)
+    out, ref = _text_anchored_case(w, vis=(0, 0), window=window)
+    _assert_close(out, ref, w.dtype, f"text-anchored window {window}")
+
+
 def test_text_anchored_multi_row_verify_shape():
     """Text-anchored attention over gamma+1 rows at once (rows slide the window up)."""
     w = gen.make_attn_workload(1, l_vis=2000, l_txt=400, gamma=5)

@@ -3,8 +3,17 @@
 Output y: max-abs <= 2e-2.  y is rounded to bf16 (2^-9 relative: 0.008 at |y| = 4, about the
 largest output of the 7B-like layer) after fp32 accumulation of every projection; the rows' q,
 k and v pass through bf16 (the cache's type) and the MLP's input too, each perturbing the output
-by a few 1e-3.  The rows' k and v written into the cache: within one bf16 step (2^-8 relative)
-of the oracle's, which rounds its own fp64 values.  The rest of the cache is untouched.
+by a few 1e-3.
+
+The rows' k and v written into the cache, element by element: the kernels feed every projection
+a bf16 input vector (the normalised x here: relative error <= 2^-9 per entry), accumulate in
+fp32 and round the result to bf16; the oracle keeps fp64 throughout and rounds only the stored
+value.  So |k_gpu - k_oracle| <= E + 2^-8 (|k_gpu| + |k_oracle|), with E = 2^-8 sum_i |W_ji a_i|
+(twice the input-rounding bound, the margin covering fp32 accumulation and the fp32 RMSNorm
+scale) and, for keys, E of both members of the rotated pair added (RoPE mixes them with
+|cos|, |sin| <= 1).  That worst case lets every rounding line up; the rounding errors are
+independent, so over all the rows' elements the RMS difference must also stay below 2^-6 of the
+oracle's RMS (about eight times the expected 2^-9).  The rest of the cache is untouched.
 """
 import numpy as np
 import pytest
@@ -35,11 +44,24 @@ def _run(w):
                           w.kv_len, w.window, dev_err=flag)
     torch.cuda.synchronize()
     assert flag.item() == 0
-    ry, rk, rv, _ = oracle.draft_layer(w, w.emb, w.hid, w.k_cache, w.v_cache, w.kv_len, w.window)
-    return y, k, v, ry, rk, rv
+    ry, rk, rv, parts = oracle.draft_layer(w, w.emb, w.hid, w.k_cache, w.v_cache, w.kv_len,
+                                           w.window)
+    return y, k, v, ry, rk, rv, parts
 
 
-def _check(w, y, k, v, ry, rk, rv):
+def _kv_bounds(w, parts):
+    """E for the rows' keys and values [h_kv][n][d] (see the module docstring)."""
+    d, hq, hk, half = w.head_dim, w.h_q, w.h_kv, w.head_dim // 2
+    a = np.abs(oracle.rmsnorm(parts["x"], w.ln1, w.rms_eps))          # [n][D]
+    wq = np.abs(gen.f32_from_bf16_bits(w.w_qkv).astype(np.float64))  # [(hq + 2 hk) d][D]
+    e = 2.0 ** -8 * (a @ wq.T)                                         # [n][(hq + 2 hk) d]
+    ek = e[:, hq * d:(hq + hk) * d].reshape(w.n, hk, d)
+    ek = ek + np.concatenate([ek[..., half:], ek[..., :half]], axis=-1)
+    ev = e[:, (hq + hk) * d:].reshape(w.n, hk, d)
+    return ek.transpose(1, 0, 2), ev.transpose(1, 0, 2)
+
+
+def _check(w, y, k, v, ry, rk, rv, parts):
     err = float(np.abs(dev.to_numpy_f64(y) - ry).max())
     assert err <= TOL, err
     lo = w.kv_len - w.n
@@ -47,10 +69,12 @@ def _check(w, y, k, v, ry, rk, rv):
     gv = v.view(torch.int16).cpu().numpy().view(np.uint16)
     np.testing.assert_array_equal(gk[:, :, :lo], w.k_cache[:, :, :lo])
     np.testing.assert_array_equal(gv[:, :, :lo], w.v_cache[:, :, :lo])
-    for got, want in ((gk, rk), (gv, rv)):
-        a = gen.f32_from_bf16_bits(got[:, :, lo:w.kv_len]).astype(np.float64)
-        b = gen.f32_from_bf16_bits(want[:, :, lo:w.kv_len]).astype(np.float64)
-        assert (np.abs(a - b) <= 2.0 ** -8 * np.abs(b) + 1e-30).all()
+    ek, ev = _kv_bounds(w, parts)
+    for got, want, bound in ((gk, rk, ek), (gv, rv, ev)):
+        a = gen.f32_from_bf16_bits(got[0, :, lo:w.kv_len]).astype(np.float64)
+        b = gen.f32_from_bf16_bits(want[0, :, lo:w.kv_len]).astype(np.float64)
+        assert (np.abs(a - b) <= bound + 2.0 ** -8 * (np.abs(a) + np.abs(b))).all()
+        assert np.sqrt(np.mean((a - b) ** 2)) <= 2.0 ** -6 * np.sqrt(np.mean(b ** 2))
     return err
 
 
