@@ -7,17 +7,19 @@
 // 128-position tile instead of 16) and the four softmax warps form P.V themselves while it
 // computes the next tile's S.
 //
-// One CTA per (split, KV head, sequence); 6 warps, one CTA per SM:
-//   warps 0-3  row copies: Q is placed four times in the 128 MMA rows, so warp w (copy w) reads
-//              its rows' scores for the tile's columns [32w, 32w + 32) from TMEM (lane r = row r)
-//              and keeps its own running max and sum per row; it writes its P (fp32) to shared
-//              memory, then every lane of the warp accumulates O[r][4 head dims] for the rows
-//              over those 32 positions, reading V straight from the TMA-staged tile
-//   warp 4     TMA producer: lane 0 K tiles, lane 1 V tiles (128 positions, 128-byte swizzle),
-//              3-stage ring, K released when S is computed, V when the four warps are done
-//   warp 5     MMA issuer (S = Q K^T into one of two 128-column TMEM buffers) and TMEM owner
-// O stays in registers (a rescale is a register multiply); the four copies are merged in shared
-// memory at the end.  Partial outputs (O, max, sum) go to the split workspace exactly as the
+// One CTA per (split, KV head, sequence); 10 warps, one CTA per SM:
+//   warps 0-7  Q is placed four times in the 128 MMA rows (copy c in TMEM lanes [32c, 32c+32));
+//              warp w reads the scores of copy w % 4 for the tile's 16 columns
+//              [32 (w % 4) + 16 (w / 4), +16) (lane r = row r), keeps its own running max and
+//              sum per row, writes its P (fp32) to shared memory, then every lane of the warp
+//              accumulates O[r][head dims of the lane] for the rows over those 16 positions,
+//              reading V straight from the TMA-staged tile.  Two such warps per SM
+//              sub-partition hide each other's latencies.
+//   warp 8     TMA producer: lane 0 K tiles, lane 1 V tiles (128 positions, 128-byte swizzle),
+//              3-stage ring, K released when S is computed, V when the eight warps are done
+//   warp 9     MMA issuer (S = Q K^T into one of two 128-column TMEM buffers) and TMEM owner
+// O stays in registers (a rescale is a register multiply); the eight partial results are merged
+// in shared memory at the end.  Partial outputs (O, max, sum) go to the split workspace exactly as the
 // other engines write them, or, with a single split, O / sum is written directly.
 // Every wait on an mbarrier is bounded (the launch's wait bound); on expiry the CTA records
 // SD_DEVERR_TIMEOUT, drains its own copies and MMAs (at most 1 s), frees TMEM and exits.
@@ -31,9 +33,11 @@ using namespace tc;
 
 constexpr int kST = 128;             // positions per tile
 constexpr int kSRows = 8;            // rows per KV head served here
-constexpr int kSThreads = 6 * 32;
-constexpr int kSProducer = 4;
-constexpr int kSMma = 5;
+constexpr int kSCompute = 8;           // compute warps
+constexpr int kSCols = kST / kSCompute;  // tile columns per compute warp
+constexpr int kSThreads = (kSCompute + 2) * 32;
+constexpr int kSProducer = kSCompute;
+constexpr int kSMma = kSCompute + 1;
 constexpr int kSStages = 3;
 constexpr uint32_t kSTmemCols = 512;  // S0 [0,128) S1 [128,256) Q [384, 384 + D/2)
 constexpr uint32_t kSColQ = 384;
@@ -44,7 +48,7 @@ template <int D>
 struct SCfg {
     static constexpr int kTileBytes = kST * D * 2;
     static constexpr int kRing = kSStages * 2 * kTileBytes;
-    static constexpr int kPBytes = 4 * 32 * kSRows * 4;  // [warp][position][row] fp32
+    static constexpr int kPBytes = kSCompute * kSCols * kSRows * 4;  // [warp][position][row]
     static constexpr int kBarOffset = kRing + kPBytes;
     static constexpr int kSmem = kBarOffset + 256 + 1024;
 };
@@ -68,7 +72,7 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
               QF = 4 * S + 5;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * S + 6);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *s_stream = reinterpret_cast<int *>(tmem_slot + 2);  // stream set-up scratch (10 ints)
+    int *s_stream = reinterpret_cast<int *>(tmem_slot + 2);  // stream set-up scratch (14 ints)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.z, g = blockIdx.y, split = blockIdx.x;
@@ -115,11 +119,11 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             mbar_init(BAR(KF + s), 1);
             mbar_init(BAR(VF + s), 1);
             mbar_init(BAR(KE + s), 1);
-            mbar_init(BAR(VE + s), 4);  // one arrival per softmax warp
+            mbar_init(BAR(VE + s), kSCompute);  // one arrival per compute warp
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(BAR(SF + s), 1);
-            mbar_init(BAR(SE + s), 4);
+            mbar_init(BAR(SE + s), kSCompute);
         }
         mbar_init(BAR(DR), 1);
         mbar_init(BAR(QF), 128);
@@ -258,8 +262,9 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     } else {
         // ---------------------------------------------------------- softmax + P.V ---------
         const unsigned FULL = 0xffffffffu;
-        const int c0 = warp * 32;  // this copy's tile columns
-        const int r = lane;        // this lane's row (real when r < R)
+        const int cp = warp & 3;                // this warp's row copy (its TMEM lanes)
+        const int c0 = cp * 32 + (warp >> 2) * kSCols;  // its first tile column
+        const int r = lane;                     // this lane's row (real when r < R)
         const bool row_ok = r < R;
         const int limit = kv_len - n_q + (row_ok ? r / G : 0);
         uint32_t lo1 = 0x80000000u, w1 = 0u, lo2 = 0x80000000u, w2 = 0u;
@@ -281,13 +286,13 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         const bool sel_all = !sparse || si.s1 <= kv_len - n_q + 1;
         const int32_t *cpos = sparse ? p.cpos + ((int64_t)b * kv.h_kv + g) * p.k_cap : nullptr;
         const float sl2 = p.scale_log2;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        float *pw = sP + warp * 32 * kSRows;  // [position][row]
-        float o[kSRows][DPL];
+        const uint32_t lane_base = tmem + ((uint32_t)(cp * 32) << 16);
+        float *pw = sP + warp * kSCols * kSRows;  // [position][row]
+        float2 o[kSRows][DPL / 2];  // head dims (2x, 2x + 1) of this lane's DPL, every row
 #pragma unroll
         for (int q = 0; q < kSRows; ++q)
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) o[q][e] = 0.f;
+            for (int e = 0; e < DPL / 2; ++e) o[q][e] = make_float2(0.f, 0.f);
         float m_used = -INFINITY, l = 0.f;
         bool ok_run = true;
         for (int t = 0; t < n_my; ++t) {
@@ -304,23 +309,23 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 break;
             }
             tc_after();
-            float v[32];
-            tmem_ld32(lane_base + sb * kST + c0, v);
+            float v[kSCols];
+            tmem_ld16(lane_base + sb * kST + c0, v);
             tc_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(SE + sb));  // this warp is done with the S buffer
             // mask (skipped for columns inside the run and visible in full to every row of the
             // warp), then this row's max over the warp's 32 columns, in base 2
             const int q0p = p0 + c0;
-            const bool in_run = q0p >= seg_lo && q0p + 32 <= seg_hi;
+            const bool in_run = q0p >= seg_lo && q0p + kSCols <= seg_hi;
             const uint32_t d1 = (uint32_t)q0p - lo1, d2 = (uint32_t)q0p - lo2;
             const bool whole = !row_ok || (cmp ? sel_all
-                                               : ((w1 >= 31 && d1 <= w1 - 31) ||
-                                                  (w2 >= 31 && d2 <= w2 - 31)));
+                                               : ((w1 >= kSCols - 1 && d1 <= w1 - (kSCols - 1)) ||
+                                                  (w2 >= kSCols - 1 && d2 <= w2 - (kSCols - 1))));
             if (!__all_sync(FULL, in_run && whole)) {
                 const uint32_t seg_w = (uint32_t)(seg_hi - seg_lo);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
+                for (int e = 0; e < kSCols; ++e) {
                     bool vis;
                     if (!cmp) {
                         const uint32_t j = (uint32_t)(q0p + e);
@@ -335,7 +340,7 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             }
             float mx = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) mx = max3(mx, v[e], v[e + 1]);
+            for (int e = 0; e < kSCols; e += 2) mx = max3(mx, v[e], v[e + 1]);
             mx = mx == -INFINITY ? -INFINITY : mx * sl2;
             // lazy rescale: the reference max moves only when the row's max grows by > 2^8
             const bool grow = mx > m_used + kSRescale;
@@ -350,7 +355,7 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
             float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
+            for (int e = 0; e < kSCols; e += 2) {
                 const float2 x = __ffma2_rn(make_float2(v[e], v[e + 1]), sc2, nm2);
                 const float2 pe = make_float2(ex2(x.x), ex2(x.y));
                 acc2 = __fadd2_rn(acc2, pe);
@@ -366,7 +371,7 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 for (int q = 0; q < kSRows; ++q) {
                     const float cq = __shfl_sync(FULL, corr, q);
 #pragma unroll
-                    for (int e = 0; e < DPL; ++e) o[q][e] *= cq;
+                    for (int e = 0; e < DPL / 2; ++e) o[q][e] = __fmul2_rn(o[q][e], make_float2(cq, cq));
                 }
             }
             __syncwarp();
@@ -376,26 +381,26 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 ok_run = false;
                 break;
             }
-            const int n_cols = max(0, min(32, seg_hi - q0p));  // V rows past the run: skipped
-            const uint8_t *vt = sKV + (size_t)s * 2 * C::kTileBytes + C::kTileBytes;
-            const int dl = lane * DPL;                      // first head dim of this lane
-            const uint32_t hoff = (uint32_t)(dl >> 6) * kSHalf;
-            const uint32_t chunk = (uint32_t)((dl & 63) >> 3), within = (uint32_t)(dl & 7) * 2;
-#pragma unroll 4
-            for (int e = 0; e < n_cols; ++e) {
-                const int row = c0 + e;
-                const uint8_t *src = vt + hoff + row * 128 + (((chunk ^ (row & 7)) << 4) | within);
-                float vf[DPL];
+            const int n_cols = max(0, min(kSCols, seg_hi - q0p));  // V rows past the run: skipped
+            const int dl = lane * DPL;                          // first head dim of this lane
+            // this lane's bytes of V row c0 + e sit at vrow + e * 128 + voff[e & 7] (128-byte
+            // swizzle: 16-byte chunk c of row r is stored in slot c ^ (r & 7))
+            const uint8_t *vrow = sKV + (size_t)s * 2 * C::kTileBytes + C::kTileBytes +
+                                  (size_t)(dl >> 6) * kSHalf + (size_t)c0 * 128;
+            uint32_t voff[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                voff[j] = ((((uint32_t)(dl & 63) >> 3) ^ (uint32_t)j) << 4) | (uint32_t)(dl & 7) * 2;
+            auto pv = [&](int e, uint32_t off) {  // off: voff[e & 7]
+                const uint8_t *src = vrow + e * 128 + off;
+                float2 vf[DPL / 2];
                 if constexpr (DPL == 4) {
                     const uint2 w2v = *reinterpret_cast<const uint2 *>(src);
-                    vf[0] = bf16_lo(w2v.x);
-                    vf[1] = bf16_hi(w2v.x);
-                    vf[2] = bf16_lo(w2v.y);
-                    vf[3] = bf16_hi(w2v.y);
+                    vf[0] = make_float2(bf16_lo(w2v.x), bf16_hi(w2v.x));
+                    vf[1] = make_float2(bf16_lo(w2v.y), bf16_hi(w2v.y));
                 } else {
                     const uint32_t w1v = *reinterpret_cast<const uint32_t *>(src);
-                    vf[0] = bf16_lo(w1v);
-                    vf[1] = bf16_hi(w1v);
+                    vf[0] = make_float2(bf16_lo(w1v), bf16_hi(w1v));
                 }
                 const float4 pa = *reinterpret_cast<const float4 *>(pw + e * kSRows);
                 const float4 pb = *reinterpret_cast<const float4 *>(pw + e * kSRows + 4);
@@ -403,19 +408,34 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
 #pragma unroll
                 for (int q = 0; q < kSRows; ++q)
 #pragma unroll
-                    for (int x = 0; x < DPL; ++x) o[q][x] = fmaf(pr[q], vf[x], o[q][x]);
+                    for (int x = 0; x < DPL / 2; ++x)
+                        o[q][x] = __ffma2_rn(make_float2(pr[q], pr[q]), vf[x], o[q][x]);
+            };
+            if (n_cols == kSCols) {
+#pragma unroll 1
+                for (int e0 = 0; e0 < kSCols; e0 += 8)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) pv(e0 + j, voff[j]);
+            } else {
+#pragma unroll 1
+                for (int e = 0; e < n_cols; ++e)
+                    pv(e, ((((uint32_t)(dl & 63) >> 3) ^ (uint32_t)(e & 7)) << 4) |
+                              (uint32_t)(dl & 7) * 2);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(VE + s));  // this warp is done with the V stage
         }
-        // ---- epilogue: merge the four copies through shared memory (the ring is idle) ----
+        // ---- epilogue: merge the eight partials through shared memory ----
+        // Once every compute warp is past its last tile (the barrier) and the MMAs have drained,
+        // no copy or MMA touches the ring any more.
         bool done = ok_run;
         if (ok_run && n_my > 0)
             done = mbar_wait(BAR(DR), 0, abort_flag, p.dev_err, p.wait_ns);
         const bool have_any = __all_sync(FULL, done) && n_my > 0;
-        float *s_m = reinterpret_cast<float *>(sKV);            // [copy][row]
-        float *s_l = s_m + 4 * kSRows;                          // [copy][row]
-        float *s_o = s_l + 4 * kSRows;                          // [copy][row][D]
+        asm volatile("bar.sync 1, %0;" ::"n"(kSCompute * 32) : "memory");
+        float *s_m = reinterpret_cast<float *>(sKV);       // [warp][row]
+        float *s_l = s_m + kSCompute * kSRows;             // [warp][row]
+        float *s_o = s_l + kSCompute * kSRows;             // [warp][row][D]
         if (r < kSRows) {
             s_m[warp * kSRows + r] = (have_any && row_ok && l > 0.f) ? m_used : -INFINITY;
             s_l[warp * kSRows + r] = (have_any && row_ok) ? l : 0.f;
@@ -423,18 +443,19 @@ attn_tc_small_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
 #pragma unroll
         for (int q = 0; q < kSRows; ++q)
 #pragma unroll
-            for (int x = 0; x < DPL; ++x)
-                s_o[(warp * kSRows + q) * D + lane * DPL + x] = have_any ? o[q][x] : 0.f;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // thread tid: head dim tid % D of rows tid / D, tid / D + 128 / D, ...
-        for (int idx = tid; idx < R * D; idx += 128) {
+            for (int x = 0; x < DPL / 2; ++x)
+                *reinterpret_cast<float2 *>(s_o + (warp * kSRows + q) * D + lane * DPL + 2 * x) =
+                    have_any ? o[q][x] : make_float2(0.f, 0.f);
+        asm volatile("bar.sync 1, %0;" ::"n"(kSCompute * 32) : "memory");
+        // thread tid: head dim tid % D of rows tid / D, tid / D + 256 / D, ...
+        for (int idx = tid; idx < R * D; idx += kSCompute * 32) {
             const int rr = idx / D, d = idx % D;
             float M = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) M = fmaxf(M, s_m[c * kSRows + rr]);
+            for (int c = 0; c < kSCompute; ++c) M = fmaxf(M, s_m[c * kSRows + rr]);
             float L = 0.f, O = 0.f;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < kSCompute; ++c) {
                 const float mc = s_m[c * kSRows + rr];
                 const float f = mc == -INFINITY ? 0.f : ex2(mc - M);
                 L += f * s_l[c * kSRows + rr];
