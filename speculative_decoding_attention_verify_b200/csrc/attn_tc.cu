@@ -748,7 +748,6 @@ cudaError_t launch_attention_tc(const AttnParams &p, const AttnPlan &plan, cudaS
     // row copies: four when the planned rows per KV head fit in 32 (the draft steps), two when
     // they fit in 64 (verification of up to 9 rows x 7 heads)
     const int rows = p.group * p.max_q_rows;
-    if (tc_small_supported(p.kv.head_dim, rows)) return launch_attention_tc_small(p, maps, s);
     const int ncp = rows <= 32 ? 4 : rows <= kNcp2Rows ? 2 : 1;
 #define SD_TC_LAUNCH(DD, PG)                                                                   \
     (ncp == 4   ? launch_t<DD, PG, 4>(p, maps, s)                                              \

@@ -24,10 +24,6 @@ struct TcMaps {
 // engine).
 bool encode_kv_maps(const AttnParams &p, int max_kv_len, TcMaps *maps);
 
-// The small-row engine (S on the tensor core, P.V on CUDA cores) for G * max_q_rows <= 8.
-bool tc_small_supported(int head_dim, int rows);
-cudaError_t launch_attention_tc_small(const AttnParams &p, const TcMaps &maps, cudaStream_t s);
-
 namespace tc {
 
 // Bound of the drains after an abort (a CTA waiting for its own copies and MMAs to finish):
@@ -179,22 +175,6 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
         : "memory");
-}
-
-// 16 consecutive fp32 columns of this thread's TMEM lane (load and wait in one statement).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane (load and wait in one statement, so
