@@ -369,7 +369,6 @@ sd_status sd_draft_layer(const sd_draft_layer_desc *w, const void *emb, const vo
     a.n = n_rows;
     a.eps = w->rms_eps;
     a.dev_err = dev_err;
-    cudaError_t e;
     // x = W_hsr [e ; h]
     a.w = static_cast<const uint16_t *>(w->w_hsr);
     a.m = D;
@@ -377,7 +376,7 @@ sd_status sd_draft_layer(const sd_draft_layer_desc *w, const void *emb, const vo
     a.in_a = static_cast<const uint16_t *>(emb);
     a.in_b = static_cast<const uint16_t *>(hid);
     a.out_f = x;
-    if ((e = launch_gemv<IN_CONCAT, OUT_F32>(a, s)) != cudaSuccess) return SD_ERR_CUDA;
+    if (launch_gemv<IN_CONCAT, OUT_F32>(a, s) != cudaSuccess) return SD_ERR_CUDA;
     // q, k, v = W_qkv RMSNorm(x) + b; RoPE; k, v into the cache
     a = GemvArgs{};
     a.n = n_rows;
@@ -397,7 +396,7 @@ sd_status sd_draft_layer(const sd_draft_layer_desc *w, const void *emb, const vo
     a.kv = kv;
     a.params = params;
     a.window = window;
-    if ((e = launch_gemv<IN_NORM, OUT_QKV>(a, s)) != cudaSuccess) return SD_ERR_CUDA;
+    if (launch_gemv<IN_NORM, OUT_QKV>(a, s) != cudaSuccess) return SD_ERR_CUDA;
     // o = text-anchored attention of the rows over the draft cache (no visual span)
     sd_q_desc q;
     attn_descs(w, n_rows, cache, max_kv_len, params, &q);
@@ -414,7 +413,7 @@ sd_status sd_draft_layer(const sd_draft_layer_desc *w, const void *emb, const vo
     a.in_a = ob;
     a.res = x;
     a.out_f = x2;
-    if ((e = launch_gemv<IN_PLAIN, OUT_F32>(a, s)) != cudaSuccess) return SD_ERR_CUDA;
+    if (launch_gemv<IN_PLAIN, OUT_F32>(a, s) != cudaSuccess) return SD_ERR_CUDA;
     // [gate ; up] = W_gate_up RMSNorm(x2)
     a = GemvArgs{};
     a.n = n_rows;
@@ -426,7 +425,7 @@ sd_status sd_draft_layer(const sd_draft_layer_desc *w, const void *emb, const vo
     a.in_f = x2;
     a.gamma = static_cast<const uint16_t *>(w->ln2);
     a.out_f = gu;
-    if ((e = launch_gemv<IN_NORM, OUT_F32>(a, s)) != cudaSuccess) return SD_ERR_CUDA;
+    if (launch_gemv<IN_NORM, OUT_F32>(a, s) != cudaSuccess) return SD_ERR_CUDA;
     // y = x2 + W_down (silu(gate) * up)
     a = GemvArgs{};
     a.n = n_rows;
@@ -437,7 +436,7 @@ sd_status sd_draft_layer(const sd_draft_layer_desc *w, const void *emb, const vo
     a.in_f = gu;
     a.res = x2;
     a.out_b = static_cast<uint16_t *>(y);
-    if ((e = launch_gemv<IN_SWIGLU, OUT_BF16_RES>(a, s)) != cudaSuccess) return SD_ERR_CUDA;
+    if (launch_gemv<IN_SWIGLU, OUT_BF16_RES>(a, s) != cudaSuccess) return SD_ERR_CUDA;
     return SD_OK;
 }
 

@@ -39,7 +39,6 @@ constexpr uint32_t kHalf = kTT * 128;  // bytes of one 64-column half of a 128-r
 
 template <int D>
 struct TaCfg {
-    static constexpr int kHalves = D / 64;
     static constexpr int kTileBytes = kTT * D * 2;
     static constexpr int kStages = 2;  // pass-1 K ring (two CTAs per SM)
     // pass 1: Q tile, K ring, barriers
