@@ -370,7 +370,42 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
     if (row >= total || row >= p.rows_cap) return;
     const int64_t stride = (int64_t)p.rows_cap * p.h_q;  // between splits, in (row, head) units
     const int64_t rh = (int64_t)row * p.h_q + h;
-    const int n_splits = p.n_splits;
+    int n_splits = p.n_splits;
+    if (p.persist_s) {
+        // Persistent tensor-core decomposition: the CTAs whose item ranges meet the row's unit
+        // wrote slots 0.. in order; a unit inside one CTA's range has its output already.
+        // the row's sequence: the last b with q_start[b] <= row, found by the warp in two
+        // ballots (32 strided entries, then up to 32 entries of the chosen stretch), or by
+        // bisection beyond 1,024 sequences
+        int lo = 0;
+        if (p.batch <= 1024) {
+            const int bs = (p.batch + 31) / 32;
+            const bool in1 = lane * bs < p.batch;
+            unsigned m = __ballot_sync(
+                0xffffffffu, in1 && __ldg(p.q_start + (in1 ? lane * bs : 0)) <= row);
+            if (m == 0) return;  // a row before the first sequence's
+            const int base_b = (31 - __clz(m)) * bs;
+            const bool in2 = lane < bs && base_b + lane < p.batch;
+            m = __ballot_sync(0xffffffffu,
+                              in2 && __ldg(p.q_start + (in2 ? base_b + lane : 0)) <= row);
+            lo = base_b + (31 - __clz(m));
+        } else {
+            int hi = p.batch - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) / 2;
+                if (__ldg(p.q_start + mid) <= row)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+        }
+        const long long n_items = (long long)p.batch * p.kv.h_kv * p.persist_s;
+        const long long base = ((long long)lo * p.kv.h_kv + h / p.group) * p.persist_s;
+        const int c0 = (int)(((base + 1) * p.persist_g - 1) / n_items);
+        const int c1 = (int)(((base + p.persist_s) * p.persist_g - 1) / n_items);
+        if (c1 == c0) return;
+        n_splits = min(c1 - c0 + 1, p.n_splits);
+    }
     float o[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) o[e] = 0.f;

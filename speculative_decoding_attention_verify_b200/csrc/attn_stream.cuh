@@ -133,6 +133,46 @@ __device__ __forceinline__ StreamInfo stream_setup(const AttnParams &p, int b, i
     return si;
 }
 
+// The stream of sequence b for verify and text-anchored calls, computed by one thread on its
+// own (no block synchronisation): the same runs as stream_setup.
+__device__ __forceinline__ StreamInfo stream_info_single(const AttnParams &p, int b, int n_q,
+                                                         int kv_len) {
+    StreamInfo si{};
+    si.vb = si.ve = si.W = 0;
+    si.tail = 0;
+    si.sel = nullptr;
+    si.s0 = si.len0 = si.s1 = si.len1 = 0;
+    if (p.kind == SD_ATTN_VERIFY) {
+        si.len0 = kv_len;
+        return si;
+    }
+    si.vb = __ldg(p.vis_begin + b);
+    si.ve = __ldg(p.vis_end + b);
+    si.W = __ldg(p.window + b);
+    if (si.vb > si.ve) {
+        set_dev_err(p.dev_err, SD_DEVERR_INDEX);
+        si.vb = si.ve = 0;
+    }
+    si.vb = min(max(si.vb, 0), kv_len);
+    si.ve = min(max(si.ve, 0), kv_len);
+    int lowest = kv_len;
+    for (int i = 0; i < n_q; ++i) {
+        int lo1, hi1, lo2, hi2;
+        window_ranges(kv_len - n_q + i, si.vb, si.ve, si.W, lo1, hi1, lo2, hi2);
+        if (lo2 <= hi2) lowest = min(lowest, lo2);
+        if (lo1 <= hi1) lowest = min(lowest, lo1);
+    }
+    if (si.vb < si.ve && lowest < si.vb) {
+        si.s0 = lowest;
+        si.len0 = si.vb - lowest;
+        si.s1 = si.ve;
+    } else {
+        si.s1 = (si.vb < si.ve && lowest >= si.vb) ? max(lowest, si.ve) : lowest;
+    }
+    si.len1 = max(0, kv_len - si.s1);
+    return si;
+}
+
 // Allowed ranges of local row lr (query row lr / G) of the stream's sequence.
 __device__ __forceinline__ void row_ranges(const AttnParams &p, const StreamInfo &si, int lr,
                                            int R, int n_q, int kv_len, int &lo1, int &hi1,

@@ -26,7 +26,8 @@ int device_sm_count() {
 }
 
 AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, int batch,
-                        int max_q_rows, long long max_stream, long long ws_stream) {
+                        int max_q_rows, long long max_stream, long long ws_stream, bool paged,
+                        long long tc_tiles) {
     AttnPlan plan{};
     const int G = h_q / h_kv;
     const int rows = G * max_q_rows;
@@ -60,12 +61,22 @@ AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, in
             }
         }
     }
-    // Tensor-core decomposition: one CTA per SM.  Modelled time of split count s: waves x
-    // (per-CTA start-up and drain, about three tiles' worth, + tiles per CTA); the smallest wins.
+    // Tensor-core decompositions, one CTA per SM; the tile count of a unit is bounded by
+    // tc_tiles (verify: the stream's tiles; text-anchored: its two runs may each add a tile,
+    // and with pages two more; sparse: given by the caller).  Classic, modelled time of split
+    // count s: waves x (per-CTA start-up and drain, about three tiles' worth, + tiles per CTA),
+    // the smallest wins.  Persistent: every unit's tiles in one list spread evenly over the
+    // SMs, about (all tiles / SMs) + three tiles' worth of start-up and drain + two for the
+    // split merge + three per switch to another unit inside a CTA (its Q, the epilogue);
+    // taken when it models faster.
     plan.tc_splits = 1;
+    plan.tc_persist_s = plan.tc_persist_g = plan.tc_slots = 0;
     if (plan.tensor_core) {
+        if (tc_tiles < 1)
+            tc_tiles = (max_stream + 127) / 128 +
+                       (kind == SD_ATTN_TEXT_ANCHORED ? 1 + (paged ? 2 : 0) : 0);
         const long long units = (long long)batch * h_kv;
-        const long long tiles = (max_stream + 127) / 128;
+        const long long tiles = tc_tiles;
         long long best = -1;
         for (long long s = 1; s <= 64; ++s) {
             if (s > 1 && tiles / s < 2) break;
@@ -77,15 +88,35 @@ AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, in
                 plan.tc_splits = (int)s;
             }
         }
+        const long long n_items = units * tiles;
+        if (tiles >= 2 && n_items <= (1LL << 40) && tc_persistent_fits(head_dim, rows)) {
+            const long long g = n_items < sms ? n_items : sms;
+            const long long q = n_items / g;  // items per CTA, at least
+            const long long per_cta = (n_items + g - 1) / g;
+            const long long switches = (per_cta + tiles - 1) / tiles;  // (upper estimate)
+            const long long t = per_cta + 3 + 2 + 3 * switches;
+            // units a CTA's range may touch: its items span at most ceil(per_cta / tiles) + 1
+            const bool segs_ok = (per_cta + tiles - 1) / tiles + 1 <= tc_persistent_max_segments();
+            if (t < best && segs_ok) {
+                plan.tc_persist_s = (int)tiles;
+                plan.tc_persist_g = (int)g;
+                // CTAs whose item range meets one unit's: a range of at least q items, so at
+                // most ceil((tiles - 1) / q) + 1 of them (one spare)
+                plan.tc_slots = (int)((tiles - 1 + q - 1) / q + 2);
+            }
+        }
     }
     if (ws_stream > max_stream) {
         const AttnPlan w = plan_attention(kind, dtype, head_dim, h_q, h_kv, batch, max_q_rows,
-                                          ws_stream);
-        const int cap = w.simt_splits > w.tc_splits ? w.simt_splits : w.tc_splits;
+                                          ws_stream, 0, paged, 0);
+        int cap = w.simt_splits > w.tc_splits ? w.simt_splits : w.tc_splits;
+        if (w.tc_slots > cap) cap = w.tc_slots;
         if (plan.simt_splits > cap) plan.simt_splits = cap;
         if (plan.tc_splits > cap) plan.tc_splits = cap;
+        if (plan.tc_slots > cap) plan.tc_persist_s = plan.tc_persist_g = plan.tc_slots = 0;
     }
-    const int splits = plan.simt_splits > plan.tc_splits ? plan.simt_splits : plan.tc_splits;
+    int splits = plan.simt_splits > plan.tc_splits ? plan.simt_splits : plan.tc_splits;
+    if (plan.tc_slots > splits) splits = plan.tc_slots;
     plan.ws_bytes = splits > 1 ? (size_t)splits * rows_cap * h_q * (head_dim + 2) * sizeof(float)
                                : 0;
     return plan;
@@ -138,7 +169,8 @@ sd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SD_OK : SD_ERR_
 
 // Common validation of the attention calls; fills the plan for the kind.
 sd_status check_attention(sd_attn_kind kind, const sd_q_desc *q, const sd_kv_desc *kv, int batch,
-                          long long max_stream, AttnPlan *plan, long long ws_stream = 0) {
+                          long long max_stream, AttnPlan *plan, long long ws_stream = 0,
+                          long long tc_tiles = 0) {
     if (!q || !kv || batch < 1 || batch > 65535) return SD_ERR_INVALID_ARG;
     if (!kv_desc_ok(kv, batch)) return SD_ERR_INVALID_ARG;
     if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
@@ -147,7 +179,7 @@ sd_status check_attention(sd_attn_kind kind, const sd_q_desc *q, const sd_kv_des
         return SD_ERR_INVALID_ARG;
     if ((long long)batch * q->max_q_rows > (1LL << 30)) return SD_ERR_INVALID_ARG;
     *plan = plan_attention(kind, kv->dtype, kv->head_dim, q->h_q, kv->h_kv, batch, q->max_q_rows,
-                           max_stream, ws_stream);
+                           max_stream, ws_stream, kv->page_size != 0, tc_tiles);
     return SD_OK;
 }
 
@@ -176,10 +208,23 @@ AttnParams base_params(sd_attn_kind kind, const sd_q_desc *q, const void *q_data
     return p;
 }
 
+// Tiles of one unit of a sparse call on the tensor-core path: the compacted selection, then
+// the tail (which, from a page boundary, may start up to 15 positions lower).
+long long sparse_tc_tiles(const sd_kv_desc *kv, long long k, long long max_tail) {
+    return (k + 127) / 128 + (max_tail + (kv->page_size != 0 ? 15 : 0) + 127) / 128;
+}
+
 void set_splits(AttnParams &p, int n_splits) {
     p.n_splits = n_splits;
     p.ws_ml = n_splits > 1 ? p.ws_o + (size_t)n_splits * p.rows_cap * p.h_q * p.kv.head_dim
                            : nullptr;
+}
+
+// The plan's tensor-core decomposition: persistent (n_splits = the partial slots) or classic.
+void set_tc_decomposition(AttnParams &p, const AttnPlan &plan) {
+    p.persist_s = plan.tc_persist_s;
+    p.persist_g = plan.tc_persist_g;
+    set_splits(p, plan.tc_persist_s ? plan.tc_slots : plan.tc_splits);
 }
 
 sd_status run_attention(AttnParams p, const AttnPlan &plan, void *stream) {
@@ -188,11 +233,12 @@ sd_status run_attention(AttnParams p, const AttnPlan &plan, void *stream) {
     const bool aligned = ((reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.out)) &
                           15) == 0;
     if (plan.tensor_core && aligned) {
-        set_splits(p, plan.tc_splits);
+        set_tc_decomposition(p, plan);
         e = launch_attention_tc(p, plan, s);
         if (e != cudaSuccess && e != cudaErrorNotSupported) return SD_ERR_CUDA;
     }
     if (e == cudaErrorNotSupported) {
+        p.persist_s = p.persist_g = 0;
         set_splits(p, plan.simt_splits);
         e = launch_attention_simt(p, plan, s);
     }
@@ -311,7 +357,7 @@ sd_status sd_attention_workspace_size(sd_attn_kind kind, const sd_q_desc *q,
     if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
     // Worst-case stream for the kind (hints of the specific call are not known here).
     const AttnPlan plan = plan_attention(kind, kv->dtype, kv->head_dim, q->h_q, kv->h_kv, batch,
-                                         q->max_q_rows, q->max_kv_len);
+                                         q->max_q_rows, q->max_kv_len, 0, kv->page_size != 0, 0);
     *bytes = plan.ws_bytes;
     return SD_OK;
 }
@@ -361,7 +407,8 @@ sd_status sd_sparse_workspace_size(const sd_q_desc *q, const sd_kv_desc *kv, int
     if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
     const AttnPlan plan = plan_attention(SD_ATTN_SPARSE, kv->dtype, kv->head_dim, q->h_q,
                                          kv->h_kv, batch, q->max_q_rows,
-                                         stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail));
+                                         stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail),
+                                         0, kv->page_size != 0, sparse_tc_tiles(kv, k, max_tail));
     *bytes = sparse_ws_bytes(plan, kv, batch, k);
     return SD_OK;
 }
@@ -377,7 +424,8 @@ sd_status sd_sparse_attention(const sd_q_desc *q, const void *q_data, const sd_k
     AttnPlan plan;
     if (!q) return SD_ERR_INVALID_ARG;
     sd_status st = check_attention(SD_ATTN_SPARSE, q, kv, batch,
-                                   stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail), &plan);
+                                   stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail), &plan,
+                                   0, sparse_tc_tiles(kv, k, max_tail));
     if (st != SD_OK) return st;
     const size_t need = sparse_ws_bytes(plan, kv, batch, k);
     if (need > workspace_bytes || (need && !workspace)) return SD_ERR_WORKSPACE;
@@ -443,7 +491,8 @@ sd_status sd_sparse_attention_staged(const sd_q_desc *q, const void *q_data,
         return SD_ERR_INVALID_ARG;
     AttnPlan plan;
     sd_status st = check_attention(SD_ATTN_SPARSE, q, kv, batch,
-                                   stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail), &plan);
+                                   stream_hint(SD_ATTN_SPARSE, q, (long long)k + max_tail), &plan,
+                                   0, sparse_tc_tiles(kv, k, max_tail));
     if (st != SD_OK) return st;
     if (!plan.tensor_core) return SD_ERR_UNSUPPORTED;  // bf16, head_dim 64/128, <= 128 rows
     if (plan.ws_bytes > workspace_bytes || (plan.ws_bytes && !workspace)) return SD_ERR_WORKSPACE;
@@ -451,7 +500,7 @@ sd_status sd_sparse_attention_staged(const sd_q_desc *q, const void *q_data,
     p.k_sel = k;
     p.tail_begin = tail_begin;
     set_selection(p, const_cast<void *>(selection), sel_layout(0, kv, batch, k), k);
-    set_splits(p, plan.tc_splits);
+    set_tc_decomposition(p, plan);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = launch_attention_tc(p, plan, s);
     if (e == cudaErrorNotSupported) return SD_ERR_UNSUPPORTED;

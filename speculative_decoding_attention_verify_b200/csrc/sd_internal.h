@@ -44,6 +44,14 @@ struct AttnParams {
     float *ws_ml;  // [n_splits][rows_cap][h_q][2] (running max in log2 units, sum)
     int32_t *dev_err;
     unsigned long long wait_ns;  // bound of every pipeline wait inside the kernel
+    // persistent tensor-core decomposition (0: one CTA per (split, KV head, sequence)): every
+    // (sequence, KV head) unit is persist_s items (tile slots, unit-local tiles 0..persist_s-1,
+    // those past the unit's own tile count empty), and CTA i of persist_g takes the items
+    // [i N / persist_g, (i+1) N / persist_g) of all units in (sequence, KV head) order
+    // (N = units * persist_s).  A unit covered by one CTA gets its normalised output directly;
+    // otherwise the k-th CTA covering it writes partial slot k, merged by attn_merge_kernel.
+    int persist_s;
+    int persist_g;
 };
 
 // Decomposition of an attention call (host side; depends on host hints only).  Both the
@@ -52,6 +60,7 @@ struct AttnParams {
 struct AttnPlan {
     bool tensor_core;  // tcgen05 path preferred
     int tc_splits;
+    int tc_persist_s, tc_persist_g, tc_slots;  // persistent tcgen05 decomposition (0: classic)
     int simt_splits;
     int n_rowblocks;     // CUDA-core path
     int rows_per_block;  // CUDA-core path
@@ -66,14 +75,18 @@ unsigned long long wait_limit_ns();  // the process-wide bound set by sd_set_wai
 // workspace query knew only max_kv_len), the split counts are capped at those of the ws_stream
 // plan, so that the workspace it reported always suffices (the split model is not monotone in
 // the stream length).
+// tc_tiles: a bound of one unit's tiles on the tensor-core path (0: derived from the stream).
 AttnPlan plan_attention(int kind, int dtype, int head_dim, int h_q, int h_kv, int batch,
-                        int max_q_rows, long long max_stream, long long ws_stream = 0);
+                        int max_q_rows, long long max_stream, long long ws_stream = 0,
+                        bool paged = false, long long tc_tiles = 0);
 
 cudaError_t launch_attention_simt(const AttnParams &p, const AttnPlan &plan, cudaStream_t s);
 cudaError_t launch_attention_tc(const AttnParams &p, const AttnPlan &plan, cudaStream_t s);
 cudaError_t launch_sparse_compact(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_attention_merge(const AttnParams &p, cudaStream_t s);
 bool tc_supported(int kind, int dtype, int head_dim, int rows);
+bool tc_persistent_fits(int head_dim, int rows);  // shared memory of a persistent launch
+int tc_persistent_max_segments();                 // units one persistent CTA may touch
 
 // Top-K.
 struct TopkParams {
