@@ -155,6 +155,27 @@ SD_API sd_status sd_attention_workspace_size(sd_attn_kind kind, const sd_q_desc 
                                       const sd_kv_desc *kv, int32_t batch, size_t *bytes);
 
 /*
+ * How an attention call with these host hints is decomposed (host values only; device arrays
+ * are not read; nothing is launched).  *engine: SD_ENGINE_CUDA_CORE, SD_ENGINE_TC (tcgen05, one
+ * CTA per split of every (sequence, KV head) unit) or SD_ENGINE_TC_PERSISTENT (tcgen05, one CTA
+ * per SM over an even share of all units' tiles, long streams); *parts: the split count, or the
+ * persistent plan's partial slots per unit.  extent: a text-anchored call's max_window or a
+ * sparse call's k (ignored for verify); max_tail: a sparse call's hint (ignored otherwise).  The
+ * tensor-core engines also need 16-byte aligned q and out at the call (else CUDA cores run it).
+ * Returns SD_ERR_INVALID_ARG for invalid descriptors, SD_ERR_UNSUPPORTED for a head_dim other
+ * than 64 or 128.
+ */
+typedef enum {
+    SD_ENGINE_CUDA_CORE = 0,
+    SD_ENGINE_TC = 1,
+    SD_ENGINE_TC_PERSISTENT = 2
+} sd_attn_engine;
+
+SD_API sd_status sd_attention_plan(sd_attn_kind kind, const sd_q_desc *q, const sd_kv_desc *kv,
+                                   int32_t batch, int32_t extent, int32_t max_tail,
+                                   int32_t *engine, int32_t *parts);
+
+/*
  * Dense verification attention [StD "Procedimento de Decodificacao"]: the target scores the
  * gamma+1 new positions of every sequence in one pass over its full cache.  For every row i
  * of sequence b and query head h:

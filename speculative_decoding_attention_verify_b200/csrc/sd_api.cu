@@ -362,6 +362,45 @@ sd_status sd_attention_workspace_size(sd_attn_kind kind, const sd_q_desc *q,
     return SD_OK;
 }
 
+sd_status sd_attention_plan(sd_attn_kind kind, const sd_q_desc *q, const sd_kv_desc *kv,
+                            int32_t batch, int32_t extent, int32_t max_tail, int32_t *engine,
+                            int32_t *parts) {
+    if (!engine || !parts || !q || !kv) return SD_ERR_INVALID_ARG;
+    if (kind != SD_ATTN_VERIFY && kind != SD_ATTN_TEXT_ANCHORED && kind != SD_ATTN_SPARSE)
+        return SD_ERR_INVALID_ARG;
+    if (kv->h_kv < 1 || q->h_q < 1 || q->h_q % kv->h_kv || batch < 1 || q->max_q_rows < 1 ||
+        q->max_kv_len < 1 || extent < 0 || max_tail < 0 || extent > (1 << 30))
+        return SD_ERR_INVALID_ARG;
+    if (!head_dim_supported(kv->head_dim)) return SD_ERR_UNSUPPORTED;
+    const bool paged = kv->page_size != 0;
+    AttnPlan plan;
+    if (kind == SD_ATTN_VERIFY) {
+        plan = plan_attention(kind, kv->dtype, kv->head_dim, q->h_q, kv->h_kv, batch,
+                              q->max_q_rows, q->max_kv_len, 0, paged, 0);
+    } else if (kind == SD_ATTN_TEXT_ANCHORED) {
+        if (extent < 1) return SD_ERR_INVALID_ARG;
+        plan = plan_attention(kind, kv->dtype, kv->head_dim, q->h_q, kv->h_kv, batch,
+                              q->max_q_rows, stream_hint(kind, q, extent), q->max_kv_len, paged,
+                              0);
+    } else {
+        if (extent > (1 << 16)) return SD_ERR_INVALID_ARG;
+        plan = plan_attention(kind, kv->dtype, kv->head_dim, q->h_q, kv->h_kv, batch,
+                              q->max_q_rows, stream_hint(kind, q, (long long)extent + max_tail),
+                              0, paged, sparse_tc_tiles(kv, extent, max_tail));
+    }
+    if (!plan.tensor_core) {
+        *engine = SD_ENGINE_CUDA_CORE;
+        *parts = plan.simt_splits;
+    } else if (plan.tc_persist_s) {
+        *engine = SD_ENGINE_TC_PERSISTENT;
+        *parts = plan.tc_slots;
+    } else {
+        *engine = SD_ENGINE_TC;
+        *parts = plan.tc_splits;
+    }
+    return SD_OK;
+}
+
 sd_status sd_verify_attention(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
                               int32_t batch, void *out, void *workspace, size_t workspace_bytes,
                               int32_t *dev_err, void *stream) {

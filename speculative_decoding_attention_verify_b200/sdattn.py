@@ -12,7 +12,7 @@ import contextlib
 import ctypes
 import os
 import threading
-from typing import Optional
+from typing import Optional, Tuple
 
 import torch
 
@@ -21,6 +21,7 @@ from . import build as _build
 SD_OK, SD_ERR_INVALID_ARG, SD_ERR_UNSUPPORTED, SD_ERR_WORKSPACE, SD_ERR_CUDA = range(5)
 SD_F32, SD_BF16 = 0, 1
 SD_ATTN_VERIFY, SD_ATTN_TEXT_ANCHORED, SD_ATTN_SPARSE = 0, 1, 2
+SD_ENGINE_CUDA_CORE, SD_ENGINE_TC, SD_ENGINE_TC_PERSISTENT = 0, 1, 2
 SD_TOPK_LAST_QUERY, SD_TOPK_MEAN_TEXT_ATTENTION = 0, 1
 SD_DEVERR_PAGE, SD_DEVERR_INDEX, SD_DEVERR_TOKEN, SD_DEVERR_NUMERIC, SD_DEVERR_SHAPE = 1, 2, 4, 8, 16
 SD_DEVERR_TIMEOUT = 32
@@ -57,7 +58,7 @@ EXPORTS = ("sd_status_string", "sd_version", "sd_attention_workspace_size", "sd_
            "sd_accept_sample", "sd_verify_attention_noalloc", "sd_sparse_workspace_size",
            "sd_sparse_selection_size", "sd_sparse_stage", "sd_sparse_attention_staged",
            "sd_topk_scored_workspace_size", "sd_topk_select_scored", "sd_set_wait_timeout_ns",
-           "sd_draft_layer_workspace_size", "sd_draft_layer")
+           "sd_draft_layer_workspace_size", "sd_draft_layer", "sd_attention_plan")
 
 # Size of the library's fixed scratch used by sd_verify_attention_noalloc.
 SD_VERIFY_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -82,6 +83,8 @@ def lib():
                 h.sd_set_wait_timeout_ns.restype = ctypes.c_uint64
                 h.sd_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
                 h.sd_attention_workspace_size.argtypes = [ctypes.c_int, P, P, I32, ctypes.POINTER(SZ)]
+                h.sd_attention_plan.argtypes = [ctypes.c_int, P, P, I32, I32, I32,
+                                                ctypes.POINTER(I32), ctypes.POINTER(I32)]
                 h.sd_verify_attention.argtypes = [P, P, P, I32, P, P, SZ, P, P]
                 h.sd_text_anchored_attention.argtypes = [P, P, P, I32, P, P, P, I32, P, P, SZ, P, P]
                 h.sd_sparse_attention.argtypes = [P, P, P, I32, P, I32, P, I32, P, P, SZ, P, P]
@@ -227,6 +230,17 @@ def sd_attention_workspace_size(kind: int, q: Queries, kv: KVCache) -> int:
     _check(lib().sd_attention_workspace_size(kind, ctypes.byref(q.desc), ctypes.byref(kv.desc),
                                              kv.batch, ctypes.byref(n)), "sd_attention_workspace_size")
     return n.value
+
+
+def sd_attention_plan(kind: int, q: Queries, kv: KVCache, extent: int = 0,
+                      max_tail: int = 0) -> Tuple[int, int]:
+    """(engine, parts) of an attention call with these hints: SD_ENGINE_* and the split count
+    (or the persistent plan's partial slots).  extent: max_window (text-anchored) or k (sparse)."""
+    e, n = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib().sd_attention_plan(kind, ctypes.byref(q.desc), ctypes.byref(kv.desc), kv.batch,
+                                   int(extent), int(max_tail), ctypes.byref(e), ctypes.byref(n)),
+           "sd_attention_plan")
+    return e.value, n.value
 
 
 def _attn_out(q: Queries, out):

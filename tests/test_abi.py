@@ -170,3 +170,48 @@ def test_wait_timeout_setting_round_trips():
     assert sd.sd_set_wait_timeout_ns(0) == 5000   # 0 restores the default ...
     assert sd.sd_set_wait_timeout_ns(0) == 10**9  # ... which is what is now set
     assert lib.sd_version() >= 200
+
+
+def _plan(kind, q, kv, batch, extent=0, max_tail=0):
+    e, n = ctypes.c_int32(-1), ctypes.c_int32(-1)
+    st = sd.lib().sd_attention_plan(kind, ctypes.byref(q), ctypes.byref(kv), batch, extent,
+                                    max_tail, ctypes.byref(e), ctypes.byref(n))
+    return st, e.value, n.value
+
+
+def test_attention_plan_picks_the_decomposition():
+    """Host-only planning (148 SMs assumed without a device): long streams over many units get
+    the persistent tensor-core decomposition, the short draft calls the per-unit one, fp32 and
+    more than 128 rows per KV head the CUDA-core engine; the workspace covers the plan."""
+    # 28 layers x 9 rows x 7 heads per KV head over 26,033 positions: persistent
+    q, kv = _descs(max_q=9, max_kv=26033)
+    st, eng, parts = _plan(sd.SD_ATTN_VERIFY, q, kv, 28)
+    assert st == sd.SD_OK and eng == sd.SD_ENGINE_TC_PERSISTENT and 2 <= parts <= 8
+    n = ctypes.c_size_t(0)
+    assert sd.lib().sd_attention_workspace_size(sd.SD_ATTN_VERIFY, ctypes.byref(q),
+                                                ctypes.byref(kv), 28, ctypes.byref(n)) == 0
+    assert n.value >= parts * 28 * 9 * 28 * (128 + 2) * 4
+    # one layer: the per-unit kernel with splits
+    st, eng, parts = _plan(sd.SD_ATTN_VERIFY, q, kv, 1)
+    assert st == sd.SD_OK and eng == sd.SD_ENGINE_TC and parts > 1
+    # the draft calls of the benchmark cycle: per-unit, one split
+    q1, kv1 = _descs(max_q=1, max_kv=26025)
+    assert _plan(sd.SD_ATTN_TEXT_ANCHORED, q1, kv1, 28, extent=1024)[1:] == (sd.SD_ENGINE_TC, 1)
+    assert _plan(sd.SD_ATTN_SPARSE, q1, kv1, 28, extent=1024, max_tail=1025)[1:] == \
+        (sd.SD_ENGINE_TC, 1)
+    # a large selection or a wide window make the draft streams long: persistent
+    assert _plan(sd.SD_ATTN_SPARSE, q1, kv1, 28, extent=8192, max_tail=1025)[1] == \
+        sd.SD_ENGINE_TC_PERSISTENT
+    assert _plan(sd.SD_ATTN_TEXT_ANCHORED, q1, kv1, 28, extent=8000)[1] == \
+        sd.SD_ENGINE_TC_PERSISTENT
+    # fp32 caches and more than 128 rows per KV head: CUDA cores
+    qf, kvf = _descs(dtype=sd.SD_F32, max_q=9, max_kv=26033)
+    assert _plan(sd.SD_ATTN_VERIFY, qf, kvf, 28)[1] == sd.SD_ENGINE_CUDA_CORE
+    qr, kvr = _descs(max_q=20, max_kv=26033)
+    assert _plan(sd.SD_ATTN_VERIFY, qr, kvr, 28)[1] == sd.SD_ENGINE_CUDA_CORE
+    # host validation
+    assert _plan(7, q, kv, 28)[0] == sd.SD_ERR_INVALID_ARG
+    assert _plan(sd.SD_ATTN_TEXT_ANCHORED, q1, kv1, 28, extent=0)[0] == sd.SD_ERR_INVALID_ARG
+    assert _plan(sd.SD_ATTN_VERIFY, q, kv, 0)[0] == sd.SD_ERR_INVALID_ARG
+    qd, kvd = _descs(d=96)
+    assert _plan(sd.SD_ATTN_VERIFY, qd, kvd, 2)[0] == sd.SD_ERR_UNSUPPORTED
