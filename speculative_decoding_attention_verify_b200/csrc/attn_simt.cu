@@ -359,59 +359,49 @@ attn_simt_kernel(const AttnParams p) {
 }
 
 // Combine the splits of every (row, head): O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-// One warp per (row, head); lanes read the splits' statistics in parallel.
+// One warp per (sequence, row of the sequence, head), so a row's sequence is known without a
+// search.  Lanes read the splits' statistics in parallel, and the first four splits' partial
+// outputs are loaded in the same round trip (their weights are applied once the maximum is
+// known).
 template <bool BF16, int D>
 __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
     constexpr int EPL = D / 32;
+    constexpr int kPre = 4;  // splits whose outputs are loaded with the statistics
     const int lane = threadIdx.x & 31;
     const int64_t gw = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-    const int row = (int)(gw / p.h_q), h = (int)(gw % p.h_q);
-    const int total = __ldg(p.q_start + p.batch);
-    if (row >= total || row >= p.rows_cap) return;
+    const int64_t per_seq = (int64_t)p.max_q_rows * p.h_q;
+    const int b = (int)(gw / per_seq);
+    if (b >= p.batch) return;
+    const int i = (int)((gw % per_seq) / p.h_q), h = (int)(gw % p.h_q);
+    const int q0 = __ldg(p.q_start + b);
+    if (i >= __ldg(p.q_start + b + 1) - q0) return;
+    const int row = q0 + i;
+    if (row >= p.rows_cap) return;
     const int64_t stride = (int64_t)p.rows_cap * p.h_q;  // between splits, in (row, head) units
     const int64_t rh = (int64_t)row * p.h_q + h;
     int n_splits = p.n_splits;
     if (p.persist_s) {
         // Persistent tensor-core decomposition: the CTAs whose item ranges meet the row's unit
         // wrote slots 0.. in order; a unit inside one CTA's range has its output already.
-        // the row's sequence: the last b with q_start[b] <= row, found by the warp in two
-        // ballots (32 strided entries, then up to 32 entries of the chosen stretch), or by
-        // bisection beyond 1,024 sequences
-        int lo = 0;
-        if (p.batch <= 1024) {
-            const int bs = (p.batch + 31) / 32;
-            const bool in1 = lane * bs < p.batch;
-            unsigned m = __ballot_sync(
-                0xffffffffu, in1 && __ldg(p.q_start + (in1 ? lane * bs : 0)) <= row);
-            if (m == 0) return;  // a row before the first sequence's
-            const int base_b = (31 - __clz(m)) * bs;
-            const bool in2 = lane < bs && base_b + lane < p.batch;
-            m = __ballot_sync(0xffffffffu,
-                              in2 && __ldg(p.q_start + (in2 ? base_b + lane : 0)) <= row);
-            lo = base_b + (31 - __clz(m));
-        } else {
-            int hi = p.batch - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) / 2;
-                if (__ldg(p.q_start + mid) <= row)
-                    lo = mid;
-                else
-                    hi = mid - 1;
-            }
-        }
         const long long n_items = (long long)p.batch * p.kv.h_kv * p.persist_s;
-        const long long base = ((long long)lo * p.kv.h_kv + h / p.group) * p.persist_s;
+        const long long base = ((long long)b * p.kv.h_kv + h / p.group) * p.persist_s;
         const int c0 = (int)(((base + 1) * p.persist_g - 1) / n_items);
         const int c1 = (int)(((base + p.persist_s) * p.persist_g - 1) / n_items);
         if (c1 == c0) return;
         n_splits = min(c1 - c0 + 1, p.n_splits);
     }
-    float o[EPL];
+    float ov[kPre][EPL];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) o[e] = 0.f;
+    for (int k = 0; k < kPre; ++k)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e)
+            ov[k][e] = k < n_splits ? p.ws_o[((int64_t)k * stride + rh) * D + lane * EPL + e] : 0.f;
     float M = -INFINITY;
     for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, p.ws_ml[(s * stride + rh) * 2]);
     M = warp_max(M);
+    float o[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) o[e] = 0.f;
     float den = 0.f;
     if (M != -INFINITY) {
         for (int s0 = 0; s0 < n_splits; s0 += 32) {
@@ -424,25 +414,20 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
             }
             den += warp_sum(w * l);
             const int n = min(32, n_splits - s0);
-            int i = 0;
-            for (; i + 4 <= n; i += 4) {
-                float ov[4][EPL];
-                float wv[4];
+            int k = 0;
+            if (s0 == 0) {  // the preloaded splits
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    wv[k] = __shfl_sync(0xffffffffu, w, i + k);
-                    const float *src = p.ws_o + ((s0 + i + k) * stride + rh) * D + lane * EPL;
+                for (int q = 0; q < kPre; ++q) {
+                    const float wq = __shfl_sync(0xffffffffu, w, q);
+                    if (q < n)
 #pragma unroll
-                    for (int e = 0; e < EPL; ++e) ov[k][e] = src[e];
+                        for (int e = 0; e < EPL; ++e) o[e] += wq * ov[q][e];
                 }
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) o[e] += wv[k] * ov[k][e];
+                k = min(kPre, n);
             }
-            for (; i < n; ++i) {
-                const float wk = __shfl_sync(0xffffffffu, w, i);
-                const float *src = p.ws_o + ((s0 + i) * stride + rh) * D + lane * EPL;
+            for (; k < n; ++k) {
+                const float wk = __shfl_sync(0xffffffffu, w, k);
+                const float *src = p.ws_o + ((s0 + k) * stride + rh) * D + lane * EPL;
 #pragma unroll
                 for (int e = 0; e < EPL; ++e) o[e] += wk * src[e];
             }
