@@ -358,7 +358,7 @@ SD_API sd_status sd_hsr_project(const void *emb, const void *hid, int32_t n_rows
  * [out][in]: w_hsr [d_model][2 d_model], ln1 / ln2 [d_model], w_qkv [(h_q + 2 h_kv) head_dim]
  * [d_model] (query heads, then key heads, then value heads), b_qkv [(h_q + 2 h_kv) head_dim] or
  * NULL, w_o [d_model][h_q head_dim], w_gate_up [2 d_ff][d_model] (the gate rows, then the up
- * rows), w_down [d_model][d_ff]; the big matrices 16-byte aligned.
+ * rows), w_down [d_model][d_ff]; the matrices and the two norm weights 16-byte aligned.
  */
 typedef struct {
     int32_t d_model, h_q, h_kv, head_dim, d_ff;

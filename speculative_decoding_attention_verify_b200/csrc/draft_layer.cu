@@ -9,14 +9,17 @@
 //             plain     a bf16 vector                          (the attention output)
 //   epilogue  f32       fp32 out (+ bias) (+ fp32 residual)
 //             bf16res   bf16 out = acc + fp32 residual         (the layer's output)
-//             qkv       + bias; RoPE on the query and key heads (pairs (i, i + d/2), computed by
-//                       the same warp), queries to a bf16 buffer, keys and values written into
-//                       the cache at the rows' positions
-// One warp per output row (a row pair for qkv), lanes over the row's 16-byte chunks with eight
-// loads in flight, the rows spread over every warp of a grid of one 16-warp CTA per SM, so that
-// every SM streams about the same share of the weights.  The input vector is rebuilt by every
-// CTA (it is tiny beside the weights).  The attention step is the library's own text-anchored
-// attention call on the draft's text-only cache.
+//             qkv       + bias; RoPE on the query and key heads (pairs (i, i + d/2), one unit
+//                       of work), queries to a bf16 buffer, keys and values written into the
+//                       cache at the rows' positions
+// One 16-warp CTA per SM owns an even share of the output rows (of row pairs for qkv) and cuts
+// each row into P parts (items), P chosen so that every warp gets several items of at least a
+// few KB (the down projection's 18,944-weight rows spread over all warps instead of one warp per
+// row).  Each warp streams two items at a time (seven 16-byte loads per lane per item in
+// flight) and stores one partial per (item, input row); the parts of a row are then summed in a
+// fixed order (deterministic) and finished by the epilogue.  The input vector is rebuilt by
+// every CTA (it is tiny beside the weights).  The attention step is the library's own
+// text-anchored attention call on the draft's text-only cache.
 #include "sd_internal.h"
 
 namespace sd {
@@ -26,7 +29,7 @@ constexpr int kDlThreads = 512;  // 16 warps
 constexpr int kDlWarps = kDlThreads / 32;
 constexpr int kDlMaxRows = 4;
 constexpr int kDlSmemMax = 200 * 1024;  // the input vectors of every row, bf16
-constexpr int kUnroll = 8;  // 16-byte weight loads in flight per lane
+constexpr int kDlSmemOptIn = 226 * 1024;  // dynamic shared memory a launch may use
 
 enum { IN_CONCAT = 0, IN_NORM = 1, IN_SWIGLU = 2, IN_PLAIN = 3 };
 enum { OUT_F32 = 0, OUT_BF16_RES = 1, OUT_QKV = 2 };
@@ -52,6 +55,7 @@ struct GemvArgs {
     int32_t *params;       // qkv: [q_start0, q_start1, vis_b, vis_e, window] for the attention
     int window;
     int32_t *dev_err;
+    int parts;             // items per weight row (chosen by the host)
 };
 
 __device__ __forceinline__ float silu(float t) { return t / (1.f + __expf(-t)); }
@@ -72,11 +76,28 @@ __device__ __forceinline__ void build_input(const GemvArgs &a, uint16_t *s_x, fl
                 *reinterpret_cast<const uint4 *>(src);
         }
     } else if constexpr (IN == IN_NORM) {
-        // 1 / sqrt(mean(x^2) + eps) per row: a block reduction in a fixed order
+        // 1 / sqrt(mean(x^2) + eps) per row: a block reduction in a fixed order.  The fp32
+        // inputs are read as float4, four per thread in flight (the loads, not the arithmetic,
+        // set the time of this prologue).
+        const int k4 = k / 4;
         for (int r = 0; r < a.n; ++r) {
+            const float4 *x4 = reinterpret_cast<const float4 *>(a.in_f + (int64_t)r * k);
             float ss = 0.f;
-            const float *x = a.in_f + (int64_t)r * k;
-            for (int i = tid; i < k; i += kDlThreads) ss = fmaf(x[i], x[i], ss);
+            for (int e0 = tid; e0 < k4; e0 += 4 * kDlThreads) {
+                float4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + u * kDlThreads;
+                    v[u] = e < k4 ? x4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    ss = fmaf(v[u].x, v[u].x, ss);
+                    ss = fmaf(v[u].y, v[u].y, ss);
+                    ss = fmaf(v[u].z, v[u].z, ss);
+                    ss = fmaf(v[u].w, v[u].w, ss);
+                }
+            }
             ss = warp_sum(ss);
             if ((tid & 31) == 0) s_red[tid >> 5] = ss;
             __syncthreads();
@@ -87,71 +108,66 @@ __device__ __forceinline__ void build_input(const GemvArgs &a, uint16_t *s_x, fl
             }
             __syncthreads();
         }
-        for (int e = tid; e < a.n * k; e += kDlThreads) {
-            const int r = e / k, i = e % k;
-            const float g = __uint_as_float((uint32_t)a.gamma[i] << 16);
-            s_x[e] = (uint16_t)f32_to_bf16_bits(a.in_f[(int64_t)r * k + i] * s_red[kDlWarps + r] *
-                                                g);
+        for (int e0 = tid; e0 < a.n * k4; e0 += 4 * kDlThreads) {
+            float4 v[4];
+            uint2 gm[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * kDlThreads;
+                const bool in = e < a.n * k4;
+                v[u] = in ? reinterpret_cast<const float4 *>(a.in_f)[e]
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                gm[u] = in ? reinterpret_cast<const uint2 *>(a.gamma)[e % k4] : make_uint2(0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * kDlThreads;
+                if (e >= a.n * k4) break;
+                const float sc = s_red[kDlWarps + e / k4];
+                const uint32_t lo = f32_to_bf16_bits(v[u].x * sc * bf16_lo(gm[u].x)) |
+                                    (f32_to_bf16_bits(v[u].y * sc * bf16_hi(gm[u].x)) << 16);
+                const uint32_t hi = f32_to_bf16_bits(v[u].z * sc * bf16_lo(gm[u].y)) |
+                                    (f32_to_bf16_bits(v[u].w * sc * bf16_hi(gm[u].y)) << 16);
+                reinterpret_cast<uint2 *>(s_x)[e] = make_uint2(lo, hi);
+            }
         }
-    } else {  // swiglu: gate/up [n][2k]
-        for (int e = tid; e < a.n * k; e += kDlThreads) {
-            const int r = e / k, i = e % k;
-            const float gt = a.in_f[(int64_t)r * 2 * k + i];
-            const float up = a.in_f[(int64_t)r * 2 * k + k + i];
-            s_x[e] = (uint16_t)f32_to_bf16_bits(silu(gt) * up);
+    } else {  // swiglu: gate/up [n][2k], read as float4, four per thread in flight
+        const int k4 = k / 4;
+        for (int e0 = tid; e0 < a.n * k4; e0 += 4 * kDlThreads) {
+            float4 gt[4], up[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * kDlThreads;
+                const bool in = e < a.n * k4;
+                const int r = in ? e / k4 : 0, i = in ? e % k4 : 0;
+                const float4 *row = reinterpret_cast<const float4 *>(a.in_f + (int64_t)r * 2 * k);
+                gt[u] = in ? row[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                up[u] = in ? row[k4 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * kDlThreads;
+                if (e >= a.n * k4) break;
+                const uint32_t lo = f32_to_bf16_bits(silu(gt[u].x) * up[u].x) |
+                                    (f32_to_bf16_bits(silu(gt[u].y) * up[u].y) << 16);
+                const uint32_t hi = f32_to_bf16_bits(silu(gt[u].z) * up[u].z) |
+                                    (f32_to_bf16_bits(silu(gt[u].w) * up[u].w) << 16);
+                reinterpret_cast<uint2 *>(s_x)[e] = make_uint2(lo, hi);
+            }
         }
     }
     __syncthreads();
 }
 
-// acc[r] += w_row . x_r over the row's chunks this lane owns (fp32).
-template <int NR>
-__device__ __forceinline__ void dot_row(const uint16_t *w_row, const uint16_t *s_x, int k, int n,
-                                        int lane, float (&acc)[NR]) {
-    const int chunks = k / 8;
-    const uint4 *wr = reinterpret_cast<const uint4 *>(w_row);
-    for (int c0 = lane; c0 < chunks; c0 += 32 * kUnroll) {
-        uint4 wv[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int c = c0 + 32 * u;
-            wv[u] = c < chunks ? ldg_stream16(wr + c) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int c = c0 + 32 * u;
-            if (c >= chunks) break;
-            float wf[8];
-            Chunk<true>::to_float(wv[u], wf);
-#pragma unroll
-            for (int r = 0; r < NR; ++r) {
-                if (r >= n) break;
-                float xf[8];
-                Chunk<true>::to_float(*reinterpret_cast<const uint4 *>(s_x + (int64_t)r * k + c * 8),
-                                      xf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[r] = fmaf(wf[e], xf[e], acc[r]);
-            }
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < NR; ++r) acc[r] = warp_sum(acc[r]);
-}
+constexpr int kItemLoads = 7;  // 16-byte loads per lane per item in flight
 
-// Lane r finishes row r of a QKV row pair (h, i) / (h, i + d/2): bias, RoPE for query and key
-// heads (angle in double: positions reach 1e5 radians), then the query buffer or the cache.
-template <int NR>
+// Finishes a QKV row pair (h, i) / (h, i + d/2) of input row r from its two dot products: bias,
+// RoPE for query and key heads (angle in double: positions reach 1e5 radians), then the query
+// buffer or the cache.
 __device__ __forceinline__ void finish_qkv(const GemvArgs &a, int h, int i, int kv_len, int r,
-                                           const float (&acc1)[NR], const float (&acc2)[NR]) {
+                                           float v1, float v2) {
     const int half = a.d / 2;
     const int o1 = h * a.d + i, o2 = o1 + half;
-    float v1 = acc1[0], v2 = acc2[0];
-#pragma unroll
-    for (int q = 1; q < NR; ++q)
-        if (r == q) {
-            v1 = acc1[q];
-            v2 = acc2[q];
-        }
     if (a.bias) {
         v1 += __uint_as_float((uint32_t)a.bias[o1] << 16);
         v2 += __uint_as_float((uint32_t)a.bias[o2] << 16);
@@ -183,14 +199,9 @@ __device__ __forceinline__ void finish_qkv(const GemvArgs &a, int h, int i, int 
     }
 }
 
-// Lane r finishes output o of row r: bias, residual, fp32 or bf16 store.
-template <int OUT, int NR>
-__device__ __forceinline__ void finish_row(const GemvArgs &a, int o, int r,
-                                           const float (&acc)[NR]) {
-    float v = acc[0];
-#pragma unroll
-    for (int q = 1; q < NR; ++q)
-        if (r == q) v = acc[q];
+// Finishes output o of input row r: bias, residual, fp32 or bf16 store.
+template <int OUT>
+__device__ __forceinline__ void finish_row(const GemvArgs &a, int o, int r, float v) {
     if (a.bias) v += __uint_as_float((uint32_t)a.bias[o] << 16);
     if (a.res) v += a.res[(int64_t)r * a.m + o];
     if (OUT == OUT_F32)
@@ -199,48 +210,148 @@ __device__ __forceinline__ void finish_row(const GemvArgs &a, int o, int r,
         a.out_b[(int64_t)r * a.m + o] = (uint16_t)f32_to_bf16_bits(v);
 }
 
+// Units of a GEMV: output rows, or (for qkv) row pairs (h, i) / (h, i + d/2).
+template <int OUT>
+__host__ __device__ __forceinline__ int gemv_units(const GemvArgs &a) {
+    return OUT == OUT_QKV ? (a.h_q + 2 * a.h_kv) * (a.d / 2) : a.m;
+}
+
 template <int IN, int OUT>
 __global__ void __launch_bounds__(kDlThreads, 1) draft_gemv_kernel(const GemvArgs a) {
-    extern __shared__ __align__(16) uint16_t s_x[];
+    constexpr int RU = OUT == OUT_QKV ? 2 : 1;  // weight rows per unit
+    constexpr int NR = kDlMaxRows;
+    extern __shared__ __align__(16) uint16_t s_x[];  // [n][k] bf16, then [items][NR] f32
     __shared__ float s_red[kDlWarps + kDlMaxRows];
-    build_input<IN>(a, s_x, s_red);
-    const int lane = threadIdx.x & 31;
-    const int gw = blockIdx.x * kDlWarps + (threadIdx.x >> 5);
-    const int n_warps = gridDim.x * kDlWarps;
-    if (OUT == OUT_QKV && blockIdx.x == 0 && threadIdx.x == 0) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (OUT == OUT_QKV && blockIdx.x == 0 && tid == 0) {
         a.params[0] = 0;
         a.params[1] = a.n;
         a.params[2] = 0;
         a.params[3] = 0;
         a.params[4] = a.window;
     }
-    if constexpr (OUT == OUT_QKV) {
-        const int half = a.d / 2;
-        const int heads = a.h_q + 2 * a.h_kv;
-        const int items = heads * half;
-        const int kv_len = __ldg(a.kv.kv_len);
-        for (int it = gw; it < items; it += n_warps) {
-            const int h = it / half, i = it % half;
-            const int o1 = h * a.d + i, o2 = o1 + half;
-            float acc1[kDlMaxRows] = {}, acc2[kDlMaxRows] = {};
-            dot_row<kDlMaxRows>(a.w + (int64_t)o1 * a.k, s_x, a.k, a.n, lane, acc1);
-            dot_row<kDlMaxRows>(a.w + (int64_t)o2 * a.k, s_x, a.k, a.n, lane, acc2);
-            if (lane < a.n) finish_qkv(a, h, i, kv_len, lane, acc1, acc2);
+    const int U = gemv_units<OUT>(a);
+    const int u0 = (int)((int64_t)U * blockIdx.x / gridDim.x);
+    const int u1 = (int)((int64_t)U * (blockIdx.x + 1) / gridDim.x);
+    const int P = a.parts;
+    const int items = (u1 - u0) * RU * P;
+    const int cpr = a.k / 8;  // 16-byte chunks per weight row
+    float *s_part = reinterpret_cast<float *>(s_x + (size_t)a.n * a.k);
+    build_input<IN>(a, s_x, s_red);  // (ends with a block barrier)
+    // weight row of local item it, and its chunk range [c_lo, c_hi)
+    auto item_row = [&](int it, int &c_lo, int &c_hi) -> const uint4 * {
+        const int u = u0 + it / (RU * P), rr = (it / P) % RU, part = it % P;
+        int row;
+        if constexpr (OUT == OUT_QKV) {
+            const int half = a.d / 2;
+            row = (u / half) * a.d + u % half + rr * half;
+        } else {
+            row = u;
         }
-    } else {
-        for (int o = gw; o < a.m; o += n_warps) {
-            float acc[kDlMaxRows] = {};
-            dot_row<kDlMaxRows>(a.w + (int64_t)o * a.k, s_x, a.k, a.n, lane, acc);
-            if (lane < a.n) finish_row<OUT>(a, o, lane, acc);
+        c_lo = (int)((int64_t)cpr * part / P);
+        c_hi = (int)((int64_t)cpr * (part + 1) / P);
+        return reinterpret_cast<const uint4 *>(a.w + (int64_t)row * a.k);
+    };
+    for (int it0 = warp; it0 < items; it0 += 2 * kDlWarps) {
+        const int its[2] = {it0, it0 + kDlWarps};
+        const uint4 *wr[2];
+        int lo[2], hi[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            lo[k] = hi[k] = 0;
+            wr[k] = its[k] < items ? item_row(its[k], lo[k], hi[k]) : nullptr;
         }
+        float part[2][NR];
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int r = 0; r < NR; ++r) part[k][r] = 0.f;
+        const int span = max(hi[0] - lo[0], hi[1] - lo[1]);
+        for (int c0 = lane; c0 < span; c0 += 32 * kItemLoads) {
+            uint4 wv[2][kItemLoads];
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+#pragma unroll
+                for (int u = 0; u < kItemLoads; ++u) {
+                    const int c = lo[k] + c0 + 32 * u;
+                    wv[k][u] = c < hi[k] ? ldg_stream16(wr[k] + c) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+#pragma unroll
+                for (int u = 0; u < kItemLoads; ++u) {
+                    const int c = lo[k] + c0 + 32 * u;
+                    if (c >= hi[k]) break;
+                    float wf[8];
+                    Chunk<true>::to_float(wv[k][u], wf);
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) {
+                        if (r >= a.n) break;
+                        float xf[8];
+                        Chunk<true>::to_float(
+                            *reinterpret_cast<const uint4 *>(s_x + (int64_t)r * a.k + c * 8), xf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) part[k][r] = fmaf(wf[e], xf[e], part[k][r]);
+                    }
+                }
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const float sum = warp_sum(part[k][r]);
+                if (lane == 0 && its[k] < items) s_part[its[k] * NR + r] = sum;
+            }
+    }
+    __syncthreads();
+    // epilogue: thread per (unit, input row); the unit's parts summed in a fixed order
+    const int kv_len = OUT == OUT_QKV ? __ldg(a.kv.kv_len) : 0;
+    for (int e = tid; e < (u1 - u0) * a.n; e += kDlThreads) {
+        const int lu = e / a.n, r = e % a.n, u = u0 + lu;
+        float v[RU];
+#pragma unroll
+        for (int rr = 0; rr < RU; ++rr) {
+            float acc = 0.f;
+            for (int q = 0; q < P; ++q) acc += s_part[((lu * RU + rr) * P + q) * NR + r];
+            v[rr] = acc;
+        }
+        if constexpr (OUT == OUT_QKV)
+            finish_qkv(a, u / (a.d / 2), u % (a.d / 2), kv_len, r, v[0], v[RU - 1]);
+        else
+            finish_row<OUT>(a, u, r, v[0]);
     }
 }
 
+// Parts per weight row: doubled (up to 8) while a CTA would hold fewer than six items per warp
+// and each part keeps at least 64 chunks per half (so two loads per lane stay in flight).
+template <int OUT>
+int gemv_parts(const GemvArgs &a, int ctas) {
+    const int ru = OUT == OUT_QKV ? 2 : 1;
+    const int units_max = (gemv_units<OUT>(a) + ctas - 1) / ctas;
+    const int cpr = a.k / 8;
+    int p = 1;
+    while (p < 8 && units_max * ru * p < 6 * kDlWarps && cpr / (2 * p * 2) >= 64) p *= 2;
+    return p;
+}
+
+// Dynamic shared memory of a launch: the input vectors and the partials.
+template <int OUT>
+size_t gemv_smem(const GemvArgs &a, int ctas) {
+    const int ru = OUT == OUT_QKV ? 2 : 1;
+    const int units_max = (gemv_units<OUT>(a) + ctas - 1) / ctas;
+    return (size_t)a.n * a.k * 2 + (size_t)units_max * ru * a.parts * kDlMaxRows * 4;
+}
+
 template <int IN, int OUT>
-cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s) {
-    cudaError_t e = set_max_dynamic_smem<draft_gemv_kernel<IN, OUT>>(kDlSmemMax);
+cudaError_t launch_gemv(GemvArgs a, cudaStream_t s) {
+    // (the opt-in leaves room for the kernel's static shared memory within the 227 KB)
+    cudaError_t e = set_max_dynamic_smem<draft_gemv_kernel<IN, OUT>>(kDlSmemOptIn);
     if (e != cudaSuccess) return e;
-    draft_gemv_kernel<IN, OUT><<<device_sm_count(), kDlThreads, a.n * a.k * 2, s>>>(a);
+    const int ctas = device_sm_count();
+    a.parts = gemv_parts<OUT>(a, ctas);
+    const size_t smem = gemv_smem<OUT>(a, ctas);
+    if (smem > (size_t)kDlSmemOptIn) return cudaErrorInvalidValue;
+    draft_gemv_kernel<IN, OUT><<<ctas, kDlThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -285,6 +396,7 @@ bool layer_desc_ok(const sd_draft_layer_desc *w, int n) {
     if (!w->w_hsr || !w->ln1 || !w->w_qkv || !w->w_o || !w->ln2 || !w->w_gate_up || !w->w_down)
         return false;
     const uintptr_t al = reinterpret_cast<uintptr_t>(w->w_hsr) |
+                         reinterpret_cast<uintptr_t>(w->ln1) | reinterpret_cast<uintptr_t>(w->ln2) |
                          reinterpret_cast<uintptr_t>(w->w_qkv) |
                          reinterpret_cast<uintptr_t>(w->w_o) |
                          reinterpret_cast<uintptr_t>(w->w_gate_up) |
