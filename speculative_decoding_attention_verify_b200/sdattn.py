@@ -213,10 +213,12 @@ class Queries:
         return self.q.shape[0]
 
 
-def _workspace(nbytes: int, device, given: Optional[torch.Tensor]):
+def _workspace(nbytes, device, given: Optional[torch.Tensor]):
+    """The caller's workspace (the library checks its size), or a new one of nbytes() bytes (the
+    size query only runs when a workspace has to be allocated)."""
     if given is not None:
         return given
-    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+    return torch.empty(max(int(nbytes()), 16), dtype=torch.uint8, device=device)
 
 
 def sd_set_wait_timeout_ns(ns: int) -> int:
@@ -250,7 +252,7 @@ def _attn_out(q: Queries, out):
 def sd_verify_attention(q: Queries, kv: KVCache, out=None, workspace=None, dev_err=None,
                         stream=None) -> torch.Tensor:
     out = _attn_out(q, out)
-    ws = _workspace(sd_attention_workspace_size(SD_ATTN_VERIFY, q, kv), q.q.device, workspace)
+    ws = _workspace(lambda: sd_attention_workspace_size(SD_ATTN_VERIFY, q, kv), q.q.device, workspace)
     with _on(q.q):
         _check(lib().sd_verify_attention(ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc),
                                          kv.batch, _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
@@ -275,7 +277,7 @@ def sd_text_anchored_attention(q: Queries, kv: KVCache, vis_begin, vis_end, wind
                                max_window: int, out=None, workspace=None, dev_err=None,
                                stream=None) -> torch.Tensor:
     out = _attn_out(q, out)
-    ws = _workspace(sd_attention_workspace_size(SD_ATTN_TEXT_ANCHORED, q, kv), q.q.device, workspace)
+    ws = _workspace(lambda: sd_attention_workspace_size(SD_ATTN_TEXT_ANCHORED, q, kv), q.q.device, workspace)
     with _on(q.q):
         _check(lib().sd_text_anchored_attention(
             ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(vis_begin),
@@ -287,7 +289,7 @@ def sd_text_anchored_attention(q: Queries, kv: KVCache, vis_begin, vis_end, wind
 def sd_sparse_attention(q: Queries, kv: KVCache, idx: torch.Tensor, tail_begin, max_tail: int,
                         out=None, workspace=None, dev_err=None, stream=None) -> torch.Tensor:
     out = _attn_out(q, out)
-    ws = _workspace(sd_sparse_workspace_size(q, kv, int(idx.shape[-1]), max_tail), q.q.device,
+    ws = _workspace(lambda: sd_sparse_workspace_size(q, kv, int(idx.shape[-1]), max_tail), q.q.device,
                     workspace)
     with _on(q.q):
         _check(lib().sd_sparse_attention(
@@ -330,7 +332,7 @@ def sd_sparse_attention_staged(q: Queries, kv: KVCache, selection: torch.Tensor,
                                tail_begin, max_tail: int, out=None, workspace=None, dev_err=None,
                                stream=None) -> torch.Tensor:
     out = _attn_out(q, out)
-    ws = _workspace(sd_sparse_workspace_size(q, kv, k, max_tail), q.q.device, workspace)
+    ws = _workspace(lambda: sd_sparse_workspace_size(q, kv, k, max_tail), q.q.device, workspace)
     with _on(q.q):
         _check(lib().sd_sparse_attention_staged(
             ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(selection),
@@ -350,7 +352,7 @@ def sd_topk_select(q: Queries, kv: KVCache, cand_begin, cand_end, max_cand: int,
                    idx_out=None, workspace=None, dev_err=None, stream=None) -> torch.Tensor:
     if idx_out is None:
         idx_out = torch.empty((kv.batch, kv.h_kv, int(k)), dtype=torch.int32, device=q.q.device)
-    ws = _workspace(sd_topk_workspace_size(kv, max_cand, k), q.q.device, workspace)
+    ws = _workspace(lambda: sd_topk_workspace_size(kv, max_cand, k), q.q.device, workspace)
     with _on(q.q):
         _check(lib().sd_topk_select(
             ctypes.byref(q.desc), _ptr(q.q), ctypes.byref(kv.desc), kv.batch, _ptr(cand_begin),
@@ -377,7 +379,7 @@ def sd_topk_select_scored(mode: int, q: Queries, kv: KVCache, cand_begin, cand_e
     [batch][h_kv][max_cand] tensor that receives every candidate's score."""
     if idx_out is None:
         idx_out = torch.empty((kv.batch, kv.h_kv, int(k)), dtype=torch.int32, device=q.q.device)
-    ws = _workspace(sd_topk_scored_workspace_size(mode, q, kv, max_cand, k), q.q.device,
+    ws = _workspace(lambda: sd_topk_scored_workspace_size(mode, q, kv, max_cand, k), q.q.device,
                     workspace)
     with _on(q.q):
         _check(lib().sd_topk_select_scored(
@@ -432,8 +434,8 @@ def sd_draft_layer(layer: DraftLayer, emb: torch.Tensor, hid: torch.Tensor, cach
     n = emb.shape[0]
     if out is None:
         out = torch.empty((n, layer.d_model), dtype=torch.bfloat16, device=emb.device)
-    nbytes = sd_draft_layer_workspace_size(layer, n, cache, max_kv_len, window)
-    ws = _workspace(nbytes, emb.device, workspace)
+    ws = _workspace(lambda: sd_draft_layer_workspace_size(layer, n, cache, max_kv_len, window),
+                    emb.device, workspace)
     with _on(emb):
         _check(lib().sd_draft_layer(ctypes.byref(layer.desc), _ptr(emb), _ptr(hid), int(n),
                                     ctypes.byref(cache.desc), int(max_kv_len), int(window),
@@ -467,7 +469,7 @@ def sd_accept_greedy(tgt_logits, draft_tok, gamma, max_gamma: int, n_acc=None, o
     n_acc = torch.empty(batch, dtype=torch.int32, device=dev) if n_acc is None else n_acc
     if out_tok is None:
         out_tok = torch.full((batch, max_gamma + 1), -1, dtype=torch.int32, device=dev)
-    ws = _workspace(sd_accept_workspace_size(batch, max_gamma, vocab), dev, workspace)
+    ws = _workspace(lambda: sd_accept_workspace_size(batch, max_gamma, vocab), dev, workspace)
     with _on(tgt_logits):
         _check(lib().sd_accept_greedy(_ptr(tgt_logits), _ptr(draft_tok), _ptr(gamma), batch,
                                       int(max_gamma), vocab, _ptr(n_acc), _ptr(out_tok),
@@ -486,7 +488,7 @@ def sd_accept_sample(tgt_logits, draft_logits, draft_tok, u, v, gamma, max_gamma
         out_tok = torch.full((batch, max_gamma + 1), -1, dtype=torch.int32, device=dev)
     if near_boundary is None:
         near_boundary = torch.zeros(batch, dtype=torch.int32, device=dev)
-    ws = _workspace(sd_accept_workspace_size(batch, max_gamma, vocab), dev, workspace)
+    ws = _workspace(lambda: sd_accept_workspace_size(batch, max_gamma, vocab), dev, workspace)
     with _on(tgt_logits):
         _check(lib().sd_accept_sample(_ptr(tgt_logits), _ptr(draft_logits), _ptr(draft_tok),
                                       _ptr(u), _ptr(v), _ptr(gamma), batch, int(max_gamma), vocab,
