@@ -1225,7 +1225,7 @@ def run_reference(args):
 
 
 CASES = ("verify", "sparse", "sparse_staged", "stage", "text_anchored", "topk", "hsr",
-         "accept_greedy", "accept_sample", "decode", "prefill_select")
+         "accept_greedy", "accept_sample", "decode", "prefill_select", "draft_layer")
 
 
 def run_case(args):
@@ -1279,6 +1279,14 @@ def run_case(args):
         hw = gen.make_hsr_workload(n=1)
         e, h, W = (dev.tensor(a, gen.BF16) for a in (hw.emb, hw.hid, hw.weight))
         call = lambda: sd.sd_hsr_project(e, h, W)
+    elif args.case == "draft_layer":  # Sparrow's full draft layer, 7B shapes, one row
+        dw = gen.make_draft_layer_workload(n=1)
+        t = lambda a: dev.tensor(a, gen.BF16)
+        layer = sd.DraftLayer(dw.d_model, dw.h_q, dw.h_kv, dw.head_dim, dw.d_ff, dw.rms_eps,
+                              dw.rope_theta, **{n: t(getattr(dw, n)) for n in sd.DraftLayer.NAMES})
+        cache = sd.KVCache(t(dw.k_cache), t(dw.v_cache), dev.int32([dw.kv_len]))
+        e, h = t(dw.emb), t(dw.hid)
+        call = lambda: sd.sd_draft_layer(layer, e, h, cache, dw.kv_len, dw.window)
     else:
         aw = gen.make_accept_workload(2, gammas=[g], batch=1)
         t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
