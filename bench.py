@@ -64,7 +64,7 @@ KERNELS = {  # call kind -> the library kernels one call launches
     "sparse_direct": "attn_* engine (+ attn_merge_kernel when split)",
     "hsr": "hsr_ring_kernel",
     "text_anchored": "attn_tc_kernel (+ attn_merge_kernel when split)",
-    "verify": "attn_tc_kernel + attn_merge_kernel",
+    "verify": "attn_tc_persist_kernel + attn_merge_kernel (persistent plan)",
     "accept_greedy": "accept_argmax_kernel + accept_greedy_kernel",
     "accept_sample": "accept_stats/decide/wsum/draw kernels",
 }
