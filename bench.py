@@ -255,11 +255,15 @@ class Cycle:
             self.gmax = int(aw.gamma.max())
             B = aw.batch
             self.ws_acc = mk(sd.sd_accept_workspace_size(B, self.gmax, aw.vocab))
-            self.n_acc_g = torch.empty(B, dtype=torch.int32, device=device)
-            self.out_g = torch.empty((B, self.gmax + 1), dtype=torch.int32, device=device)
-            self.n_acc_s = torch.empty(B, dtype=torch.int32, device=device)
-            self.out_s = torch.empty((B, self.gmax + 1), dtype=torch.int32, device=device)
-            self.near = torch.empty(B, dtype=torch.int32, device=device)
+            # the step's results, views of one buffer (one device-to-host copy brings them back)
+            nt = B * (self.gmax + 1)
+            self.results = torch.empty(3 * B + 2 * nt, dtype=torch.int32, device=device)
+            r = self.results
+            self.n_acc_g = r[0:B]
+            self.out_g = r[B:B + nt].view(B, self.gmax + 1)
+            self.n_acc_s = r[B + nt:2 * B + nt]
+            self.out_s = r[2 * B + nt:2 * B + 2 * nt].view(B, self.gmax + 1)
+            self.near = r[2 * B + 2 * nt:3 * B + 2 * nt]
         self.calls = self._calls()
         self.bytes = {}
         for kind, step, _ in self.calls:
@@ -802,7 +806,7 @@ class HostIO:
                 sets[b] += [torch.empty_like(t, device=cyc.k.device) for t in self.kv_rows[2:]]
             self.host += list(self.kv_rows[2:])
         if cyc.aw is not None:
-            self.outs = [cyc.n_acc_g, cyc.out_g, cyc.n_acc_s, cyc.out_s, cyc.near]
+            self.outs = [cyc.results]  # accepted counts and tokens of both rules, near-ties
         else:
             self.outs = [cyc.o_verify]
         self.res = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
