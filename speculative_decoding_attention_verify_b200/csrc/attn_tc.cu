@@ -4,7 +4,7 @@
 // Serves every bf16 attention call with d = 64 or 128 and R = G * max_q_rows <= 128 rows per
 // KV head (7B-like layers: R = 7 for a draft step, 42..63 for verification of 6..9 rows).
 //
-// One CTA per (split, KV head g, sequence b); 6 warps, one CTA per SM:
+// One CTA per (split, KV head g, sequence b); 7 warps, one CTA per SM:
 //   warps 0-3  softmax: TMEM lane r holds MMA row r; with NCP row copies the R rows are
 //              placed NCP times (copy c in lanes [c * 128/NCP, ...)) and each warp handles
 //              the 128/NCP tile columns of its copy (rows past R are padding, never read back)
@@ -13,17 +13,23 @@
 //              half of every stage (a stage's K is released once S is computed, its V once
 //              P.V is); contiguous caches: one 4-D box per half of head_dim; paged caches: one
 //              box per 16-position page
-//   warp 5     MMA issuer (one elected thread) and TMEM owner
-// Per tile t (double-buffered S in TMEM):
-//   S_t = Q K_t^T        tcgen05.mma kind::f16, M=128, N=128, A = Q (TMEM, written once by
-//                        the softmax warps), B = K tile (smem, K-major), fp32 accumulators
+//   warp 5     S = Q K^T issuer (one thread) and TMEM owner
+//   warp 6     O += P V issuer (one thread)
+// Per tile t (three S buffers in TMEM):
+//   S_t = Q K_t^T        tcgen05.mma kind::f16, M=128, N=128, A = Q (a shared-memory tile in
+//                        the K tile's layout, written once by the softmax warps), B = K tile
+//                        (smem, K-major), fp32 accumulators
 //   softmax              each thread reads its row's columns of S_t from TMEM, applies the
 //                        run bounds and the row's visible ranges, updates its running max
 //                        (base 2) and writes P_t = 2^(s - m) as bf16 over S_t in TMEM.  The
 //                        running max used for the exponent only moves when the true max grows
 //                        by more than 2^8 ("lazy rescale"), so O is rarely touched.
 //   O += P_t V_t         tcgen05.mma with A = P_t from TMEM, B = V tile (smem, MN-major)
-// The issuer issues S of tile t+1 and P.V of tile t in whichever order their operands arrive.
+// One thread issues a tcgen05.mma no faster than every ~150 SM cycles whatever its shape, and
+// a tile takes 16 of them (8 for S over d = 128, 8 for P.V over the tile's 128 positions), so
+// the two products have an issuing warp each and S runs up to three tiles ahead: S of tile t
+// goes into buffer t % 3 once the P.V of tile t-3, which reads P from that buffer, has
+// completed.  (Q sits in shared memory to leave TMEM room for the third buffer.)
 // The row copies' partial (m, l, O) are merged in shared memory at the end.  Partial outputs
 // (O, max, sum) go to the split workspace exactly like the CUDA-core engine, or, with a single
 // split, O / sum is written directly.
@@ -34,7 +40,11 @@
 //   attn_tc_persist_kernel  one CTA per SM, each taking an equal contiguous share of all units'
 //                           tiles and running its units back to back (long streams: verify,
 //                           plain decoding), so no partial last wave idles SMs; partials of
-//                           units shared by two CTAs are merged by attn_merge_kernel
+//                           units shared by two CTAs are merged by attn_merge_kernel.  Its
+//                           streams are bound by HBM and its merge scratch leaves no shared
+//                           memory for Q: Q stays in TMEM, S is double-buffered and one
+//                           thread issues both products, S of tile t+1 and P.V of tile t in
+//                           whichever order their operands arrive (6 warps)
 // The host plans one or the other from a time model.  They are separate kernels because the
 // per-unit bookkeeping costs the short draft calls registers and time per tile.
 // Every wait on an mbarrier is bounded (the launch's wait bound, 1 s by default); on expiry the
@@ -52,11 +62,17 @@ using namespace tc;
 constexpr int kTile = 128;            // positions per tile
 constexpr int kRows = 128;            // MMA M
 constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 6 * 32;
-constexpr uint32_t kTmemCols = 512;   // S0 [0,128) S1 [128,256) O [256,256+D) Q [384,384+D/2)
+constexpr int kMmaWarp = 5;           // S = Q K^T issuer (persistent: both products), TMEM owner
+constexpr int kPvWarp = 6;            // per-unit kernel: O += P V issuer
+constexpr int kThreads = 6 * 32;      // persistent kernel
+constexpr int kThreadsUnit = 7 * 32;  // per-unit kernel
+constexpr uint32_t kTmemCols = 512;
+// persistent kernel: S0 [0,128) S1 [128,256) O [256,256+D) Q [384,384+D/2)
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kColQ = 384;       // Q as packed bf16 pairs: the A operand of S = Q K^T
+// per-unit kernel: S0 S1 S2 [0,384) O [384,384+D)
+constexpr int kSBufs = 3;
+constexpr uint32_t kColOUnit = 384;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kHalfBytes = kTile * 128;  // one 64-column half of a 128-row tile
 constexpr int kMaxSegs = 8;      // segments (units) one CTA may touch
@@ -71,6 +87,10 @@ struct Cfg {
     static constexpr int kSegOffset = kBarOffset + 256;  // the CTA's segment table
     static constexpr int kMergeOffset = kSegOffset + kSegBytes;  // persistent: merge scratch
     static constexpr int kSmem = kMergeOffset + 1024;  // (+ slack to align the base to 1 KB)
+    // per-unit kernel: the Q tile (the K tile's layout, 1 KB aligned) where the persistent
+    // kernel keeps its merge scratch
+    static constexpr int kQOffset = kMergeOffset;
+    static constexpr int kSmemUnit = kQOffset + kTileBytes + 1024;
 };
 
 // ---------------------------------------------------------------- the kernel --------------
@@ -225,6 +245,19 @@ struct TileCursor {
     }
 };
 
+// Drain of one issuing warp: once `bar` (committed here) flips, every MMA its lane 0 issued
+// has completed.  Bounded (kDrainNs): an aborted CTA must still free its TMEM.
+__device__ __forceinline__ void mma_drain(uint32_t bar, bool issued, int lane) {
+    const bool any_issued = __any_sync(0xffffffffu, issued);
+    if (lane == 0 && any_issued) {
+        mma_commit(bar);
+        const unsigned long long t0 = now_ns();
+        while (!mbar_try(bar, 0) && now_ns() - t0 < kDrainNs) {
+        }
+    }
+    __syncwarp();
+}
+
 // NCP row copies: with R <= 128 / NCP rows per KV head, the rows are placed NCP times in the
 // 128 MMA rows (copy c in rows [c * 128/NCP, (c+1) * 128/NCP)) and softmax warp w, of copy
 // c = w / (4 / NCP), handles the columns [c * 128/NCP, (c+1) * 128/NCP) of every tile: the
@@ -232,7 +265,7 @@ struct TileCursor {
 // one or two.  Each copy keeps its own running max, sum and output rows; the copies are
 // merged in shared memory at the end.
 template <int D, bool PAGED, int NCP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsUnit, 1)
 attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     constexpr int RPC = kRows / NCP;  // rows per copy
     constexpr int NC = kTile / NCP;   // columns per softmax warp
@@ -243,16 +276,22 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sKV = smem;  // stage s: K at s*2*tile, V at s*2*tile + tile
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
-    // barrier slots: k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_full[2],
-    // o_done, drain.  A stage's K half is released as soon as S = Q K^T is computed, its V
-    // half once P.V is, so the next K copy starts a softmax earlier.
+    uint8_t *sQ = smem + C::kQOffset;  // Q rows: the A operand of S = Q K^T
+    // barrier slots: k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[3], p_full[3],
+    // pv_done[3] (per S buffer), drain (P.V issuer), s_drain (S issuer), q_full.  A stage's K
+    // half is released as soon as S = Q K^T is computed, its V half once P.V is, so the next
+    // K copy starts a softmax earlier.
     const uint32_t bar0 = saddr(bars);
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    const int KF = 0, VF = S, KE = 2 * S, VE = 3 * S, SF = 4 * S, PF = 4 * S + 2, OD = 4 * S + 4,
-              DR = 4 * S + 5, QF = 4 * S + 6;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * S + 7);
+    const int KF = 0, VF = S, KE = 2 * S, VE = 3 * S, SF = 4 * S, PF = SF + kSBufs,
+              PD = PF + kSBufs, DR = PD + kSBufs, DS = DR + 1, QF = DS + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + QF + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *s_stream = reinterpret_cast<int *>(tmem_slot + 2);  // stream set-up scratch
+    // stream set-up scratch: 4 ints (sparse streams are set up without it, so stream_setup's
+    // per-warp counts are never written here)
+    int *s_stream = reinterpret_cast<int *>(tmem_slot + 2);
+    static_assert((4 * S + 3 * kSBufs + 3) * 8 + 8 + 16 <= C::kSegOffset - C::kBarOffset,
+                  "barrier region");
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.z, g = blockIdx.y, split = blockIdx.x;
@@ -279,7 +318,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         si.s1 = min(max(__ldg(p.tail_begin + b), 0), kv_len);
         si.len1 = kv_len - si.s1;
     } else {
-        si = stream_setup<kThreads>(p, b, g, n_q, kv_len, s_stream);
+        si = stream_setup<kThreadsUnit>(p, b, g, n_q, kv_len, s_stream);
     }
     const int a0 = (PAGED && !sparse) ? (si.s0 & ~(kPageSize - 1)) : si.s0;
     const int a1 = PAGED ? (si.s1 & ~(kPageSize - 1)) : si.s1;
@@ -307,13 +346,14 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             mbar_init(BAR(KE + s), 1);
             mbar_init(BAR(VE + s), 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kSBufs; ++s) {
             mbar_init(BAR(SF + s), 1);
             mbar_init(BAR(PF + s), 32 * n_active);
+            mbar_init(BAR(PD + s), 1);
         }
-        mbar_init(BAR(OD), 1);
         mbar_init(BAR(DR), 1);
-        mbar_init(BAR(QF), 128);  // Q in TMEM (warps 0-3)
+        mbar_init(BAR(DS), 1);
+        mbar_init(BAR(QF), 128);  // Q in shared memory (warps 0-3)
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -321,40 +361,23 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
     __syncthreads();
     tc_after();
     const uint32_t tmem = *tmem_slot;
-    // Q rows into TMEM columns [kColQ, kColQ + D/2) as packed bf16 pairs, the A operand of
-    // S = Q K^T (read by the tensor core from TMEM, not re-read from shared memory every
-    // tile): lane rr holds query row rr % RPC of the group (zero past R).  Each of warps 0-3
-    // writes its own 32 lanes, after the producer has started its first copies; the MMA
-    // issuer waits for it before the first S = Q K^T.
+    // Q rows into shared memory in the K tile's layout (64-element halves of 128-byte rows,
+    // 16-byte chunk c of row rr in slot c ^ (rr & 7): the 128-byte swizzle), the A operand of
+    // S = Q K^T: row rr holds query row rr % RPC of the group (zero past R).  Each of warps
+    // 0-3 writes its own 32 rows, after the producer has started its first copies; the S
+    // issuer waits for all of them.
     if (warp < 4) {
         const int rr = warp * 32 + lane, r = rr % RPC;
-        uint32_t qv[D / 2];
-        if (r < R) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                reinterpret_cast<const unsigned short *>(p.q) +
-                ((int64_t)(q0 + r / G) * p.h_q + g * G + r % G) * D);
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            reinterpret_cast<const unsigned short *>(p.q) +
+            ((int64_t)(q0 + (r < R ? r / G : 0)) * p.h_q + g * G + (r < R ? r % G : 0)) * D);
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-                const uint4 x = __ldg(src + c);
-                qv[4 * c] = x.x;
-                qv[4 * c + 1] = x.y;
-                qv[4 * c + 2] = x.z;
-                qv[4 * c + 3] = x.w;
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < D / 2; ++c) qv[c] = 0u;
+        for (int c = 0; c < D / 8; ++c) {
+            const uint4 x = r < R ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(sQ + (c >> 3) * kHalfBytes + rr * 128 +
+                                       (((c & 7) ^ (rr & 7)) << 4)) = x;
         }
-        const uint32_t qaddr = tmem + ((uint32_t)(warp * 32) << 16) + kColQ;
-        if constexpr (D == 128) {
-            tmem_st64(qaddr, qv);
-        } else {
-            float qf[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) qf[c] = __uint_as_float(qv[c]);
-            tmem_st32(qaddr, qf);
-        }
-        tc_before();
+        fence_async_smem();
         mbar_arrive(BAR(QF));
     }
 
@@ -411,22 +434,29 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             }
         }
     } else if (warp == kMmaWarp) {
-        // ---------------------------------------------------------- MMA issuer ------------
+        // ------------------------------------------------------- S = Q K^T issuer ---------
         // Lane 0 waits and issues; the decision is broadcast so the warp stays converged.
-        // S = Q K^T of tile t+1 is issued before waiting for the softmax of tile t, so the
-        // tensor core computes it while the softmax warps work.
+        // S of tile t waits for its K stage, for Q (first tile) and for the completion of the
+        // P.V of tile t-3, which reads P from the S buffer this S overwrites.
         const uint32_t idesc_qk = idesc_bf16(kTile, false);
-        const uint32_t idesc_pv = idesc_bf16(D, true);
+        const uint32_t qb = saddr(sQ);
         bool issued = false;
-        auto issue_qk = [&](int t) {  // S = Q K^T of tile t (its K stage has landed)
-            const int s = t % S, sb = t & 1;
-            const uint32_t kb = saddr(sKV + (size_t)s * 2 * C::kTileBytes);
+        for (int t = 0; t < n_my; ++t) {
+            const int s = t % S, use = t / S, sb = t % kSBufs;
+            bool ok = true;
+            if (lane == 0)
+                ok = (t > 0 || mbar_wait(BAR(QF), 0, abort_flag, p.dev_err, p.wait_ns)) &&
+                     mbar_wait(BAR(KF + s), use & 1, abort_flag, p.dev_err, p.wait_ns) &&
+                     (t < kSBufs || mbar_wait(BAR(PD + sb), ((t - kSBufs) / kSBufs) & 1,
+                                              abort_flag, p.dev_err, p.wait_ns));
+            if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
             tc_after();
             if (lane == 0) {
+                const uint32_t kb = saddr(sKV + (size_t)s * 2 * C::kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                    mma_ts(tmem + sb * kTile, tmem + kColQ + kk * 8, desc_k_sw128(kb + off),
+                    mma_ss(tmem + sb * kTile, desc_k_sw128(qb + off), desc_k_sw128(kb + off),
                            idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(BAR(SF + sb));
@@ -434,9 +464,22 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 issued = true;
             }
             __syncwarp();
-        };
-        auto issue_pv = [&](int t) {  // O += P V of tile t (its P and V stage are ready)
-            const int s = t % S, sb = t & 1;
+        }
+        mma_drain(BAR(DS), issued, lane);
+    } else if (warp == kPvWarp) {
+        // ------------------------------------------------------- O += P V issuer ----------
+        // P.V of tile t waits for P_t (the softmax warps) and its V stage; its completion
+        // releases the V stage and frees S buffer t % 3 for S of tile t+3.
+        const uint32_t idesc_pv = idesc_bf16(D, true);
+        bool issued = false;
+        for (int t = 0; t < n_my; ++t) {
+            const int s = t % S, use = t / S, sb = t % kSBufs;
+            bool ok = true;
+            if (lane == 0)
+                ok = mbar_wait(BAR(PF + sb), (t / kSBufs) & 1, abort_flag, p.dev_err,
+                               p.wait_ns) &&
+                     mbar_wait(BAR(VF + s), use & 1, abort_flag, p.dev_err, p.wait_ns);
+            if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
             // V rows past the end of the sequence may hold anything (NaN included): zero
             // them so that 0 * V cannot poison O.
             uint8_t *vs = sKV + (size_t)s * 2 * C::kTileBytes + C::kTileBytes;
@@ -458,74 +501,17 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 const uint32_t vb = saddr(vs);
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ts(tmem + kColO, tmem + sb * kTile + kk * 8,
+                    mma_ts(tmem + kColOUnit, tmem + sb * kTile + kk * 8,
                            desc_mn_sw128(vb + kk * 2048, kHalfBytes), idesc_pv,
                            (t > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(BAR(VE + s));
-                mma_commit(BAR(OD));
+                mma_commit(BAR(PD + sb));
+                issued = true;
             }
             __syncwarp();
-        };
-        bool alive = true;
-        if (n_my > 0) {
-            bool qok = true;
-            if (lane == 0)
-                qok = mbar_wait(BAR(QF), 0, abort_flag, p.dev_err, p.wait_ns) &&
-                      mbar_wait(BAR(KF), 0, abort_flag, p.dev_err, p.wait_ns);
-            alive = __shfl_sync(0xffffffffu, qok ? 1 : 0, 0) != 0;
-            if (alive) issue_qk(0);
         }
-        for (int t = 0; alive && t < n_my; ++t) {
-            // S of tile t+1 and P.V of tile t, in whichever order their operands arrive (S
-            // first when both are ready, so the softmax warps get their next tile early).  S of
-            // t+1 overwrites the buffer of tile t-1, whose P.V was issued in the previous
-            // iteration, so either order is safe.
-            const int s = t % S, use = t / S, sb = t & 1;
-            const int s1 = (t + 1) % S, use1 = (t + 1) / S;
-            bool qk_done = t + 1 >= n_my, pv_done = false;
-            const unsigned long long t0 = now_ns();
-            const uint32_t hint = poll_hint(p.wait_ns);
-            for (unsigned it = 1; !(qk_done && pv_done); ++it) {
-                int flags = 0;  // bit 0: S can go, bit 1: P.V can go, bit 2: give up
-                if (lane == 0) {
-                    if (!qk_done && mbar_try_for(BAR(KF + s1), use1 & 1, hint)) flags |= 1;
-                    if (!pv_done && mbar_try_for(BAR(PF + sb), (t >> 1) & 1, hint) &&
-                        mbar_try_for(BAR(VF + s), use & 1, hint))
-                        flags |= 2;
-                    if (flags == 0) {
-                        if (now_ns() - t0 > p.wait_ns) {
-                            *abort_flag = 1;
-                            set_dev_err(p.dev_err, SD_DEVERR_TIMEOUT);
-                            flags = 4;
-                        } else if ((it & 7u) == 0 && *abort_flag) {
-                            flags = 4;
-                        }
-                    }
-                }
-                flags = __shfl_sync(0xffffffffu, flags, 0);
-                if (flags & 4) {
-                    alive = false;
-                    break;
-                }
-                if (flags & 1) {
-                    issue_qk(t + 1);
-                    qk_done = true;
-                }
-                if (flags & 2) {
-                    issue_pv(t);
-                    pv_done = true;
-                }
-            }
-        }
-        // Drain: every MMA this warp issued has completed once the drain barrier flips.
-        const bool any_issued = __any_sync(0xffffffffu, issued);
-        if (lane == 0 && any_issued) {
-            mma_commit(BAR(DR));
-            const unsigned long long t0 = now_ns();
-            while (!mbar_try(BAR(DR), 0) && now_ns() - t0 < kDrainNs) {
-            }
-        }
-        __syncwarp();
+        // (the softmax warps' epilogue waits on the same drain barrier: O is complete)
+        mma_drain(BAR(DR), issued, lane);
     } else if (warp < n_active) {
         // ---------------------------------------------------------- softmax ---------------
         // tcgen05.ld / st are warp-collective: every lane executes them, row validity only
@@ -564,14 +550,14 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
         float m_used = -INFINITY, l = 0.f;
         bool ok_run = true;
         for (int t = 0; t < n_my; ++t) {
-            const int sb = t & 1;
+            const int sb = t % kSBufs;
             const int tt = tile_lo + t;
             const int p0 = tile_start(tt);
             // the run this tile belongs to: positions [seg_lo, seg_hi)
             const int seg_lo = tt < nt0 ? si.s0 : si.s1;
             const int seg_hi = tt < nt0 ? si.s0 + si.len0 : si.s1 + si.len1;
             const bool got =
-                mbar_wait(BAR(SF + sb), (t >> 1) & 1, abort_flag, p.dev_err, p.wait_ns);
+                mbar_wait(BAR(SF + sb), (t / kSBufs) & 1, abort_flag, p.dev_err, p.wait_ns);
             if (!__all_sync(FULL, got)) {
                 ok_run = false;
                 break;
@@ -626,10 +612,12 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             const bool rescale_o = grow && m_used != -INFINITY;
             if (__any_sync(FULL, rescale_o)) {
                 // O holds tiles < t: wait for the P.V of tile t-1, then rescale O in TMEM.
-                // S_t was committed after the P.V of tile t-2 and the P.V of tile t needs this
-                // warp's arrival, so o_done is in phase t-1 or t: its parity test is exact.
-                const bool done =
-                    mbar_wait(BAR(OD), (t - 1) & 1, abort_flag, p.dev_err, p.wait_ns);
+                // (pv_done of buffer (t-1) % 3: S_{t-1} was issued once the P.V of tile t-4,
+                // that buffer's previous use, had completed, and its next use, tile t+2, needs
+                // this warp's later arrivals, so the parity test is exact.)
+                const int pb = (t - 1) % kSBufs;
+                const bool done = mbar_wait(BAR(PD + pb), ((t - 1) / kSBufs) & 1, abort_flag,
+                                            p.dev_err, p.wait_ns);
                 if (!__all_sync(FULL, done)) {
                     ok_run = false;
                     break;
@@ -639,10 +627,10 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                 float o[32];
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    tmem_ld32(lane_base + kColO + c * 32, o);
+                    tmem_ld32(lane_base + kColOUnit + c * 32, o);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] *= corr;
-                    tmem_st32(lane_base + kColO + c * 32, o);
+                    tmem_st32(lane_base + kColOUnit + c * 32, o);
                 }
                 l *= corr;
             }
@@ -706,7 +694,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
             s_l[cp * RPC + r] = l_out;
             {
                 float o[D];
-                if (read_o) tmem_ld_cols<D>(lane_base + kColO, o);
+                if (read_o) tmem_ld_cols<D>(lane_base + kColOUnit, o);
                 float4 *dst = s_o + (cp * RPC + r) * (D / 4);
 #pragma unroll
                 for (int k = 0; k < D / 4; ++k)
@@ -754,7 +742,7 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
                     o[4 * k + 3] = acc.w;
                 }
             } else {
-                if (read_o) tmem_ld32(lane_base + kColO + c * 32, o);
+                if (read_o) tmem_ld32(lane_base + kColOUnit + c * 32, o);
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
                     if (!have) o[e] = 0.f;
@@ -1449,19 +1437,20 @@ int row_copies(int rows) { return rows <= 32 ? 4 : rows <= kNcp2Rows ? 2 : 1; }
 // Shared memory of a launch: the ring and barriers, plus, for a persistent launch with row
 // copies, the merge scratch ((m, l) of every MMA row and the O rows of copies 1..).
 int tc_smem_bytes(int head_dim, int rows, bool persistent) {
+    if (!persistent) return head_dim == 128 ? Cfg<128>::kSmemUnit : Cfg<64>::kSmemUnit;
     const int base = head_dim == 128 ? Cfg<128>::kSmem : Cfg<64>::kSmem;
     const int ncp = row_copies(rows);
-    if (!persistent || ncp == 1) return base;
+    if (ncp == 1) return base;
     return base + (2 * kRows + (ncp - 1) * rows * head_dim) * 4;
 }
 
 template <int D, bool PAGED, int NCP>
 cudaError_t launch_t(const AttnParams &p, const TcMaps &maps, cudaStream_t s) {
     if (p.persist_s == 0) {
-        cudaError_t e = set_max_dynamic_smem<attn_tc_kernel<D, PAGED, NCP>>(Cfg<D>::kSmem);
+        cudaError_t e = set_max_dynamic_smem<attn_tc_kernel<D, PAGED, NCP>>(Cfg<D>::kSmemUnit);
         if (e != cudaSuccess) return e;
-        attn_tc_kernel<D, PAGED, NCP>
-            <<<dim3(p.n_splits, p.kv.h_kv, p.batch), kThreads, Cfg<D>::kSmem, s>>>(p, maps);
+        attn_tc_kernel<D, PAGED, NCP><<<dim3(p.n_splits, p.kv.h_kv, p.batch), kThreadsUnit,
+                                        Cfg<D>::kSmemUnit, s>>>(p, maps);
         return cudaGetLastError();
     }
     const int smem = tc_smem_bytes(D, p.group * p.max_q_rows, true);
