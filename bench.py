@@ -58,7 +58,7 @@ SPECS = {
 }
 
 KERNELS = {  # call kind -> the library kernels one call launches
-    "topk": "topk_score_kernel + topk_select_smem_kernel",
+    "topk": "topk_score_fast_kernel + topk_select_fast_kernel",
     "stage": "sparse_compact_kernel",
     "sparse": "attn_tc_kernel (+ attn_merge_kernel when split)",
     "sparse_direct": "attn_* engine (+ attn_merge_kernel when split)",

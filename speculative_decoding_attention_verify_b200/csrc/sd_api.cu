@@ -636,7 +636,8 @@ sd_status sd_topk_select_scored(sd_topk_score mode, const sd_q_desc *q, const vo
     const long long tiles = ((long long)max_cand + 127) / 128;
     double best = -1.0;
     p.n_splits = 1;
-    for (long long sp = 1; sp <= 1024; ++sp) {
+    const int max_splits = topk_part_stride(max_cand);
+    for (long long sp = 1; sp <= max_splits; ++sp) {
         if (sp > 1 && tiles / sp < 4) break;
         const long long ctas = units * sp;
         const long long waves = (ctas + slots - 1) / slots;
@@ -646,6 +647,10 @@ sd_status sd_topk_select_scored(sd_topk_score mode, const sd_q_desc *q, const vo
             p.n_splits = (int)sp;
         }
     }
+    // the scoring's per-split partials follow the keys
+    p.part_stride = max_splits;
+    p.parts = reinterpret_cast<uint2 *>(static_cast<char *>(workspace) +
+                                        (size_t)units * max_cand * sizeof(unsigned long long));
     return cuda_status(launch_topk(p, s));
 }
 

@@ -113,8 +113,13 @@ struct TopkParams {
     float *lse;         // [rows_cap][h_q]
     double *scores;     // nullable: [batch][h_kv][max_cand] every candidate's score
     unsigned long long wait_ns;  // bound of every pipeline wait inside the kernels
+    // fp32 scoring (last-query mode without scores_out): per (unit, split) the largest error
+    // sum of the split's candidates (float bits) and whether any score was not finite
+    uint2 *parts;       // [batch][h_kv][part_stride]
+    int part_stride;    // >= n_splits
 };
 size_t topk_workspace_bytes(int batch, int h_kv, int max_cand);
+int topk_part_stride(int max_cand);  // the largest split count the scoring may use
 int topk_score_ctas_per_sm();  // resident scoring CTAs per SM
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t s);
 // The selection half of top-K (radix select of p.keys, ascending output).

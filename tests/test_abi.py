@@ -139,7 +139,9 @@ def test_workspace_sizes_scale_with_the_problem():
     assert n1.value > 0 and n2.value > 0
     _, kv = _descs()
     assert lib.sd_topk_workspace_size(ctypes.byref(kv), 28, 25000, 1024, ctypes.byref(n1)) == 0
-    assert n1.value == 28 * 4 * 25000 * 8
+    # 64-bit key slots per candidate, then the fp32 scoring's per-split partials (8 bytes for
+    # each of up to ceil(25000 / 128) / 4 = 49 splits)
+    assert n1.value == 28 * 4 * 25000 * 8 + 28 * 4 * 49 * 8
 
 
 def test_topk_scored_validation():

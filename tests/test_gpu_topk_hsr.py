@@ -140,6 +140,76 @@ def test_topk_huge_query_values():
     assert _assert_same_sets(got, ref, gap) == 0
 
 
+def _boundary(w, k, cb, ce):
+    """Oracle scores [b][g][t] and, per (b, g), the position of the k-th best candidate."""
+    sc = oracle.topk_scores(w.h_q, w.q_verify, w.q_verify_start, oracle.cache_from_workload(w),
+                            cb, ce)
+    order = np.argsort(-sc, axis=-1, kind="stable")
+    return sc, order[..., k - 1] + cb[:, None]
+
+
+def test_topk_exact_ties_across_the_boundary():
+    """Seven candidates share the k-th best score exactly (copies of its key row, placed below
+    and above it): the lowest positions among them are kept, in every KV head."""
+    w = gen.make_attn_workload(1, l_vis=3000, l_txt=50)
+    k, cb, ce = 100, np.zeros(1, np.int32), np.array([3000], np.int32)
+    _, jstar = _boundary(w, k, cb, ce)
+    kk = w.k.copy()
+    for g in range(w.h_kv):
+        j = int(jstar[0, g])
+        for dst in (5, 333, 1200, 1201, 2222, 2999):
+            if dst != j:
+                kk[0, g, dst] = kk[0, g, j]
+    w.k = kk
+    got, ref, gap = _run_topk(w, k, cand_begin=cb, cand_end=ce)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_near_ties_finer_than_fp32_are_ranked_in_fp64():
+    """Near-copies of the k-th best key row that differ in one dimension whose group query sum
+    is 2^-20: their scores differ by ~1e-9 relative, far below the fp32 scores' resolution, so
+    only the fp64 rescoring of the boundary band orders them (not by position)."""
+    w = gen.make_attn_workload(1, l_vis=3000, l_txt=50)
+    q = w.q_verify.copy()
+    last = int(w.q_verify_start[1]) - 1
+    e0 = 17
+    G = w.h_q // w.h_kv
+    for g in range(w.h_kv):
+        q[last, g * G:(g + 1) * G, e0] = 0
+        q[last, g * G, e0] = 0x3580  # 2^-20
+    w.q_verify = q
+    k, cb, ce = 150, np.zeros(1, np.int32), np.array([3000], np.int32)
+    _, jstar = _boundary(w, k, cb, ce)
+    kk = w.k.copy()
+    for g in range(w.h_kv):
+        j = int(jstar[0, g])
+        base = int(kk[0, g, j, e0])
+        if base & 0x7F80 in (0, 0x7F80):  # keep the edited element a normal number
+            base = 0x3F80
+            kk[0, g, j, e0] = base
+        # (a positive bf16 value grows with its bit pattern; a negative one shrinks)
+        for dst, step in ((7, 2), (400, -1), (1300, 3), (2100, -3), (2900, 1)):
+            if dst != j:
+                kk[0, g, dst] = kk[0, g, j]
+                kk[0, g, dst, e0] = base + step
+    w.k = kk
+    got, ref, gap = _run_topk(w, k, cand_begin=cb, cand_end=ce)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_band_wider_than_shared_memory_takes_the_fp64_path():
+    """Every key row of one KV head identical: all 3,000 scores tie, the band around the
+    threshold holds every candidate (more than the 1,024 ranked in shared memory), and the
+    fp64 selection keeps the lowest positions; the other heads take the fp32 path."""
+    w = gen.make_attn_workload(1, l_vis=3000, l_txt=50)
+    kk = w.k.copy()
+    kk[0, 2, :3000] = kk[0, 2, 1234]
+    w.k = kk
+    got, ref, gap = _run_topk(w, 200)
+    assert np.array_equal(got, ref)
+    assert np.array_equal(got[0, 2], np.arange(200))
+
+
 # ---------------------------------------------------------------- HSR ----------------------
 
 
