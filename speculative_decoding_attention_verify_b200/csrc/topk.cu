@@ -413,6 +413,31 @@ constexpr uint32_t kKeyDropped = 0u;         // band candidate ranked out
 constexpr float kErrScale = 0x1p-15f;        // E = kErrScale * max B + kErrFloor
 constexpr double kErrFloor = 0x1p-140;
 
+constexpr int kGroupRowsCap = 2048;  // group x d query elements staged in shared memory
+
+// The group's query elements of row `last` into s_qh [G][D] (floats: exact for both dtypes),
+// by `nthreads` threads numbered t, four independent loads in flight per thread (a loop over
+// the heads would wait for each load in turn).  Requires G * D <= kGroupRowsCap.
+template <bool BF16, int D>
+__device__ __forceinline__ void stage_group_rows(const TopkParams &p, int last, int g, float *s_qh,
+                                                 int t, int nthreads) {
+    const int total = p.group * D;
+    for (int base = 0; base < total; base += 4 * nthreads) {
+        float v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = base + t + j * nthreads;
+            v[j] = i < total ? query_elem<BF16, D>(p.q, p.h_q, last, g * p.group + i / D, i % D)
+                             : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = base + t + j * nthreads;
+            if (i < total) s_qh[i] = v[j];
+        }
+    }
+}
+
 // The fp32 scoring streams each CTA's candidate rows through a ring of 64-row stages filled by
 // plain bulk copies (one per run of rows contiguous in the cache: the whole tile, or a page's
 // rows) issued by a copy warp; eight warps score (four threads per candidate, as the fp64
@@ -442,6 +467,7 @@ topk_score_fast_kernel(const TopkParams p) {
     __shared__ __align__(8) uint64_t s_full[S], s_empty[S];
     __shared__ unsigned long long s_live[S];  // bit r: row r of the stage holds a cache row
     __shared__ float s_q[D], s_qu[D];
+    __shared__ float s_qh[kGroupRowsCap];  // the group's query elements [G][D]
     __shared__ float s_bmax[kFastWarps];
     __shared__ int s_bad[kFastWarps];
     __shared__ int s_abort;
@@ -522,11 +548,19 @@ topk_score_fast_kernel(const TopkParams p) {
         }
     } else {
         // ---- scoring warps: thread quad (4c .. 4c+3) takes candidate c of each stage ----
-        // (the query sums are formed while the first copies are in flight)
+        // (the query sums are formed while the first copies are in flight; the group's
+        // elements are summed in head order, in fp64)
+        const bool staged = p.group * D <= kGroupRowsCap;
+        if (staged) {
+            stage_group_rows<BF16, D>(p, last, g, s_qh, tid, kFastWarps * 32);
+            asm volatile("bar.sync 1, %0;" ::"n"(kFastWarps * 32) : "memory");
+        }
         for (int e = tid; e < D; e += kFastWarps * 32) {
             double acc = 0.0, mag = 0.0;
-            for (int h = g * p.group; h < (g + 1) * p.group; ++h) {
-                const double x = (double)query_elem<BF16, D>(p.q, p.h_q, last, h, e);
+            for (int h = 0; h < p.group; ++h) {
+                const double x = staged ? (double)s_qh[h * D + e]
+                                        : (double)query_elem<BF16, D>(p.q, p.h_q, last,
+                                                                      g * p.group + h, e);
                 acc += x;
                 mag += fabs(x);
             }
@@ -693,6 +727,7 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_fast_kernel(const 
     __shared__ unsigned long long s_prefix;
     __shared__ int s_remaining;
     __shared__ double s_qbar[D];
+    __shared__ float s_qh[kGroupRowsCap];             // the group's query elements [G][D]
     __shared__ int s_band[kBandCap];                  // band: local candidate index
     __shared__ unsigned long long s_bkey[kBandCap];   // and its fp64 score key
     __shared__ float s_bmax;
@@ -712,10 +747,16 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_fast_kernel(const 
         for (int e = tid; e < p.k; e += kSelectThreads) out[e] = e < n ? cb + e : -1;
         return;
     }
-    for (int e = tid; e < D; e += kSelectThreads) {
+    const bool staged = p.group * D <= kGroupRowsCap;
+    if (staged) {
+        stage_group_rows<BF16, D>(p, last, g, s_qh, tid, kSelectThreads);
+        __syncthreads();
+    }
+    for (int e = tid; e < D; e += kSelectThreads) {  // (head order, fp64)
         double acc = 0.0;
-        for (int h = g * p.group; h < (g + 1) * p.group; ++h)
-            acc += (double)query_elem<BF16, D>(p.q, p.h_q, last, h, e);
+        for (int h = 0; h < p.group; ++h)
+            acc += staged ? (double)s_qh[h * D + e]
+                          : (double)query_elem<BF16, D>(p.q, p.h_q, last, g * p.group + h, e);
         s_qbar[e] = acc;
     }
     if (warp == 0) {
@@ -736,10 +777,24 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_fast_kernel(const 
     }
     uint32_t *gkeys = reinterpret_cast<uint32_t *>(p.keys + (int64_t)unit * p.max_cand);
     const bool in_smem = p.max_cand <= kSmemKeys32;
-    if (in_smem) {  // (the unit's key slots start 8-byte aligned: two keys per load)
+    if (in_smem) {  // (the unit's key slots start 8-byte aligned: two keys per load, four
+                    // loads in flight per thread)
         const uint2 *src = reinterpret_cast<const uint2 *>(gkeys);
-        for (int e = tid; e < n / 2; e += kSelectThreads)
-            reinterpret_cast<uint2 *>(s_k32)[e] = src[e];
+        uint2 *dst = reinterpret_cast<uint2 *>(s_k32);
+        const int n2 = n / 2;
+        for (int base = 0; base < n2; base += 4 * kSelectThreads) {
+            uint2 v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int e = base + tid + j * kSelectThreads;
+                v[j] = e < n2 ? src[e] : make_uint2(0u, 0u);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int e = base + tid + j * kSelectThreads;
+                if (e < n2) dst[e] = v[j];
+            }
+        }
         if ((n & 1) && tid == 0) s_k32[n - 1] = gkeys[n - 1];
     }
     __syncthreads();
