@@ -68,6 +68,8 @@ __device__ __forceinline__ void chunk_range(int vocab, int n_chunks, int c, int 
 // ---------------------------------------------------------------- greedy -----------------
 
 __global__ void __launch_bounds__(kThreads) accept_argmax_kernel(const AcceptParams p) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     __shared__ unsigned long long s_red[kThreads / 32];
     const int c = blockIdx.x, slot = blockIdx.y;
     const int b = slot / (p.max_gamma + 1), i = slot % (p.max_gamma + 1);
@@ -95,6 +97,8 @@ __global__ void __launch_bounds__(kThreads) accept_argmax_kernel(const AcceptPar
 }
 
 __global__ void accept_greedy_kernel(const AcceptParams p) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     extern __shared__ int s_t[];  // argmax of every target row of this sequence
     const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gm = __ldg(p.gamma + b);
@@ -135,6 +139,8 @@ __global__ void accept_greedy_kernel(const AcceptParams p) {
 
 // Row slot layout of the statistics: target rows first (batch*(max_gamma+1)), then draft rows.
 __global__ void __launch_bounds__(kThreads) accept_stats_kernel(const AcceptParams p) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     __shared__ float s_m[kThreads / 32], s_s[kThreads / 32];
     const int c = blockIdx.x, slot = blockIdx.y;
     const int n_tslots = p.batch * (p.max_gamma + 1);
@@ -196,6 +202,8 @@ __device__ __forceinline__ double *chunk_sums(const AcceptParams &p) {
 
 // One warp per sequence.
 __global__ void accept_decide_kernel(const AcceptParams p) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     const int b = blockIdx.x, lane = threadIdx.x;
     const int gm = __ldg(p.gamma + b);
     Decision *dec = decisions(p) + b;
@@ -271,6 +279,8 @@ __device__ double block_sum_d(double x, double *s_red) {
 
 // (sequence, chunk) -> sum of the draw weights of the chunk.
 __global__ void __launch_bounds__(kThreads) accept_wsum_kernel(const AcceptParams p) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     __shared__ double s_red[kThreads / 32];
     const int c = blockIdx.x, b = blockIdx.y;
     const Decision dec = decisions(p)[b];
@@ -290,6 +300,8 @@ __global__ void __launch_bounds__(kThreads) accept_wsum_kernel(const AcceptParam
 
 // One CTA per sequence: locate v*Z, finish the outputs.
 __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const AcceptParams p) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     __shared__ double s_red[kThreads / 32];
     __shared__ double s_warp_tot[kThreads / 32];
     __shared__ int s_found;
@@ -418,25 +430,22 @@ size_t accept_workspace_bytes(int batch, int max_gamma, int vocab, int *n_chunks
 
 cudaError_t launch_accept_greedy(const AcceptParams &p, cudaStream_t s) {
     dim3 g1(p.n_chunks, p.batch * (p.max_gamma + 1));
-    accept_argmax_kernel<<<g1, kThreads, 0, s>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(accept_argmax_kernel, g1, dim3(kThreads), 0, s, p);
     if (e != cudaSuccess) return e;
-    accept_greedy_kernel<<<p.batch, 256, (p.max_gamma + 1) * sizeof(int), s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(accept_greedy_kernel, dim3(p.batch), dim3(256),
+                      (p.max_gamma + 1) * sizeof(int), s, p);
 }
 
 cudaError_t launch_accept_sample(const AcceptParams &p, cudaStream_t s) {
     dim3 g1(p.n_chunks, p.batch * (2 * p.max_gamma + 1));
-    accept_stats_kernel<<<g1, kThreads, 0, s>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(accept_stats_kernel, g1, dim3(kThreads), 0, s, p);
     if (e != cudaSuccess) return e;
-    accept_decide_kernel<<<p.batch, 32, 0, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(accept_decide_kernel, dim3(p.batch), dim3(32), 0, s, p)) != cudaSuccess)
+        return e;
     dim3 g3(p.n_chunks, p.batch);
-    accept_wsum_kernel<<<g3, kThreads, 0, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    accept_draw_kernel<<<p.batch, kThreads, 0, s>>>(p);
-    return cudaGetLastError();
+    if ((e = launch_pdl(accept_wsum_kernel, g3, dim3(kThreads), 0, s, p)) != cudaSuccess)
+        return e;
+    return launch_pdl(accept_draw_kernel, dim3(p.batch), dim3(kThreads), 0, s, p);
 }
 
 }  // namespace sd

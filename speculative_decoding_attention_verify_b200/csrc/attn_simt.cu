@@ -365,6 +365,8 @@ attn_simt_kernel(const AttnParams p) {
 // known).
 template <bool BF16, int D>
 __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     constexpr int EPL = D / 32;
     constexpr int kPre = 4;  // splits whose outputs are loaded with the statistics
     const int lane = threadIdx.x & 31;
@@ -459,8 +461,7 @@ template <bool BF16, int D>
 cudaError_t launch_merge_t(const AttnParams &p, cudaStream_t s) {
     const int64_t warps = (int64_t)p.rows_cap * p.h_q;
     const int blocks = (int)((warps + 3) / 4);
-    attn_merge_kernel<BF16, D><<<blocks, 128, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(attn_merge_kernel<BF16, D>, dim3(blocks), dim3(128), 0, s, p);
 }
 
 }  // namespace

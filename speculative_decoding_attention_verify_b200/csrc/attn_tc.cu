@@ -267,6 +267,8 @@ __device__ __forceinline__ void mma_drain(uint32_t bar, bool issued, int lane) {
 template <int D, bool PAGED, int NCP>
 __global__ void __launch_bounds__(kThreadsUnit, 1)
 attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     constexpr int RPC = kRows / NCP;  // rows per copy
     constexpr int NC = kTile / NCP;   // columns per softmax warp
     using C = Cfg<D>;
@@ -807,6 +809,8 @@ attn_tc_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
 template <int D, bool PAGED, int NCP>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_persist_kernel(const AttnParams p, const __grid_constant__ TcMaps maps) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     constexpr int RPC = kRows / NCP;  // rows per copy
     constexpr int NC = kTile / NCP;   // columns per softmax warp
     using C = Cfg<D>;
@@ -1449,16 +1453,15 @@ cudaError_t launch_t(const AttnParams &p, const TcMaps &maps, cudaStream_t s) {
     if (p.persist_s == 0) {
         cudaError_t e = set_max_dynamic_smem<attn_tc_kernel<D, PAGED, NCP>>(Cfg<D>::kSmemUnit);
         if (e != cudaSuccess) return e;
-        attn_tc_kernel<D, PAGED, NCP><<<dim3(p.n_splits, p.kv.h_kv, p.batch), kThreadsUnit,
-                                        Cfg<D>::kSmemUnit, s>>>(p, maps);
-        return cudaGetLastError();
+        return launch_pdl(attn_tc_kernel<D, PAGED, NCP>, dim3(p.n_splits, p.kv.h_kv, p.batch),
+                          dim3(kThreadsUnit), Cfg<D>::kSmemUnit, s, p, maps);
     }
     const int smem = tc_smem_bytes(D, p.group * p.max_q_rows, true);
     // (the opt-in is the largest any launch may ask for: the merge scratch varies)
     cudaError_t e = set_max_dynamic_smem<attn_tc_persist_kernel<D, PAGED, NCP>>(kMaxDynSmem);
     if (e != cudaSuccess) return e;
-    attn_tc_persist_kernel<D, PAGED, NCP><<<dim3(p.persist_g), kThreads, smem, s>>>(p, maps);
-    return cudaGetLastError();
+    return launch_pdl(attn_tc_persist_kernel<D, PAGED, NCP>, dim3(p.persist_g), dim3(kThreads),
+                      smem, s, p, maps);
 }
 
 }  // namespace

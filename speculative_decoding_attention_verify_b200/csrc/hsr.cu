@@ -26,6 +26,8 @@ template <int NR>
 __global__ void __launch_bounds__(kWarps * 32)
 hsr_kernel(const uint16_t *emb, const uint16_t *hid, int n_rows, int d_model, const uint16_t *w,
            const uint16_t *bias, uint16_t *y, int max_rows_per_cta) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     extern __shared__ uint4 s_x4[];  // [NR][2*d_model] bf16 chunks, then [rows][kParts][NR] f32
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g0 = blockIdx.y * NR;
@@ -120,6 +122,8 @@ template <int NR, int S>
 __global__ void __launch_bounds__(kRingThreads, 1)
 hsr_ring_kernel(const uint16_t *emb, const uint16_t *hid, int n_rows, int d_model,
                 const uint16_t *w, const uint16_t *bias, uint16_t *y) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     // [NR][cpr] input chunks, then the ring [S][16][cpp] chunks, then [items][NR] f32 partials
     extern __shared__ __align__(16) uint4 s_x4[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -208,11 +212,11 @@ cudaError_t launch_ring_t(const void *emb, const void *hid, int n_rows, int d_mo
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(ctas, (n_rows + NR - 1) / NR);
-    kern<<<grid, kRingThreads, smem, s>>>(
-        reinterpret_cast<const uint16_t *>(emb), reinterpret_cast<const uint16_t *>(hid), n_rows,
-        d_model, reinterpret_cast<const uint16_t *>(w), reinterpret_cast<const uint16_t *>(bias),
-        reinterpret_cast<uint16_t *>(y));
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(kRingThreads), smem, s,
+                      reinterpret_cast<const uint16_t *>(emb),
+                      reinterpret_cast<const uint16_t *>(hid), n_rows, d_model,
+                      reinterpret_cast<const uint16_t *>(w),
+                      reinterpret_cast<const uint16_t *>(bias), reinterpret_cast<uint16_t *>(y));
 }
 
 template <int NR>
@@ -244,11 +248,12 @@ cudaError_t launch_hsr_t(const void *emb, const void *hid, int n_rows, int d_mod
         if (e != cudaSuccess) return e;
     }
     dim3 grid(ctas, (n_rows + NR - 1) / NR);
-    kern<<<grid, kWarps * 32, smem, s>>>(
-        reinterpret_cast<const uint16_t *>(emb), reinterpret_cast<const uint16_t *>(hid), n_rows,
-        d_model, reinterpret_cast<const uint16_t *>(w), reinterpret_cast<const uint16_t *>(bias),
-        reinterpret_cast<uint16_t *>(y), max_rows);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(kWarps * 32), smem, s,
+                      reinterpret_cast<const uint16_t *>(emb),
+                      reinterpret_cast<const uint16_t *>(hid), n_rows, d_model,
+                      reinterpret_cast<const uint16_t *>(w),
+                      reinterpret_cast<const uint16_t *>(bias), reinterpret_cast<uint16_t *>(y),
+                      max_rows);
 }
 
 }  // namespace

@@ -28,6 +28,40 @@ struct KVView {
     const int32_t *kv_len;
 };
 
+// Programmatic dependent launch.  A kernel launched by launch_pdl may be scheduled while the
+// previous kernel on its stream is still running (once that kernel's CTAs have all started,
+// each of them calling pdl_trigger first); every such kernel calls pdl_wait before its first
+// global memory access, which returns once the previous kernel has completed and its writes
+// are visible.  The next call's launch and CTA scheduling thus overlap this call's tail.  Only
+// launches made one by one take it: on a stream being captured into a CUDA graph the launch
+// is plain (a replayed graph has its launches prepared already, and there the waiting CTAs
+// only held SMs early: a speculative-decoding cycle replayed 1.6% slower with it, while the
+// same cycle launched call by call ran 6% faster).  Without the attribute pdl_wait returns at
+// once.
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    const bool eager = cudaStreamIsCapturing(s, &cs) == cudaSuccess &&
+                       cs == cudaStreamCaptureStatusNone;
+    cfg.attrs = attr;
+    cfg.numAttrs = eager ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Opt kernel Kern in to `bytes` of dynamic shared memory, once per device (the attribute is
 // per device, and a process may drive several).  `bytes` must be the same on every call.
 template <auto Kern>

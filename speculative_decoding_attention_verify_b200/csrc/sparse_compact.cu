@@ -26,6 +26,8 @@ __device__ __forceinline__ bool kept(const int32_t *sel, int e, int tail) {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) sparse_compact_kernel(const AttnParams p) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     constexpr int CPR = D * 2 / 16;  // 16-byte chunks per row (bf16)
     constexpr int RPI = 32 / CPR;    // rows per warp instruction
     __shared__ int s_warp[kThreads / 32];
@@ -127,9 +129,9 @@ cudaError_t launch_sparse_compact(const AttnParams &p, cudaStream_t s) {
     const int parts = max(1, min(want, by_len));
     dim3 grid(parts, p.kv.h_kv, p.batch);
     if (p.kv.head_dim == 128)
-        sparse_compact_kernel<128><<<grid, kThreads, 0, s>>>(p);
+        return launch_pdl(sparse_compact_kernel<128>, grid, dim3(kThreads), 0, s, p);
     else
-        sparse_compact_kernel<64><<<grid, kThreads, 0, s>>>(p);
+        return launch_pdl(sparse_compact_kernel<64>, grid, dim3(kThreads), 0, s, p);
     return cudaGetLastError();
 }
 

@@ -453,6 +453,8 @@ constexpr int fast_stages(int tile_bytes) { return tile_bytes <= 16384 ? 6 : 3; 
 template <bool BF16, int D>
 __global__ void __launch_bounds__(kFastThreads, kScoreCtasPerSm)
 topk_score_fast_kernel(const TopkParams p) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     using CH = Chunk<BF16>;
     using namespace tc;
     constexpr int ESZ = BF16 ? 2 : 4;
@@ -721,6 +723,8 @@ constexpr int kBandCap = 1024;      // band candidates ranked in shared memory
 // scoring flagged the unit or the band does not fit.
 template <bool BF16, int D>
 __global__ void __launch_bounds__(kSelectThreads) topk_select_fast_kernel(const TopkParams p) {
+    pdl_trigger();  // (see launch_pdl)
+    pdl_wait();
     extern __shared__ uint32_t s_k32[];  // the unit's keys when max_cand <= kSmemKeys32
     __shared__ int s_hist[kRadixBins];
     __shared__ int s_warp[32];
@@ -949,16 +953,15 @@ cudaError_t launch_fast_t(const TopkParams &p, cudaStream_t s) {
     const int dyn = fast_stages(tile) * tile;
     cudaError_t e = set_max_dynamic_smem<topk_score_fast_kernel<BF16, D>>(dyn);
     if (e != cudaSuccess) return e;
-    topk_score_fast_kernel<BF16, D>
-        <<<dim3(p.n_splits, p.kv.h_kv, p.batch), kFastThreads, dyn, s>>>(p);
-    e = cudaGetLastError();
+    e = launch_pdl(topk_score_fast_kernel<BF16, D>, dim3(p.n_splits, p.kv.h_kv, p.batch),
+                   dim3(kFastThreads), dyn, s, p);
     if (e != cudaSuccess) return e;
     const size_t sdyn = p.max_cand <= kSmemKeys32 ? (size_t)p.max_cand * sizeof(uint32_t) : 0;
     e = set_max_dynamic_smem<topk_select_fast_kernel<BF16, D>>(
         (int)(kSmemKeys32 * sizeof(uint32_t)));
     if (e != cudaSuccess) return e;
-    topk_select_fast_kernel<BF16, D><<<dim3(p.kv.h_kv, p.batch), kSelectThreads, sdyn, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(topk_select_fast_kernel<BF16, D>, dim3(p.kv.h_kv, p.batch),
+                      dim3(kSelectThreads), sdyn, s, p);
 }
 
 }  // namespace
