@@ -9,12 +9,14 @@
 // rows.
 //
 // Ring kernel (the weight share's items are contiguous in memory): stage u holds items
-// [16u, 16u + 16), copied by all threads with 16-byte cp.async chunks, S - 1 stages ahead
-// (112 KB in flight per SM for d_model = 3584), so the copies stream continuously; warp w
-// dots item 16u + w with the input rows.
+// [16u, 16u + 16), one bulk copy issued by a copy warp up to S stages ahead (full / empty
+// mbarriers per stage; 56 KB per stage for d_model = 3584), so the copies stream
+// continuously; warp w dots item 16u + w with the input rows and releases its share of the
+// stage.
 // Fallback kernel (rows too large for a ring of at least two stages): the 16 warps take the
 // items round-robin, two at a time (14 coalesced 16-byte loads per lane in flight).
 #include "sd_internal.h"
+#include "tc_ptx.cuh"
 
 namespace sd {
 namespace {
@@ -114,18 +116,22 @@ hsr_kernel(const uint16_t *emb, const uint16_t *hid, int n_rows, int d_model, co
     }
 }
 
-constexpr int kRingWarps = 16;
-constexpr int kRingThreads = kRingWarps * 32;
-constexpr size_t kRingSmemMax = 227 * 1024;
+constexpr int kRingWarps = 16;                     // consumer warps: one item each per stage
+constexpr int kRingThreads = (kRingWarps + 1) * 32;  // + the copy warp
+constexpr size_t kRingSmemMax = 227 * 1024 - 256;  // (dynamic: the barriers are static)
+constexpr unsigned long long kRingWaitNs = 1000000000ull;  // bound of every pipeline wait
 
 template <int NR, int S>
 __global__ void __launch_bounds__(kRingThreads, 1)
 hsr_ring_kernel(const uint16_t *emb, const uint16_t *hid, int n_rows, int d_model,
                 const uint16_t *w, const uint16_t *bias, uint16_t *y) {
+    using namespace tc;
     pdl_trigger();  // (see launch_pdl)
     pdl_wait();
     // [NR][cpr] input chunks, then the ring [S][16][cpp] chunks, then [items][NR] f32 partials
     extern __shared__ __align__(16) uint4 s_x4[];
+    __shared__ __align__(8) uint64_t s_full[S], s_empty[S];
+    __shared__ int s_abort;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g0 = blockIdx.y * NR;
     const int nr = min(NR, n_rows - g0);
@@ -138,60 +144,90 @@ hsr_ring_kernel(const uint16_t *emb, const uint16_t *hid, int n_rows, int d_mode
     float *s_part = reinterpret_cast<float *>(ring + (size_t)S * kRingWarps * cpp);
     const uint4 *wbase = reinterpret_cast<const uint4 *>(w) + (int64_t)r0 * cpr;
     const int n_stages = (items + kRingWarps - 1) / kRingWarps;
-    auto issue = [&](int u) {
-        const uint32_t dst = static_cast<uint32_t>(
-            __cvta_generic_to_shared(ring + (size_t)(u % S) * kRingWarps * cpp));
-        const int i0 = u * kRingWarps;
-        const int nchunk = min(kRingWarps, items - i0) * cpp;
-        const uint4 *src = wbase + (int64_t)i0 * cpp;
-        for (int e = tid; e < nchunk; e += kRingThreads) cp_async16(dst + 16u * e, src + e);
-    };
-    for (int u = 0; u < S - 1; ++u) {
-        if (u < n_stages) issue(u);
-        cp_async_commit();
-    }
-    for (int e = tid; e < NR * cpr; e += kRingThreads) {
-        const int r = e / cpr, c = e % cpr;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < nr) {
-            const int col = c * 8;
-            const uint16_t *src = col < d_model ? emb + (int64_t)(g0 + r) * d_model + col
-                                                : hid + (int64_t)(g0 + r) * d_model + (col - d_model);
-            v = *reinterpret_cast<const uint4 *>(src);
+    if (tid == 0) {
+        for (int st = 0; st < S; ++st) {
+            mbar_init(saddr(&s_full[st]), 1);
+            mbar_init(saddr(&s_empty[st]), kRingWarps);
         }
-        s_x4[e] = v;
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    for (int u = 0; u < n_stages; ++u) {
-        cp_async_wait<S - 2>();
-        __syncthreads();  // stage u has landed for every thread; stage u - 1 is consumed
-        if (u + S - 1 < n_stages) issue(u + S - 1);
-        cp_async_commit();
-        const int it = u * kRingWarps + warp;
-        if (it < items) {
-            const uint4 *wr = ring + (size_t)(u % S) * kRingWarps * cpp + (size_t)warp * cpp;
-            const int col0 = (it % kParts) * cpp;
-            float part[NR];
+    __syncthreads();
+    volatile int *abort_flag = &s_abort;
+    int n_issued = 0;
+    if (warp == kRingWarps) {
+        // ---- copy warp: stage u (items [16u, 16u + 16), contiguous) is one bulk copy ----
+        if (lane == 0) {
+            for (int u = 0; u < n_stages; ++u) {
+                const int st = u % S;
+                if (u >= S && !mbar_wait(saddr(&s_empty[st]), ((u / S) - 1) & 1, abort_flag,
+                                         nullptr, kRingWaitNs))
+                    break;
+                const int i0 = u * kRingWarps;
+                const uint32_t bytes = (uint32_t)(min(kRingWarps, items - i0) * cpp * 16);
+                mbar_arrive_tx(saddr(&s_full[st]), bytes);
+                bulk_load(saddr(ring + (size_t)st * kRingWarps * cpp), wbase + (int64_t)i0 * cpp,
+                          bytes, saddr(&s_full[st]));
+                n_issued = u + 1;
+                if (*abort_flag) break;
+            }
+        }
+    } else {
+        for (int e = tid; e < NR * cpr; e += kRingWarps * 32) {
+            const int r = e / cpr, c = e % cpr;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (r < nr) {
+                const int col = c * 8;
+                const uint16_t *src = col < d_model
+                                          ? emb + (int64_t)(g0 + r) * d_model + col
+                                          : hid + (int64_t)(g0 + r) * d_model + (col - d_model);
+                v = *reinterpret_cast<const uint4 *>(src);
+            }
+            s_x4[e] = v;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kRingWarps * 32) : "memory");  // input rows in
+        for (int u = 0; u < n_stages; ++u) {
+            const int st = u % S;
+            const bool got =
+                mbar_wait(saddr(&s_full[st]), (u / S) & 1, abort_flag, nullptr, kRingWaitNs);
+            if (!__all_sync(0xffffffffu, got)) break;  // (the warp leaves together)
+            const int it = u * kRingWarps + warp;
+            if (it < items) {
+                const uint4 *wr = ring + (size_t)st * kRingWarps * cpp + (size_t)warp * cpp;
+                const int col0 = (it % kParts) * cpp;
+                float part[NR];
 #pragma unroll
-            for (int r = 0; r < NR; ++r) part[r] = 0.f;
-            for (int c = lane; c < cpp; c += 32) {
-                float wf[8];
-                Chunk<true>::to_float(wr[c], wf);
+                for (int r = 0; r < NR; ++r) part[r] = 0.f;
+                for (int c = lane; c < cpp; c += 32) {
+                    float wf[8];
+                    Chunk<true>::to_float(wr[c], wf);
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) {
+                        float xf[8];
+                        Chunk<true>::to_float(s_x4[r * cpr + col0 + c], xf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) part[r] = fmaf(wf[e], xf[e], part[r]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(saddr(&s_empty[st]));  // the item is read
 #pragma unroll
                 for (int r = 0; r < NR; ++r) {
-                    float xf[8];
-                    Chunk<true>::to_float(s_x4[r * cpr + col0 + c], xf);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) part[r] = fmaf(wf[e], xf[e], part[r]);
+                    const float sum = warp_sum(part[r]);
+                    if (lane == 0) s_part[it * NR + r] = sum;
                 }
-            }
-#pragma unroll
-            for (int r = 0; r < NR; ++r) {
-                const float sum = warp_sum(part[r]);
-                if (lane == 0) s_part[it * NR + r] = sum;
+            } else if (lane == 0) {
+                mbar_arrive(saddr(&s_empty[st]));
             }
         }
     }
-    cp_async_wait<0>();
+    // ---- teardown: after an abort, the copy lane waits (bounded) for its copies in flight ----
+    if (warp == kRingWarps && lane == 0 && *abort_flag) {
+        const unsigned long long t0 = now_ns();
+        for (int u = (n_issued > S ? n_issued - S : 0); u < n_issued; ++u)
+            while (!mbar_try(saddr(&s_full[u % S]), (u / S) & 1) && now_ns() - t0 < kDrainNs) {
+            }
+    }
     __syncthreads();
     for (int e = tid; e < nr * (r1 - r0); e += kRingThreads) {
         const int r = e / (r1 - r0), i = e % (r1 - r0);
