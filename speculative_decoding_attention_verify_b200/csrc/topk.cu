@@ -715,6 +715,8 @@ __device__ double exact_score(const TopkParams &p, const double *s_qbar, int las
 
 constexpr int kSmemKeys32 = 49152;  // 192 KB of 32-bit keys
 constexpr int kRadixBins = 2048;    // 11-bit digits
+constexpr int kKeyGroups = 8;       // 32-key groups a warp reads per step (loads in flight)
+constexpr int kGroupKeys = 32 * kKeyGroups;
 constexpr int kBandCap = 1024;      // band candidates ranked in shared memory
 
 // One CTA per (sequence, KV head): the radix select of the k-th largest fp32 key (tau), the
@@ -805,22 +807,21 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_fast_kernel(const 
     bool exact = s_flag != 0;
     if (!exact) {
         uint32_t *keys = in_smem ? s_k32 : gkeys;
-        // thread t owns the keys [t * kpt, t * kpt + kpt), kpt a multiple of 4: shared-memory
-        // keys are read four at a time (the tail and global keys one at a time)
-        const int kpt = ((n + 4 * kSelectThreads - 1) / (4 * kSelectThreads)) * 4;
-        const int first = tid * kpt;
-        const int mine = max(0, min(kpt, n - first));  // keys owned by this thread
-        auto load4 = [&](int i, uint32_t (&k4)[4]) {
-            const int idx = first + i;
-            if (in_smem && i + 4 <= mine) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(keys + idx);
-                k4[0] = v.x; k4[1] = v.y; k4[2] = v.z; k4[3] = v.w;
-            } else {
+        // warp w owns the keys [w * seg, w * seg + seg) (seg a multiple of kGroupKeys), which its
+        // lanes read 32 consecutive keys at a time (coalesced in global memory, conflict-free in
+        // shared memory), kKeyGroups groups in flight; keys past the segment or n read 0
+        const int seg = ((n + 32 * kGroupKeys - 1) / (32 * kGroupKeys)) * kGroupKeys;
+        const int wbeg = warp * seg;
+        const int wend = min(n, wbeg + seg);
+        auto load_groups = [&](int i, uint32_t (&kg)[kKeyGroups]) {  // (i: offset in the segment)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) k4[j] = i + j < mine ? keys[idx + j] : 0u;
+            for (int j = 0; j < kKeyGroups; ++j) {
+                const int idx = wbeg + i + 32 * j + lane;
+                kg[j] = idx < wend ? keys[idx] : 0u;
             }
         };
         // ---- radix select of the k-th largest key (digits of 11, 11 and 10 bits) ----
+        // (a real key is never 0: that is the key of NaN, which flags the unit)
         uint32_t prefix = 0u, mask = 0u;
         int remaining = p.k;
         for (int pass = 0; pass < 3; ++pass) {
@@ -828,13 +829,13 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_fast_kernel(const 
             const uint32_t dmask = pass == 2 ? 1023u : 2047u;
             for (int i = tid; i < kRadixBins; i += kSelectThreads) s_hist[i] = 0;
             __syncthreads();
-            for (int i = 0; i < mine; i += 4) {
-                uint32_t k4[4];
-                load4(i, k4);
+            for (int i = 0; wbeg + i < wend; i += kGroupKeys) {
+                uint32_t kg[kKeyGroups];
+                load_groups(i, kg);
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (i + j < mine && (k4[j] & mask) == prefix)
-                        atomicAdd(&s_hist[(k4[j] >> shift) & dmask], 1);
+                for (int j = 0; j < kKeyGroups; ++j)
+                    if (kg[j] != 0u && (kg[j] & mask) == prefix)
+                        atomicAdd(&s_hist[(kg[j] >> shift) & dmask], 1);
             }
             __syncthreads();
             // cumulative counts from the largest bucket down: thread t takes buckets
@@ -862,13 +863,13 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_fast_kernel(const 
         const uint32_t key_hi = score_key32(__double2float_rd(tau + 2.0 * E));
         const uint32_t key_lo = score_key32(__double2float_ru(tau - 2.0 * E));
         int n_in = 0, n_band = 0;
-        for (int i = 0; i < mine; i += 4) {
-            uint32_t k4[4];
-            load4(i, k4);
+        for (int i = 0; wbeg + i < wend; i += kGroupKeys) {
+            uint32_t kg[kKeyGroups];
+            load_groups(i, kg);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {  // (keys past the thread's range read 0: out)
-                n_in += k4[j] > key_hi ? 1 : 0;
-                n_band += (k4[j] >= key_lo && k4[j] <= key_hi) ? 1 : 0;
+            for (int j = 0; j < kKeyGroups; ++j) {  // (0, past the range, is below key_lo)
+                n_in += kg[j] > key_hi ? 1 : 0;
+                n_band += (kg[j] >= key_lo && kg[j] <= key_hi) ? 1 : 0;
             }
         }
         int in_total, band_total;
@@ -878,9 +879,12 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_fast_kernel(const 
         // least k; a violation would mean a broken bound: the fp64 path decides then)
         exact = band_total > kBandCap || in_total >= p.k || in_total + band_total < p.k;
         if (!exact) {
-            for (int i = 0; i < mine; ++i) {
-                const uint32_t kk = keys[first + i];
-                if (kk >= key_lo && kk <= key_hi) s_band[pos++] = first + i;
+            for (int i = 0; wbeg + i < wend; i += kGroupKeys) {
+                uint32_t kg[kKeyGroups];
+                load_groups(i, kg);
+#pragma unroll
+                for (int j = 0; j < kKeyGroups; ++j)
+                    if (kg[j] >= key_lo && kg[j] <= key_hi) s_band[pos++] = wbeg + i + 32 * j + lane;
             }
             __syncthreads();
             for (int m = warp; m < band_total; m += kSelectThreads / 32) {
@@ -906,18 +910,42 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_fast_kernel(const 
             __syncthreads();
             // ---- output: kept positions, ascending ----
             // (kKeyKept is above every key, kKeyDropped below: the kept keys are those above
-            // key_hi)
+            // key_hi.)  Each warp counts its segment's, one scan over the warps gives its first
+            // slot, and the warp writes its kept positions in order, 32 keys at a time.
             int keep_n = 0;
-            for (int i = 0; i < mine; i += 4) {
-                uint32_t k4[4];
-                load4(i, k4);
+            for (int i = 0; wbeg + i < wend; i += kGroupKeys) {
+                uint32_t kg[kKeyGroups];
+                load_groups(i, kg);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) keep_n += k4[j] > key_hi ? 1 : 0;
+                for (int j = 0; j < kKeyGroups; ++j) keep_n += kg[j] > key_hi ? 1 : 0;
             }
-            int keep_total;
-            int w = block_inclusive_scan(keep_n, s_warp, keep_total) - keep_n;
-            for (int i = 0; i < mine; ++i)
-                if (keys[first + i] > key_hi) out[w++] = cb + first + i;
+            keep_n = __reduce_add_sync(0xffffffffu, keep_n);
+            if (lane == 0) s_warp[warp] = keep_n;
+            __syncthreads();
+            if (warp == 0) {
+                const int c = s_warp[lane];
+                int incl = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                s_warp[lane] = incl - c;
+            }
+            __syncthreads();
+            int w = s_warp[warp];
+            for (int i = 0; wbeg + i < wend; i += kGroupKeys) {
+                uint32_t kg[kKeyGroups];
+                load_groups(i, kg);
+#pragma unroll
+                for (int j = 0; j < kKeyGroups; ++j) {
+                    const bool keep = kg[j] > key_hi;
+                    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                    if (keep)
+                        out[w + __popc(bal & ((1u << lane) - 1u))] = cb + wbeg + i + 32 * j + lane;
+                    w += __popc(bal);
+                }
+            }
         }
     }
     if (exact) {  // (uniform: from the flag or from block-wide totals)
