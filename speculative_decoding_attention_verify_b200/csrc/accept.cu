@@ -8,11 +8,15 @@
 //           accept_greedy_kernel  per sequence: reduce the chunks of every row, then the
 //                                 longest matching prefix and the bonus token.
 // Sampling: accept_stats_kernel   (row, chunk) -> (max, sum exp(z - max)) in fp32
-//           accept_decide_kernel  per sequence: log-sum-exp of every row in fp64, the accept
-//                                 decisions u <= p/q (ratio in fp64), which row draws and how
-//           accept_wsum_kernel    (sequence, chunk) -> sum of the draw weights (fp64)
-//           accept_draw_kernel    per sequence: find the chunk holding v*Z, then the token by
-//                                 an in-order prefix sum inside it; write the outputs.
+//           accept_decide_kernel  per sequence: log-sum-exp of every row in fp64 (a warp per
+//                                 row), then the accept decisions u <= p/q (ratio in fp64),
+//                                 which row draws and how
+//           accept_wsum_kernel    (sequence, chunk) -> sum of the draw weights (fp64); the
+//                                 drawing row has chunks of its own, about two CTAs per SM
+//                                 over the batch
+//           accept_draw_kernel    per sequence: find the chunk holding v*Z (a warp scans the
+//                                 chunk sums), then the token by an in-order prefix sum inside
+//                                 it; write the outputs.
 #include "sd_internal.h"
 
 namespace sd {
@@ -196,19 +200,23 @@ __device__ __forceinline__ Decision *decisions(const AcceptParams &p) {
     return reinterpret_cast<Decision *>(base);
 }
 
-__device__ __forceinline__ double *chunk_sums(const AcceptParams &p) {
+__device__ __forceinline__ double *chunk_sums(const AcceptParams &p) {  // [batch][n_wchunks]
     return reinterpret_cast<double *>(decisions(p) + p.batch);
 }
 
-// One warp per sequence.
-__global__ void accept_decide_kernel(const AcceptParams p) {
+constexpr int kDecideWarps = 8;
+
+// One CTA per sequence: the log-sum-exps of its rows (a warp per row) and the draft tokens'
+// logits first, in parallel; then the accept decisions in order from shared memory.
+__global__ void __launch_bounds__(kDecideWarps * 32) accept_decide_kernel(const AcceptParams p) {
     pdl_trigger();  // (see launch_pdl)
     pdl_wait();
-    const int b = blockIdx.x, lane = threadIdx.x;
+    extern __shared__ double s_dec[];  // lse of target rows [gm + 1], draft rows [gm], ratios [gm]
+    const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gm = __ldg(p.gamma + b);
     Decision *dec = decisions(p) + b;
     if (gm < 0 || gm > p.max_gamma) {
-        if (lane == 0) {
+        if (tid == 0) {
             set_dev_err(p.dev_err, SD_DEVERR_SHAPE);
             dec->n = -1;
         }
@@ -217,38 +225,48 @@ __global__ void accept_decide_kernel(const AcceptParams p) {
     int64_t off_t, off_d;
     row_offsets(p.gamma, b, off_t, off_d);
     const int n_tslots = p.batch * (p.max_gamma + 1);
-    int n = 0, near = 0;
-    bool rejected = false;
-    for (int i = 1; i <= gm; ++i) {
-        const double lp = row_lse(p, b * (p.max_gamma + 1) + (i - 1), lane);
-        const double lq = row_lse(p, n_tslots + b * p.max_gamma + (i - 1), lane);
-        const int x = __ldg(p.draft_tok + off_d + i - 1);
+    double *s_lp = s_dec, *s_lq = s_dec + (gm + 1), *s_r = s_lq + gm;
+    for (int j = warp; j < 2 * gm + 1; j += kDecideWarps) {
+        const bool target = j <= gm;
+        const int i = target ? j : j - (gm + 1);
+        const double l = row_lse(p, target ? b * (p.max_gamma + 1) + i
+                                           : n_tslots + b * p.max_gamma + i, lane);
+        if (lane == 0) (target ? s_lp : s_lq)[i] = l;
+    }
+    __syncthreads();
+    // ratio p/q of every draft token (fp64), with the row checks
+    for (int i = tid; i < gm; i += kDecideWarps * 32) {
+        const double lp = s_lp[i], lq = s_lq[i];
+        const int x = __ldg(p.draft_tok + off_d + i);
         double r = 0.0;
         if (x >= 0 && x < p.vocab) {
-            const double zp = (double)__ldg(p.tgt + (off_t + i - 1) * (int64_t)p.vocab + x);
-            const double zq = (double)__ldg(p.drf + (off_d + i - 1) * (int64_t)p.vocab + x);
+            const double zp = (double)__ldg(p.tgt + (off_t + i) * (int64_t)p.vocab + x);
+            const double zq = (double)__ldg(p.drf + (off_d + i) * (int64_t)p.vocab + x);
             r = exp((zp - lp) - (zq - lq));
-        } else if (lane == 0) {
+        } else {
             set_dev_err(p.dev_err, SD_DEVERR_TOKEN);
         }
-        if (!(lp == lp) || !(lq == lq) || isinf(lp) || isinf(lq)) {
-            if (lane == 0) set_dev_err(p.dev_err, SD_DEVERR_NUMERIC);
-        }
-        const double u = (double)__ldg(p.u + off_d + i - 1);
-        if (fabs(u - r) < kNearBoundary) ++near;
-        if (u <= r) {
-            ++n;
-        } else {
-            rejected = true;
-            break;
-        }
+        if (!(lp == lp) || !(lq == lq) || isinf(lp) || isinf(lq))
+            set_dev_err(p.dev_err, SD_DEVERR_NUMERIC);
+        s_r[i] = r;
     }
-    const double lp = row_lse(p, b * (p.max_gamma + 1) + n, lane);
-    double lq = 0.0;
-    if (rejected) lq = row_lse(p, n_tslots + b * p.max_gamma + n, lane);
-    if (lane == 0) {
-        dec->lse_p = lp;
-        dec->lse_q = lq;
+    __syncthreads();
+    if (tid == 0) {
+        int n = 0, near = 0;
+        bool rejected = false;
+        for (int i = 0; i < gm; ++i) {
+            const double u = (double)__ldg(p.u + off_d + i);
+            const double r = s_r[i];
+            if (fabs(u - r) < kNearBoundary) ++near;
+            if (u <= r) {
+                ++n;
+            } else {
+                rejected = true;
+                break;
+            }
+        }
+        dec->lse_p = s_lp[n];
+        dec->lse_q = rejected ? s_lq[n] : 0.0;
         dec->n = n;
         dec->residual = rejected ? 1 : 0;
         dec->near = near;
@@ -290,12 +308,12 @@ __global__ void __launch_bounds__(kThreads) accept_wsum_kernel(const AcceptParam
     const float *zp = p.tgt + (off_t + dec.n) * (int64_t)p.vocab;
     const float *zq = p.drf + (off_d + dec.n) * (int64_t)p.vocab;
     int lo, hi;
-    chunk_range(p.vocab, p.n_chunks, c, lo, hi);
+    chunk_range(p.vocab, p.n_wchunks, c, lo, hi);
     double s = 0.0;
     for (int x = lo + threadIdx.x; x < hi; x += kThreads)
         s += draw_weight(zp, zq, dec.lse_p, dec.lse_q, dec.residual != 0, x);
     s = block_sum_d(s, s_red);
-    if (threadIdx.x == 0) chunk_sums(p)[(int64_t)b * p.n_chunks + c] = s;
+    if (threadIdx.x == 0) chunk_sums(p)[(int64_t)b * p.n_wchunks + c] = s;
 }
 
 // One CTA per sequence: locate v*Z, finish the outputs.
@@ -314,34 +332,64 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const AcceptParam
     const float *zp = p.tgt + (off_t + dec.n) * (int64_t)p.vocab;
     const float *zq = p.drf + (off_d + dec.n) * (int64_t)p.vocab;
     bool residual = dec.residual != 0;
-    const double *cs = chunk_sums(p) + (int64_t)b * p.n_chunks;
-    double Z = 0.0;
-    for (int c = 0; c < p.n_chunks; ++c) Z += cs[c];
-    int c_lo = 0, c_hi = p.n_chunks;  // chunks to scan
+    const int nw = p.n_wchunks;
+    const double *cs = chunk_sums(p) + (int64_t)b * nw;
+    const double v_draw = (double)__ldg(p.v + off_t + dec.n);
+    __shared__ double s_z, s_before;
+    __shared__ int s_clo;
+    // Z, and the chunk where the running total first exceeds v*Z: warp 0 reads the chunk sums
+    // 32 at a time (Z: lane-strided partials, then the warp's tree; a fixed order)
+    if (warp == 0) {
+        double t = 0.0;
+        for (int c = lane; c < nw; c += 32) t += cs[c];
+        t = warp_sum_d(t);
+        const double tgt = v_draw * t;
+        double run = 0.0, bef = 0.0;
+        int found = nw - 1;
+        for (int c0 = 0; c0 < nw; c0 += 32) {
+            const int c = c0 + lane;
+            const double x = c < nw ? cs[c] : 0.0;
+            double incl = x;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            // (the last chunk takes whatever rounding leaves past the total)
+            const unsigned hit = __ballot_sync(0xffffffffu, c < nw && (c == nw - 1 || run + incl > tgt));
+            if (hit) {
+                const int l = __ffs(hit) - 1;
+                found = c0 + l;
+                bef = run + __shfl_sync(0xffffffffu, incl - x, l);
+                break;
+            }
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            s_z = t;
+            s_clo = found;
+            s_before = bef;
+        }
+    }
+    __syncthreads();
+    double Z = s_z;
+    int c_lo = 0, c_hi = nw;  // chunks to scan
     double before = 0.0;
     if (residual && !(Z > 0.0)) {  // empty residual: draw from p over the whole vocabulary
         residual = false;
         Z = 0.0;
-        for (int c = 0; c < p.n_chunks; ++c) {
+        for (int c = 0; c < nw; ++c) {
             int lo, hi;
-            chunk_range(p.vocab, p.n_chunks, c, lo, hi);
+            chunk_range(p.vocab, nw, c, lo, hi);
             double s = 0.0;
             for (int x = lo + tid; x < hi; x += kThreads)
                 s += draw_weight(zp, zq, dec.lse_p, 0.0, false, x);
             Z += block_sum_d(s, s_red);
         }
     } else {
-        // The chunk where the running total first exceeds v*Z.
-        const double target = (double)__ldg(p.v + off_t + dec.n) * Z;
-        double run = 0.0;
-        int c = 0;
-        for (; c < p.n_chunks - 1; ++c) {
-            if (run + cs[c] > target) break;
-            run += cs[c];
-        }
-        c_lo = c;
-        c_hi = c + 1;
-        before = run;
+        c_lo = s_clo;
+        c_hi = c_lo + 1;
+        before = s_before;
     }
     const double target = (double)__ldg(p.v + off_t + dec.n) * Z;
     if (tid == 0) s_found = -1;
@@ -350,7 +398,7 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const AcceptParam
     double run = before;
     for (int c = c_lo; c < c_hi; ++c) {
         int lo, hi;
-        chunk_range(p.vocab, p.n_chunks, c, lo, hi);
+        chunk_range(p.vocab, nw, c, lo, hi);
         for (int base = lo; base < hi; base += kThreads) {
             const int x = base + tid;
             const double w = x < hi ? draw_weight(zp, zq, dec.lse_p, dec.lse_q,
@@ -414,17 +462,25 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const AcceptParam
 
 }  // namespace
 
-size_t accept_workspace_bytes(int batch, int max_gamma, int vocab, int *n_chunks_out) {
+size_t accept_workspace_bytes(int batch, int max_gamma, int vocab, int *n_chunks_out,
+                              int *n_wchunks_out) {
     const int slots_t = batch * (max_gamma + 1);
     int n_chunks = (2 * 148 + slots_t - 1) / slots_t;
     const int max_chunks = (vocab + 2047) / 2048;
     if (n_chunks > max_chunks) n_chunks = max_chunks;
     if (n_chunks < 1) n_chunks = 1;
     if (n_chunks_out) *n_chunks_out = n_chunks;
+    // the drawing row of each sequence: about two CTAs per SM over the batch, at least 512
+    // tokens per chunk
+    int n_wchunks = (2 * 148 + batch - 1) / batch;
+    const int max_wchunks = (vocab + 511) / 512;
+    if (n_wchunks > max_wchunks) n_wchunks = max_wchunks;
+    if (n_wchunks < 1) n_wchunks = 1;
+    if (n_wchunks_out) *n_wchunks_out = n_wchunks;
     const size_t greedy = (size_t)slots_t * n_chunks * sizeof(unsigned long long);
     const size_t n_slots = (size_t)batch * (2 * max_gamma + 1);
     const size_t sample = n_slots * n_chunks * sizeof(float2) + (size_t)batch * sizeof(Decision) +
-                          (size_t)batch * n_chunks * sizeof(double);
+                          (size_t)batch * n_wchunks * sizeof(double);
     return greedy > sample ? greedy : sample;
 }
 
@@ -440,9 +496,10 @@ cudaError_t launch_accept_sample(const AcceptParams &p, cudaStream_t s) {
     dim3 g1(p.n_chunks, p.batch * (2 * p.max_gamma + 1));
     cudaError_t e = launch_pdl(accept_stats_kernel, g1, dim3(kThreads), 0, s, p);
     if (e != cudaSuccess) return e;
-    if ((e = launch_pdl(accept_decide_kernel, dim3(p.batch), dim3(32), 0, s, p)) != cudaSuccess)
+    if ((e = launch_pdl(accept_decide_kernel, dim3(p.batch), dim3(kDecideWarps * 32),
+                        (size_t)(3 * p.max_gamma + 1) * sizeof(double), s, p)) != cudaSuccess)
         return e;
-    dim3 g3(p.n_chunks, p.batch);
+    dim3 g3(p.n_wchunks, p.batch);
     if ((e = launch_pdl(accept_wsum_kernel, g3, dim3(kThreads), 0, s, p)) != cudaSuccess)
         return e;
     return launch_pdl(accept_draw_kernel, dim3(p.batch), dim3(kThreads), 0, s, p);

@@ -682,8 +682,8 @@ static sd_status accept_common(const float *tgt, const int32_t *draft_tok, const
         vocab < 1 || out_stride < max_gamma + 1 || (max_gamma > 0 && !draft_tok))
         return SD_ERR_INVALID_ARG;
     if ((long long)batch * (2 * max_gamma + 1) > 65535) return SD_ERR_UNSUPPORTED;
-    int n_chunks = 1;
-    const size_t need = accept_workspace_bytes(batch, max_gamma, vocab, &n_chunks);
+    int n_chunks = 1, n_wchunks = 1;
+    const size_t need = accept_workspace_bytes(batch, max_gamma, vocab, &n_chunks, &n_wchunks);
     if (need > workspace_bytes || !workspace) return SD_ERR_WORKSPACE;
     *p = AcceptParams{};
     p->tgt = tgt;
@@ -696,6 +696,7 @@ static sd_status accept_common(const float *tgt, const int32_t *draft_tok, const
     p->out_tok = out_tok;
     p->out_stride = out_stride;
     p->n_chunks = n_chunks;
+    p->n_wchunks = n_wchunks;
     p->ws = workspace;
     return SD_OK;
 }

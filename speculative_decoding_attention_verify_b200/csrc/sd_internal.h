@@ -146,11 +146,13 @@ struct AcceptParams {
     int32_t *out_tok;
     int out_stride;
     int32_t *near_boundary;
-    int n_chunks;  // vocabulary chunks per row
+    int n_chunks;   // vocabulary chunks per row (statistics, argmax)
+    int n_wchunks;  // vocabulary chunks of a sequence's drawing row (draw weights)
     void *ws;
     int32_t *dev_err;
 };
-size_t accept_workspace_bytes(int batch, int max_gamma, int vocab, int *n_chunks);
+size_t accept_workspace_bytes(int batch, int max_gamma, int vocab, int *n_chunks,
+                              int *n_wchunks = nullptr);
 cudaError_t launch_accept_greedy(const AcceptParams &p, cudaStream_t s);
 cudaError_t launch_accept_sample(const AcceptParams &p, cudaStream_t s);
 
