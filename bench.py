@@ -439,8 +439,8 @@ class Flusher:
 
 class Rotations:
     """Copies of a cycle's buffers for back-to-back timing of one call kind: consecutive calls
-    read different memory, so that no call finds its operands in L2 (SURVEY's protocol: rotate
-    over enough distinct buffers to exceed 4x the L2).  Rotation 0 is the cycle's own buffers;
+    read different memory, so that no call finds its operands in L2 (the rotation spans enough
+    distinct buffers to exceed 4x the L2).  Rotation 0 is the cycle's own buffers;
     the others are clones on the device (the values do not change the work)."""
 
     def __init__(self, cyc, n_kv, n_small):
