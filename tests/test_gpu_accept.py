@@ -96,7 +96,31 @@ SAMPLE_CASES = [(0, {}), (0, dict(batch=64)), (2, {}), (4, {}), (4, dict(batch=2
 
 @pytest.mark.parametrize("cfg,kw", SAMPLE_CASES)
 def test_sample_matches_oracle(cfg, kw):
-    aw = gen.make_accept_workload(cfg, **kw)
+    _check_sample(gen.make_accept_workload(cfg, **kw))
+
+
+def test_sample_long_and_empty_drafts():
+    """Draft lengths 24, 17 and 0 in one batch over vocab 152,064: the decision kernel's warps
+    take several of the 2 gamma + 1 rows each, one CTA draws over ~300 vocabulary chunks of its
+    own, and a sequence without drafts draws its bonus token from p."""
+    aw = gen.make_accept_workload(4, batch=3, gammas=[24, 17, 0])
+    _check_sample(aw)
+    _assert_greedy(aw, aw.draft_tokens_greedy)
+
+
+def test_sample_long_drafts_accept_all():
+    """Draft rows equal to their target rows and u just below 1: all 24 and 17 drafts are kept
+    and the bonus token is drawn from the last target row (as the oracle draws it)."""
+    aw = gen.make_accept_workload(4, batch=3, gammas=[24, 17, 0])
+    rows = np.split(aw.target_logits, np.cumsum(aw.gamma + 1)[:-1])
+    aw.draft_logits = np.concatenate([r[:g] for r, g in zip(rows, aw.gamma)]).copy()
+    aw.u = np.full(aw.u.shape, 0.999, np.float32)
+    n, out, _ = _sample(aw)
+    assert n.tolist() == [24, 17, 0]
+    _check_sample(aw)
+
+
+def _check_sample(aw):
     n, out, near = _sample(aw)
     rn, rout, am, dm = oracle.accept_sample(aw.target_logits, aw.draft_logits,
                                             aw.draft_tokens_sampled, aw.u, aw.v, aw.gamma,
@@ -108,7 +132,8 @@ def test_sample_matches_oracle(cfg, kw):
         margins = am[off:off + g]
         same = n[b] == rn[b] and out[b, :n[b] + 1].tolist() == rout[b, :rn[b] + 1].tolist()
         if not same:
-            near_decision = np.nanmin(np.abs(margins[:min(n[b], rn[b]) + 1])) < EPS
+            seen = np.abs(margins[:min(n[b], rn[b]) + 1])
+            near_decision = seen.size > 0 and np.nanmin(seen) < EPS
             near_draw = dm[b] < EPS
             assert near_decision or near_draw, f"sequence {b} differs away from any boundary"
             exceptions += 1
