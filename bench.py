@@ -264,6 +264,8 @@ class Cycle:
             self.gmax = int(aw.gamma.max())
             B = aw.batch
             self.ws_acc = mk(sd.sd_accept_workspace_size(B, self.gmax, aw.vocab))
+            # the greedy rule's own workspace: the two rules may run at the same time
+            self.ws_acc_g = mk(sd.sd_accept_workspace_size(B, self.gmax, aw.vocab))
             # the step's results, views of one buffer (one device-to-host copy brings them back)
             nt = B * (self.gmax + 1)
             self.results = torch.empty(3 * B + 2 * nt, dtype=torch.int32, device=device)
@@ -274,6 +276,8 @@ class Cycle:
             self.out_s = r[2 * B + nt:2 * B + 2 * nt].view(B, self.gmax + 1)
             self.near = r[2 * B + 2 * nt:3 * B + 2 * nt]
         self.calls = self._calls()
+        self.side = torch.cuda.Stream(device)
+        self.events = [torch.cuda.Event() for _ in range(4)]
         self.bytes = {}
         for kind, step, _ in self.calls:
             if kind == "stage":
@@ -316,7 +320,7 @@ class Cycle:
         if sp["accept"]:
             calls.append(("accept_greedy", 0, lambda s, b: sd.sd_accept_greedy(
                 self.acc_in[b]["tgt"], self.acc_in[b]["tok_g"], self.gam, self.gmax,
-                n_acc=self.n_acc_g, out_tok=self.out_g, workspace=self.ws_acc, stream=s)))
+                n_acc=self.n_acc_g, out_tok=self.out_g, workspace=self.ws_acc_g, stream=s)))
             calls.append(("accept_sample", 0, lambda s, b: sd.sd_accept_sample(
                 self.acc_in[b]["tgt"], self.acc_in[b]["drf"], self.acc_in[b]["tok_s"],
                 self.acc_in[b]["u"], self.acc_in[b]["v"], self.gam, self.gmax,
@@ -325,9 +329,42 @@ class Cycle:
         return calls
 
     def step(self, stream=None, buf=0, kinds=None):
+        """Issues the cycle's calls on `stream` (None: the current stream), with input set
+        `buf`.  With `kinds`, only those calls, in order on the one stream.
+
+        The whole cycle is two chains that only verification joins: Sparse-to-Dense's (top-K,
+        staging, the sparse draft steps) and Sparrow's (the HSR projection and text-anchored
+        attention of every draft step); after verification the greedy and the sampling rule
+        read the same logits, independently.  Sparrow's chain and the greedy rule run on a
+        second stream, forked from and joined back to `stream` through events (a CUDA graph
+        captured from the step holds the same edges), so one method's calls fill the SMs and
+        the HBM time the other's leave idle (a call's start, its last tiles).  Every chain
+        keeps its own order, and the results are those of the one-stream order."""
+        if kinds is not None:
+            for kind, _, fn in self.calls:
+                if kind in kinds:
+                    fn(stream, buf)
+            return
+        torch = self.torch
+        main = stream if stream is not None else torch.cuda.current_stream()
+        side, ev = self.side, self.events
+        ev[0].record(main)
+        side.wait_event(ev[0])
         for kind, _, fn in self.calls:
-            if kinds is None or kind in kinds:
-                fn(stream, buf)
+            if kind in ("hsr", "text_anchored"):
+                fn(side, buf)
+            elif kind == "verify":
+                ev[1].record(side)
+                main.wait_event(ev[1])
+                fn(main, buf)
+            elif kind == "accept_greedy":
+                ev[2].record(main)
+                side.wait_event(ev[2])
+                fn(side, buf)
+            else:
+                fn(main, buf)
+        ev[3].record(side)
+        main.wait_event(ev[3])
 
     def decode_step_calls(self):
         """Plain decoding of the draft steps' tokens: each token is one dense single-row
@@ -968,7 +1005,9 @@ def workload_config(cyc):
                 topk=w.topk if sp["topk"] else None,
                 hsr_weight_copies=len(cyc.W) if sp["hsr"] else 0,
                 vocab=cyc.aw.vocab if cyc.aw is not None else None,
-                parallelism="replicas (no data-path collective)")
+                parallelism="replicas (no data-path collective)",
+                streams=("2: Sparrow's chain (HSR, text-anchored) and the greedy rule on a "
+                         "second stream beside Sparse-to-Dense's chain, joined at verification"))
 
 
 def run_ours(args):
