@@ -504,6 +504,22 @@ topk_score_fast_kernel(const TopkParams p) {
         if (lane == 0) {
             const char *kbase = reinterpret_cast<const char *>(p.kv.k);
             constexpr int kMaxRuns = kFastTile / kPageSize + 1;
+            const bool paged = p.kv.page_size != 0;
+            // Paged caches: the block-table entries of the pages tile u touches (-1 past its
+            // rows), loaded together and one tile ahead, so that their latency passes while
+            // the lane waits for a free stage instead of once per page on the issue path.
+            const int32_t *btab = paged ? p.kv.block_table + (int64_t)b * p.kv.max_pages : nullptr;
+            auto tile_pages = [&](int u, int *ent) {
+                const int pos0 = cb + t_begin + u * kFastTile;
+                const int end = u < n_tiles ? cb + min(t_begin + (u + 1) * kFastTile, t_end) : 0;
+#pragma unroll
+                for (int i = 0; i < kMaxRuns; ++i) {
+                    const int pg = (pos0 >> 4) + i;
+                    ent[i] = pg * kPageSize < end ? __ldg(btab + pg) : -1;
+                }
+            };
+            int ent[kMaxRuns];
+            if (paged) tile_pages(0, ent);
             for (int u = 0; u < n_tiles; ++u) {
                 const int st = u % S;
                 if (u >= S && !mbar_wait(saddr(&s_empty[st]), ((u / S) - 1) & 1, abort_flag,
@@ -515,26 +531,33 @@ topk_score_fast_kernel(const TopkParams p) {
                 int rbeg[kMaxRuns], rlen[kMaxRuns];
                 int nruns = 0;
                 unsigned long long live = 0ull;
-                if (p.kv.page_size == 0) {  // every row of the tile, one run
+                if (!paged) {  // every row of the tile, one run
                     roff[0] = kv_row_offset(p.kv, b, g, cb + t0, p.dev_err);
                     rbeg[0] = 0;
                     rlen[0] = rows;
                     nruns = 1;
                     live = rows == 64 ? ~0ull : ((1ull << rows) - 1ull);
                 } else {  // a run per page (pages without a valid entry: no copy, not live)
-                    for (int r = 0; r < rows;) {
-                        const int pos = cb + t0 + r;
-                        const int len = min(rows - r, kPageSize - (pos & (kPageSize - 1)));
-                        const int64_t off = kv_row_offset(p.kv, b, g, pos, p.dev_err);
-                        if (off >= 0) {
-                            roff[nruns] = off;
+                    const int pos0 = cb + t0;
+#pragma unroll
+                    for (int i = 0; i < kMaxRuns; ++i) {
+                        const int pg = (pos0 >> 4) + i;
+                        const int r = max(pg * kPageSize - pos0, 0);  // the page's first row
+                        if (r >= rows) continue;
+                        const int len = min(rows - r, kPageSize - ((pos0 + r) & (kPageSize - 1)));
+                        const int e = ent[i];
+                        if (e >= 0 && e < p.kv.num_pages) {
+                            roff[nruns] = (((int64_t)e * p.kv.h_kv + g) * kPageSize +
+                                           ((pos0 + r) & (kPageSize - 1))) * p.kv.head_dim;
                             rbeg[nruns] = r;
                             rlen[nruns] = len;
                             ++nruns;
                             live |= ((len == 64 ? ~0ull : ((1ull << len) - 1ull)) << r);
+                        } else {
+                            set_dev_err(p.dev_err, SD_DEVERR_PAGE);
                         }
-                        r += len;
                     }
+                    tile_pages(u + 1, ent);  // (the next tile's entries, while this one copies)
                 }
                 uint32_t bytes = 0;
                 for (int i = 0; i < nruns; ++i) bytes += (uint32_t)(rlen[i] * ROWB);
