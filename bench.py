@@ -1284,14 +1284,16 @@ CASES = ("verify", "sparse", "sparse_staged", "stage", "text_anchored", "topk", 
 
 
 def run_case(args):
-    """One call kind of the default workload on a reduced layer count (``--layers``), repeated
-    ``--steps`` times after ``--warmup``; prints its device time.  Used for ncu captures of one
-    kernel on a small case."""
+    """One call kind of the default workload on a reduced layer count (``--layers``), or of
+    workload ``--config`` as it is, repeated ``--steps`` times after ``--warmup``; prints its
+    device time.  Used for ncu captures of one kernel on a small case."""
     import torch
     from speculative_decoding_attention_verify_b200 import device as dev
     from speculative_decoding_attention_verify_b200 import inputs as gen
     from speculative_decoding_attention_verify_b200 import sdattn as sd
-    w = gen.make_attn_workload(DEFAULT_CONFIG, layers=args.layers)
+    # the default workload on --layers layers, or another configuration as it is (--config)
+    w = gen.make_attn_workload(DEFAULT_CONFIG, layers=args.layers) \
+        if args.config == DEFAULT_CONFIG else gen.make_attn_workload(args.config)
     L, g = w.n_seq, int(w.gamma[0])
     k = dev.tensor(w.k, w.dtype)
     v = dev.tensor(w.v, w.dtype)
@@ -1360,7 +1362,7 @@ def run_case(args):
         call()
     e1.record()
     torch.cuda.synchronize()
-    print(json.dumps({"case": args.case, "layers": args.layers,
+    print(json.dumps({"case": args.case, "config": args.config, "layers": w.n_seq,
                       "ms_per_call": round(e0.elapsed_time(e1) / args.steps, 4)}), flush=True)
 
 
