@@ -450,6 +450,78 @@ constexpr int kFastThreads = (kFastWarps + 1) * 32;           // + the copy warp
 // ring depth: about 96 KB of rows per CTA (two CTAs per SM)
 constexpr int fast_stages(int tile_bytes) { return tile_bytes <= 16384 ? 6 : 3; }
 
+// Parts of the fp32 scoring.  Every part holds `chunk` candidates of one (sequence, KV head)
+// unit, the same count for every unit, so a batch of ragged sequences gives its long sequences
+// more parts instead of longer ones: chunk = the batch's candidates over units * n_splits parts
+// (the host's split count for this batch size), at least four 128-candidate spans and at least
+// max_cand / part_stride (no unit needs more parts than its part slots).  A unit of n
+// candidates takes max(1, ceil(n / chunk)) parts; their sum is at most units * (n_splits + 1),
+// the launch's CTA count.  Warp-collective: every lane returns chunk.
+constexpr long long kMinPart = 4 * 128;
+__device__ long long fast_part_chunk(const TopkParams &p, int lane) {
+    long long tot = 0;
+    for (int bb = lane; bb < p.batch; bb += 32) {
+        int c0, nn;
+        cand_range(p, bb, c0, nn, false);
+        tot += nn;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    const long long units = (long long)p.batch * p.kv.h_kv;
+    const long long parts = units * p.n_splits;
+    long long chunk = (tot * p.kv.h_kv + parts - 1) / parts;
+    chunk = max(chunk, kMinPart);
+    chunk = max(chunk, ((long long)p.max_cand + p.part_stride - 1) / p.part_stride);
+    return chunk;
+}
+
+__device__ __forceinline__ int fast_parts_of(long long n, long long chunk) {
+    return (int)max(1LL, (n + chunk - 1) / chunk);
+}
+
+// The part CTA x scores: m[0] = sequence (-1: x is past the batch's parts), m[1] = KV head,
+// m[2] = part, m[3] = chunk.  Units in (sequence, KV head) order, each unit's parts together.
+// Warp-collective; lane 0 writes m.
+__device__ void fast_part_of_cta(const TopkParams &p, long long x, int lane, long long *m) {
+    const long long chunk = fast_part_chunk(p, lane);
+    long long base = 0;
+    int fb = -1, fg = 0, fs = 0;
+    for (int b0 = 0; b0 < p.batch; b0 += 32) {
+        const int bb = b0 + lane;
+        int parts = 0;
+        if (bb < p.batch) {
+            int c0, nn;
+            cand_range(p, bb, c0, nn, false);
+            parts = fast_parts_of(nn, chunk);
+        }
+        const long long cnt = (long long)parts * p.kv.h_kv;  // CTAs of sequence bb
+        long long inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        const long long lo = base + inc - cnt;
+        const unsigned hit = __ballot_sync(0xffffffffu, bb < p.batch && x >= lo && x < lo + cnt);
+        if (hit) {
+            const int src = __ffs(hit) - 1;
+            const long long r = x - __shfl_sync(0xffffffffu, lo, src);
+            const int np = __shfl_sync(0xffffffffu, parts, src);
+            fb = b0 + src;
+            fg = (int)(r / np);
+            fs = (int)(r % np);
+            break;
+        }
+        base += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) {
+        m[0] = fb;
+        m[1] = fg;
+        m[2] = fs;
+        m[3] = chunk;
+    }
+}
+
 template <bool BF16, int D>
 __global__ void __launch_bounds__(kFastThreads, kScoreCtasPerSm)
 topk_score_fast_kernel(const TopkParams p) {
@@ -473,15 +545,20 @@ topk_score_fast_kernel(const TopkParams p) {
     __shared__ float s_bmax[kFastWarps];
     __shared__ int s_bad[kFastWarps];
     __shared__ int s_abort;
+    __shared__ long long s_part[4];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = blockIdx.z, g = blockIdx.y, split = blockIdx.x;
+    if (warp == 0) fast_part_of_cta(p, blockIdx.x, lane, s_part);
+    __syncthreads();
+    if (s_part[0] < 0) return;  // (past the batch's parts)
+    const int b = (int)s_part[0], g = (int)s_part[1], split = (int)s_part[2];
+    const long long chunk = s_part[3];
     const int last = __ldg(p.q_start + b + 1) - 1;
     if (last < __ldg(p.q_start + b)) {  // (the select kernel writes -1 without reading more)
         if (tid == 0 && split == 0) set_dev_err(p.dev_err, SD_DEVERR_SHAPE);
         return;
     }
     int cb, n;
-    cand_range(p, b, cb, n);
+    cand_range(p, b, cb, n, tid == 0 && split == 0);
     if (tid == 0) {
         for (int st = 0; st < S; ++st) {
             mbar_init(saddr(&s_full[st]), 1);
@@ -493,8 +570,8 @@ topk_score_fast_kernel(const TopkParams p) {
     __syncthreads();
     volatile int *abort_flag = &s_abort;
     const int unit = b * p.kv.h_kv + g;
-    const int t_begin = (int)((int64_t)n * split / p.n_splits);
-    const int t_end = (int)((int64_t)n * (split + 1) / p.n_splits);
+    const int t_begin = (int)min((long long)n, split * chunk);
+    const int t_end = (int)min((long long)n, (split + 1) * chunk);
     const int n_tiles = (t_end - t_begin + kFastTile - 1) / kFastTile;
     float bmax = 0.f;
     bool bad = false;
@@ -791,7 +868,8 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_fast_kernel(const 
     if (warp == 0) {
         float m = 0.f;
         uint32_t f = 0u;
-        for (int i = lane; i < p.n_splits; i += 32) {
+        const int n_parts = fast_parts_of(n, fast_part_chunk(p, lane));  // (the scoring's)
+        for (int i = lane; i < n_parts; i += 32) {
             const uint2 v = p.parts[(int64_t)unit * p.part_stride + i];
             m = fmaxf(m, __uint_as_float(v.x));
             f |= v.y;
@@ -1004,8 +1082,11 @@ cudaError_t launch_fast_t(const TopkParams &p, cudaStream_t s) {
     const int dyn = fast_stages(tile) * tile;
     cudaError_t e = set_max_dynamic_smem<topk_score_fast_kernel<BF16, D>>(dyn);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(topk_score_fast_kernel<BF16, D>, dim3(p.n_splits, p.kv.h_kv, p.batch),
-                   dim3(kFastThreads), dyn, s, p);
+    // one CTA per part, enough for every partition of the batch (fast_part_chunk)
+    const long long ctas = (long long)p.batch * p.kv.h_kv * (p.n_splits + 1);
+    if (ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    e = launch_pdl(topk_score_fast_kernel<BF16, D>, dim3((unsigned)ctas), dim3(kFastThreads), dyn,
+                   s, p);
     if (e != cudaSuccess) return e;
     const size_t sdyn = p.max_cand <= kSmemKeys32 ? (size_t)p.max_cand * sizeof(uint32_t) : 0;
     e = set_max_dynamic_smem<topk_select_fast_kernel<BF16, D>>(

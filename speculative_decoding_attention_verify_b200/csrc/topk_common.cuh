@@ -15,8 +15,9 @@ __device__ __forceinline__ unsigned long long score_key(double x) {
 }
 
 // Clamp the candidate range of sequence b to [0, kv_len) and to max_cand entries (a range
-// outside those bounds sets SD_DEVERR_INDEX).
-__device__ __forceinline__ void cand_range(const TopkParams &p, int b, int &cb, int &n) {
+// outside those bounds sets SD_DEVERR_INDEX when `report`).
+__device__ __forceinline__ void cand_range(const TopkParams &p, int b, int &cb, int &n,
+                                           bool report) {
     const int kv_len = __ldg(p.kv.kv_len + b);
     int lo = __ldg(p.cand_begin + b), hi = __ldg(p.cand_end + b);
     const bool bad = lo < 0 || hi > kv_len || hi - lo > p.max_cand ||
@@ -27,7 +28,12 @@ __device__ __forceinline__ void cand_range(const TopkParams &p, int b, int &cb, 
     hi = min(hi, lo + p.max_cand);
     cb = lo;
     n = max(0, hi - lo);
-    if (bad && threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
+    if (bad && report) set_dev_err(p.dev_err, SD_DEVERR_INDEX);
+}
+
+// The same, reported by thread 0 of the CTAs with blockIdx.x == 0.
+__device__ __forceinline__ void cand_range(const TopkParams &p, int b, int &cb, int &n) {
+    cand_range(p, b, cb, n, threadIdx.x == 0 && blockIdx.x == 0);
 }
 
 }  // namespace sd
