@@ -21,6 +21,10 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I" + INCLUDE, "-I" + CSRC]
+# SD_NVTX=1: every compute entry point opens an NVTX range named after itself (for profilers;
+# a no-op without one).  Objects do not record the flag: rebuild with force=True on a change.
+if os.environ.get("SD_NVTX", "") not in ("", "0"):
+    FLAGS = FLAGS + ["-DSD_NVTX"]
 
 
 def _headers():

@@ -441,6 +441,7 @@ sd_status sd_draft_layer(const sd_draft_layer_desc *w, const void *emb, const vo
                          int32_t n_rows, const sd_kv_desc *cache, int32_t max_kv_len,
                          int32_t window, void *y, void *workspace, size_t workspace_bytes,
                          int32_t *dev_err, void *stream) {
+    SD_RANGE("sd_draft_layer");
     if (!emb || !hid || !y || !cache || !layer_desc_ok(w, n_rows) || max_kv_len < n_rows ||
         window < 1)
         return SD_ERR_INVALID_ARG;

@@ -404,6 +404,7 @@ sd_status sd_attention_plan(sd_attn_kind kind, const sd_q_desc *q, const sd_kv_d
 sd_status sd_verify_attention(const sd_q_desc *q, const void *q_data, const sd_kv_desc *kv,
                               int32_t batch, void *out, void *workspace, size_t workspace_bytes,
                               int32_t *dev_err, void *stream) {
+    SD_RANGE("sd_verify_attention");
     AttnPlan plan;
     if (!q_data || !out) return SD_ERR_INVALID_ARG;
     sd_status st = check_attention(SD_ATTN_VERIFY, q, kv, batch, q ? q->max_kv_len : 0, &plan);
@@ -419,6 +420,7 @@ sd_status sd_text_anchored_attention(const sd_q_desc *q, const void *q_data,
                                      const int32_t *window, int32_t max_window, void *out,
                                      void *workspace, size_t workspace_bytes, int32_t *dev_err,
                                      void *stream) {
+    SD_RANGE("sd_text_anchored_attention");
     if (!q_data || !out || !vis_begin || !vis_end || !window || max_window < 1)
         return SD_ERR_INVALID_ARG;
     AttnPlan plan;
@@ -457,6 +459,7 @@ sd_status sd_sparse_attention(const sd_q_desc *q, const void *q_data, const sd_k
                               const int32_t *tail_begin, int32_t max_tail, void *out,
                               void *workspace, size_t workspace_bytes, int32_t *dev_err,
                               void *stream) {
+    SD_RANGE("sd_sparse_attention");
     if (!q_data || !out || !tail_begin || k < 0 || (k > 0 && !idx) || max_tail < 0 ||
         k > (1 << 16))
         return SD_ERR_INVALID_ARG;
@@ -497,6 +500,7 @@ sd_status sd_sparse_selection_size(const sd_kv_desc *kv, int32_t batch, int32_t 
 sd_status sd_sparse_stage(const sd_kv_desc *kv, int32_t batch, const int32_t *idx, int32_t k,
                           const int32_t *tail_begin, void *selection, size_t selection_bytes,
                           int32_t *dev_err, void *stream) {
+    SD_RANGE("sd_sparse_stage");
     if (!tail_begin || k < 0 || (k > 0 && !idx) || k > (1 << 16) || batch < 1 || batch > 65535)
         return SD_ERR_INVALID_ARG;
     if (!kv_desc_ok(kv, batch)) return SD_ERR_INVALID_ARG;
@@ -522,6 +526,7 @@ sd_status sd_sparse_attention_staged(const sd_q_desc *q, const void *q_data,
                                      int32_t k, const int32_t *tail_begin, int32_t max_tail,
                                      void *out, void *workspace, size_t workspace_bytes,
                                      int32_t *dev_err, void *stream) {
+    SD_RANGE("sd_sparse_attention_staged");
     if (!q || !q_data || !out || !tail_begin || !selection || k < 0 || max_tail < 0 ||
         k > (1 << 16))
         return SD_ERR_INVALID_ARG;
@@ -560,6 +565,7 @@ sd_status sd_topk_select(const sd_q_desc *q, const void *q_data, const sd_kv_des
                          int32_t batch, const int32_t *cand_begin, const int32_t *cand_end,
                          int32_t max_cand, int32_t k, int32_t *idx_out, void *workspace,
                          size_t workspace_bytes, int32_t *dev_err, void *stream) {
+    SD_RANGE("sd_topk_select");
     return sd_topk_select_scored(SD_TOPK_LAST_QUERY, q, q_data, kv, batch, cand_begin, cand_end,
                                  max_cand, k, idx_out, nullptr, workspace, workspace_bytes,
                                  dev_err, stream);
@@ -585,6 +591,7 @@ sd_status sd_topk_select_scored(sd_topk_score mode, const sd_q_desc *q, const vo
                                 const int32_t *cand_end, int32_t max_cand, int32_t k,
                                 int32_t *idx_out, double *scores_out, void *workspace,
                                 size_t workspace_bytes, int32_t *dev_err, void *stream) {
+    SD_RANGE("sd_topk_select_scored");
     if (mode != SD_TOPK_LAST_QUERY && mode != SD_TOPK_MEAN_TEXT_ATTENTION)
         return SD_ERR_INVALID_ARG;
     if (!q || !q_data || !cand_begin || !cand_end || !idx_out || k < 1 || max_cand < 0 ||
@@ -656,6 +663,7 @@ sd_status sd_topk_select_scored(sd_topk_score mode, const sd_q_desc *q, const vo
 
 sd_status sd_hsr_project(const void *emb, const void *hid, int32_t n_rows, int32_t d_model,
                          const void *weight, const void *bias, void *y, void *stream) {
+    SD_RANGE("sd_hsr_project");
     if (!emb || !hid || !weight || !y || n_rows < 1 || n_rows > 16 || d_model < 16 ||
         d_model % 16 != 0 || d_model > (1 << 20))
         return SD_ERR_INVALID_ARG;
@@ -705,6 +713,7 @@ sd_status sd_accept_greedy(const float *tgt_logits, const int32_t *draft_tok,
                            const int32_t *gamma, int32_t batch, int32_t max_gamma, int32_t vocab,
                            int32_t *n_acc, int32_t *out_tok, int32_t out_stride, void *workspace,
                            size_t workspace_bytes, int32_t *dev_err, void *stream) {
+    SD_RANGE("sd_accept_greedy");
     AcceptParams p;
     sd_status st = accept_common(tgt_logits, draft_tok, gamma, batch, max_gamma, vocab, n_acc,
                                  out_tok, out_stride, workspace, workspace_bytes, &p);
@@ -719,6 +728,7 @@ sd_status sd_accept_sample(const float *tgt_logits, const float *draft_logits,
                            int32_t *n_acc, int32_t *out_tok, int32_t out_stride,
                            int32_t *near_boundary, void *workspace, size_t workspace_bytes,
                            int32_t *dev_err, void *stream) {
+    SD_RANGE("sd_accept_sample");
     if (!v || (max_gamma > 0 && (!draft_logits || !u))) return SD_ERR_INVALID_ARG;
     AcceptParams p;
     sd_status st = accept_common(tgt_logits, draft_tok, gamma, batch, max_gamma, vocab, n_acc,

@@ -8,6 +8,26 @@
 #include "sd_attn.h"
 #include "sd_common.cuh"
 
+// Profiling ranges.  Built with -DSD_NVTX (SD_NVTX=1 in the environment of the package's
+// build), every compute entry point opens an NVTX range named after itself for the duration
+// of the host call (validation, planning and the launches; the GPU work itself is timed by
+// the profiler).  NVTX 3 is header-only and does nothing unless a tool is attached.  The
+// default build defines the macro away.
+#ifdef SD_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace sd {
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+}  // namespace sd
+#define SD_RANGE(name) ::sd::NvtxRange sd_nvtx_range_(name)
+#else
+#define SD_RANGE(name) ((void)0)
+#endif
+
 namespace sd {
 
 // Parameters of one attention launch (all three kinds).

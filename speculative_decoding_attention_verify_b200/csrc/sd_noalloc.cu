@@ -67,6 +67,7 @@ extern "C" {
 sd_status sd_verify_attention_noalloc(const sd_q_desc *q, const void *q_data,
                                       const sd_kv_desc *kv, int32_t batch, void *out,
                                       int32_t *dev_err, void *stream) {
+    SD_RANGE("sd_verify_attention_noalloc");
     sd::AttnPlan plan;
     sd_status st = sd::verify_plan(q, q_data, kv, batch, out, &plan);
     if (st != SD_OK) return st;
