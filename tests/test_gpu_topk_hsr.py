@@ -58,6 +58,16 @@ def test_topk_matches_oracle_exactly(cfg, kw, k):
     assert near == 0
 
 
+def test_topk_ragged_batch_beyond_one_warp():
+    """40 sequences, more than one warp's worth of the device's scan over the sequences' part
+    counts, with candidate counts from 200 to 1,448: the scorer's parts follow each sequence's
+    own count (one to three parts of 512), and the select reads exactly those parts."""
+    w = gen.make_attn_workload(4, l_vis=1500, l_txt=100, batch=40)
+    ce = (200 + 32 * np.arange(w.n_seq)).astype(np.int32)
+    got, ref, gap = _run_topk(w, 128, cand_end=ce)
+    assert _assert_same_sets(got, ref, gap) == 0
+
+
 def test_topk_c3_full_launch_sampled_layers():
     w = gen.make_attn_workload(3)
     kv = dev.kv_cache(w)
